@@ -1,0 +1,664 @@
+// pw_api.cu -- host side of the C ABI (include/pw.h): argument checks, the
+// per-block page table, the asynchronous bitwidth switch, workspace and the
+// launch sequence of one forward.
+//
+// PagedWeight (legiblepapers summary, "Summary & Methodology Analysis"): the
+// bit-plane and LUT buffers are GPU-resident pages reloaded or offloaded
+// asynchronously to hide latency; (arxivlens abstract) asynchronous page
+// movement overlaps with serving.  Here a bitwidth change is a page move on a
+// side stream that the forward after next waits for (see pw_set_block_bits).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "pw_internal.h"
+#include "tc.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+pw_status_t fail(pw_status_t st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+pw_status_t fail(pw_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+#define PW_CUDA(call)                                                                  \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return fail(PW_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));        \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library needs no link-time dependency on libcuda.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// The tensor-core path stages planes with 3-D TMA tiles (words x rows x
+// plane), whose row pitch must be a multiple of 16 bytes, and reads its
+// activation rows with 16-byte vectors.
+bool tc_shape_ok(int cols) {
+  const int words = (cols + 31) / 32;
+  return words % 4 == 0 && cols % 8 == 0;
+}
+
+pw_status_t make_plane_map(CUtensorMap* m, const uint32_t* planes, int n_planes, int rows,
+                           int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int words = (cols + 31) / 32;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(n_planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(words) * 4,
+                           static_cast<cuuint64_t>(words) * 4 * rows};
+  cuuint32_t box[3] = {8, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(planes), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return PW_OK;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  return v ? atoi(v) : dflt;
+}
+
+}  // namespace
+
+struct pw_moe {
+  pw_moe_config_t cfg{};
+  int n_blocks = 0, G = 0, device = 0, n_sm = 0;
+  struct Blk {
+    int rows, cols;
+    uint32_t* d_planes;
+    uint16_t* d_lut[2];
+    const uint32_t* h_planes;
+    const uint16_t* h_lut[PW_MAX_BITS + 1];
+    int bits, slot;            // active bitwidth and LUT slot
+    int pend_bits;             // 0 = none
+    long long pend_due;        // forward index from which the change applies
+    cudaEvent_t ready;
+  };
+  std::vector<Blk> blk;
+  long long n_forwards = 0;
+  cudaEvent_t fwd_done = nullptr;
+  bool any_forward = false;
+  // workspace
+  pw::RouteWorkspace ws{};
+  float* gu = nullptr;
+  float* ysorted = nullptr;
+  int* err = nullptr;
+  CUtensorMap* d_tmaps = nullptr;
+  uint16_t* stage_x = nullptr;
+  uint16_t* stage_y = nullptr;
+  int P_max = 0, gu_stride = 0, max_split = 8, last_T = 0;
+  bool tc_gu = false, tc_down = false;
+  void* ws_base = nullptr;
+  // per-launch timing (pw_profile_*): 5 events per forward bracket 4 launches
+  bool profiling = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<std::vector<cudaEvent_t>> ev_pending;
+};
+
+namespace {
+
+int block_rows(const pw_moe_config_t& c, int id) {
+  const int e = id / 3, proj = id % 3;
+  const int F = (e == c.n_experts) ? c.shared_ffn : c.ffn;
+  return proj < 2 ? F : c.hidden;
+}
+int block_cols(const pw_moe_config_t& c, int id) {
+  const int e = id / 3, proj = id % 3;
+  const int F = (e == c.n_experts) ? c.shared_ffn : c.ffn;
+  return proj < 2 ? c.hidden : F;
+}
+
+void free_all(pw_moe* h) {
+  if (!h) return;
+  for (auto& v : h->ev_pending)
+    for (auto e : v) cudaEventDestroy(e);
+  for (auto e : h->ev_pool) cudaEventDestroy(e);
+  for (auto& b : h->blk)
+    if (b.ready) cudaEventDestroy(b.ready);
+  if (h->fwd_done) cudaEventDestroy(h->fwd_done);
+  if (h->ws_base) cudaFree(h->ws_base);
+  delete h;
+}
+
+int down_splits(const pw_moe* h, int T) {
+  const pw_moe_config_t& c = h->cfg;
+  const int forced = env_int("PW_DOWN_SPLIT", 0);
+  if (forced > 0) return forced < h->max_split ? forced : h->max_split;
+  const int row_tiles = (c.hidden + 127) / 128;
+  int groups = T * c.top_k < c.n_experts ? T * c.top_k : c.n_experts;
+  if (c.shared_ffn > 0) groups += 1;
+  const int items = row_tiles * groups;
+  int ns = (4 * h->n_sm + items - 1) / items;
+  const int stages = ((c.ffn + 31) / 32 + 7) / 8;
+  if (ns > stages) ns = stages;
+  if (ns > h->max_split) ns = h->max_split;
+  if (ns < 1) ns = 1;
+  return ns;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pw_abi_version(void) { return PW_ABI_VERSION; }
+const char* pw_last_error(void) { return g_err.c_str(); }
+
+pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blocks,
+                          int32_t n_blocks, pw_moe_t** out) {
+  if (!cfg || !blocks || !out) return fail(PW_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  const pw_moe_config_t c = *cfg;
+  if (c.hidden < 8 || c.hidden % 8) return fail(PW_ERR_INVALID_ARG, "hidden must be a positive multiple of 8");
+  if (c.ffn < 1) return fail(PW_ERR_INVALID_ARG, "ffn must be positive");
+  if (c.n_experts < 1 || c.n_experts > PW_MAX_EXPERTS)
+    return fail(PW_ERR_INVALID_ARG, "n_experts must be in [1, %d]", PW_MAX_EXPERTS);
+  if (c.top_k < 1 || c.top_k > c.n_experts || c.top_k > PW_MAX_TOPK)
+    return fail(PW_ERR_INVALID_ARG, "top_k must be in [1, min(E, %d)]", PW_MAX_TOPK);
+  if (c.shared_ffn < 0) return fail(PW_ERR_INVALID_ARG, "shared_ffn must be >= 0");
+  if (c.n_max < 1 || c.n_max > PW_MAX_BITS) return fail(PW_ERR_INVALID_ARG, "n_max must be in [1, 8]");
+  if (c.max_tokens < 1) return fail(PW_ERR_INVALID_ARG, "max_tokens must be >= 1");
+  const int want_blocks = 3 * (c.n_experts + (c.shared_ffn > 0 ? 1 : 0));
+  if (n_blocks != want_blocks)
+    return fail(PW_ERR_INVALID_ARG, "expected %d blocks, got %d", want_blocks, n_blocks);
+  for (int i = 0; i < n_blocks; ++i) {
+    const pw_block_desc_t& b = blocks[i];
+    if (!b.d_planes || !b.d_lut[0] || !b.d_lut[1])
+      return fail(PW_ERR_INVALID_ARG, "block %d: null device buffer", i);
+    if (!aligned16(b.d_planes) || !aligned16(b.d_lut[0]) || !aligned16(b.d_lut[1]))
+      return fail(PW_ERR_INVALID_ARG, "block %d: device buffers must be 16-byte aligned", i);
+    if (b.bits < 1 || b.bits > c.n_max)
+      return fail(PW_ERR_INVALID_ARG, "block %d: bits %d outside [1, n_max]", i, b.bits);
+  }
+
+  pw_moe* h = new (std::nothrow) pw_moe();
+  if (!h) return fail(PW_ERR_OOM, "host allocation failed");
+  h->cfg = c;
+  h->n_blocks = n_blocks;
+  h->G = c.n_experts + (c.shared_ffn > 0 ? 1 : 0);
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    free_all(h);
+    return fail(PW_ERR_CUDA, "no CUDA device");
+  }
+  h->blk.resize(n_blocks);
+  for (int i = 0; i < n_blocks; ++i) {
+    auto& d = h->blk[i];
+    const pw_block_desc_t& b = blocks[i];
+    d.rows = block_rows(c, i);
+    d.cols = block_cols(c, i);
+    d.d_planes = b.d_planes;
+    d.d_lut[0] = b.d_lut[0];
+    d.d_lut[1] = b.d_lut[1];
+    d.h_planes = b.h_planes;
+    for (int k = 0; k <= PW_MAX_BITS; ++k) d.h_lut[k] = b.h_lut[k];
+    d.bits = b.bits;
+    d.slot = 0;
+    d.pend_bits = 0;
+    d.pend_due = 0;
+    d.ready = nullptr;
+    if (cudaEventCreateWithFlags(&d.ready, cudaEventDisableTiming) != cudaSuccess) {
+      free_all(h);
+      return fail(PW_ERR_CUDA, "cudaEventCreate failed");
+    }
+  }
+  if (cudaEventCreateWithFlags(&h->fwd_done, cudaEventDisableTiming) != cudaSuccess) {
+    free_all(h);
+    return fail(PW_ERR_CUDA, "cudaEventCreate failed");
+  }
+
+  // workspace, one allocation
+  const int T = c.max_tokens, E = c.n_experts, k = c.top_k;
+  const int S = c.shared_ffn;
+  h->P_max = T * k + (S > 0 ? T : 0);
+  const int Fmax = c.ffn > S ? c.ffn : S;
+  h->gu_stride = 2 * Fmax;
+  h->tc_gu = tc_shape_ok(c.hidden) && env_int("PW_FORCE_SIMPLE", 0) == 0;
+  h->tc_down = tc_shape_ok(c.ffn) && (S == 0 || tc_shape_ok(S)) && env_int("PW_FORCE_SIMPLE", 0) == 0;
+  auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
+  size_t off = 0;
+  const size_t o_logits = off; off += al(sizeof(float) * T * E);
+  const size_t o_tki = off; off += al(sizeof(int32_t) * T * k);
+  const size_t o_tkw = off; off += al(sizeof(float) * T * k);
+  const size_t o_off = off; off += al(sizeof(int32_t) * (h->G + 1));
+  const size_t o_st = off; off += al(sizeof(int32_t) * h->P_max);
+  const size_t o_sw = off; off += al(sizeof(float) * h->P_max);
+  const size_t o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
+  const size_t o_tk = off; off += al(sizeof(uint32_t) * 4);
+  const size_t o_err = off; off += al(sizeof(int) * 4);
+  const size_t o_tm = off; off += al(sizeof(CUtensorMap) * n_blocks);
+  const size_t o_gu = off; off += al(sizeof(float) * size_t(h->P_max) * h->gu_stride);
+  const size_t o_ys = off; off += al(sizeof(float) * size_t(h->max_split) * h->P_max * c.hidden);
+  const size_t o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
+  const size_t o_sy = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
+  if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
+    free_all(h);
+    return fail(PW_ERR_OOM, "workspace allocation of %zu bytes failed", off);
+  }
+  char* w = static_cast<char*>(h->ws_base);
+  h->ws.logits = reinterpret_cast<float*>(w + o_logits);
+  h->ws.topk_idx = reinterpret_cast<int32_t*>(w + o_tki);
+  h->ws.topk_w = reinterpret_cast<float*>(w + o_tkw);
+  h->ws.offsets = reinterpret_cast<int32_t*>(w + o_off);
+  h->ws.slot_token = reinterpret_cast<int32_t*>(w + o_st);
+  h->ws.slot_w = reinterpret_cast<float*>(w + o_sw);
+  h->ws.token_pos = reinterpret_cast<int32_t*>(w + o_tp);
+  h->ws.ticket = reinterpret_cast<uint32_t*>(w + o_tk);
+  h->err = reinterpret_cast<int*>(w + o_err);
+  h->d_tmaps = reinterpret_cast<CUtensorMap*>(w + o_tm);
+  h->gu = reinterpret_cast<float*>(w + o_gu);
+  h->ysorted = reinterpret_cast<float*>(w + o_ys);
+  h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
+  h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
+  if (cudaMemset(w + o_tk, 0, al(sizeof(uint32_t) * 4) + al(sizeof(int) * 4)) != cudaSuccess) {
+    free_all(h);
+    return fail(PW_ERR_CUDA, "cudaMemset failed");
+  }
+  // plane tensor maps for the tensor-core passes
+  if (h->tc_gu || h->tc_down) {
+    std::vector<CUtensorMap> maps(n_blocks);
+    for (int i = 0; i < n_blocks; ++i) {
+      std::memset(&maps[i], 0, sizeof(CUtensorMap));
+      if (!tc_shape_ok(h->blk[i].cols)) continue;
+      pw_status_t st = make_plane_map(&maps[i], h->blk[i].d_planes, c.n_max, h->blk[i].rows,
+                                      h->blk[i].cols);
+      if (st != PW_OK) {
+        free_all(h);
+        return st;
+      }
+    }
+    if (cudaMemcpy(h->d_tmaps, maps.data(), sizeof(CUtensorMap) * n_blocks,
+                   cudaMemcpyHostToDevice) != cudaSuccess) {
+      free_all(h);
+      return fail(PW_ERR_CUDA, "tensor map upload failed");
+    }
+  }
+  *out = h;
+  return PW_OK;
+}
+
+pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
+                              pw_stream_t side_stream) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  if (block_id < 0 || block_id >= h->n_blocks)
+    return fail(PW_ERR_INVALID_ARG, "block id %d out of range", block_id);
+  auto& b = h->blk[block_id];
+  if (new_bits < 1 || new_bits > h->cfg.n_max)
+    return fail(PW_ERR_INVALID_ARG, "bits %d outside [1, n_max]", new_bits);
+  if (b.pend_bits) return fail(PW_ERR_STATE, "block %d: a change to %d bits is still pending", block_id, b.pend_bits);
+  if (new_bits == b.bits) return PW_OK;
+  if (!b.h_lut[new_bits])
+    return fail(PW_ERR_INVALID_ARG, "block %d: no host LUT for %d bits", block_id, new_bits);
+  if (new_bits > b.bits && !b.h_planes)
+    return fail(PW_ERR_INVALID_ARG, "block %d: raising bits needs the host planes", block_id);
+  cudaStream_t s = static_cast<cudaStream_t>(side_stream);
+  if (h->any_forward) PW_CUDA(cudaStreamWaitEvent(s, h->fwd_done, 0));
+  const size_t plane_elems = static_cast<size_t>(b.rows) * ((b.cols + 31) / 32);
+  if (new_bits > b.bits) {
+    PW_CUDA(cudaMemcpyAsync(b.d_planes + b.bits * plane_elems, b.h_planes + b.bits * plane_elems,
+                            sizeof(uint32_t) * plane_elems * (new_bits - b.bits),
+                            cudaMemcpyHostToDevice, s));
+  }
+  PW_CUDA(cudaMemcpyAsync(b.d_lut[b.slot ^ 1], b.h_lut[new_bits],
+                          sizeof(uint16_t) * static_cast<size_t>(b.rows) << new_bits,
+                          cudaMemcpyHostToDevice, s));
+  PW_CUDA(cudaEventRecord(b.ready, s));
+  b.pend_bits = new_bits;
+  b.pend_due = h->n_forwards + 1;
+  return PW_OK;
+}
+
+pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_next,
+                              int32_t* bits_pending) {
+  if (!h || !bits_next) return fail(PW_ERR_INVALID_ARG, "null argument");
+  if (block_id < 0 || block_id >= h->n_blocks)
+    return fail(PW_ERR_INVALID_ARG, "block id %d out of range", block_id);
+  const auto& b = h->blk[block_id];
+  const bool due = b.pend_bits && b.pend_due <= h->n_forwards;
+  *bits_next = due ? b.pend_bits : b.bits;
+  if (bits_pending) *bits_pending = due ? 0 : b.pend_bits;
+  return PW_OK;
+}
+
+static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
+                                const float* d_wr, const float* d_bias, uint16_t* d_y,
+                                cudaStream_t s) {
+  const pw_moe_config_t& c = h->cfg;
+  // page moves that are due: the stream waits for their copies
+  for (auto& b : h->blk) {
+    if (b.pend_bits && b.pend_due <= h->n_forwards) {
+      PW_CUDA(cudaStreamWaitEvent(s, b.ready, 0));
+      b.bits = b.pend_bits;
+      b.slot ^= 1;
+      b.pend_bits = 0;
+    }
+  }
+  h->n_forwards++;
+  h->last_T = T;
+  if (T == 0) {
+    PW_CUDA(cudaEventRecord(h->fwd_done, s));
+    h->any_forward = true;
+    return PW_OK;
+  }
+  pw::PageTable pt;
+  for (int i = 0; i < h->n_blocks; ++i) {
+    pt.blk[i].planes = h->blk[i].d_planes;
+    pt.blk[i].lut = h->blk[i].d_lut[h->blk[i].slot];
+    pt.bits[i] = static_cast<uint8_t>(h->blk[i].bits);
+  }
+  const int has_shared = c.shared_ffn > 0 ? 1 : 0;
+  std::vector<cudaEvent_t> evs;
+  if (h->profiling) {
+    for (int i = 0; i < 5; ++i) {
+      cudaEvent_t e;
+      if (!h->ev_pool.empty()) {
+        e = h->ev_pool.back();
+        h->ev_pool.pop_back();
+      } else {
+        PW_CUDA(cudaEventCreate(&e));
+      }
+      evs.push_back(e);
+    }
+  }
+  auto mark = [&](int i) -> cudaError_t {
+    return h->profiling ? cudaEventRecord(evs[i], s) : cudaSuccess;
+  };
+  PW_CUDA(mark(0));
+
+  pw::RouteParams rp{};
+  rp.x = d_x;
+  rp.wr = d_wr;
+  rp.bias = d_bias;
+  rp.T = T;
+  rp.H = c.hidden;
+  rp.E = c.n_experts;
+  rp.k = c.top_k;
+  rp.renorm = c.renorm_topk;
+  rp.has_shared = has_shared;
+  rp.ws = h->ws;
+  PW_CUDA(pw::launch_route(rp, h->n_sm, s));
+  PW_CUDA(mark(1));
+
+  // gate/up pass
+  if (h->tc_gu) {
+    pw::TcParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    tp.pt = pt;
+    tp.tmaps = h->d_tmaps;
+    tp.mode = pw::kTcGateUp;
+    tp.H = c.hidden;
+    tp.F = c.ffn;
+    tp.S = c.shared_ffn;
+    tp.E = c.n_experts;
+    tp.n_groups = h->G;
+    tp.n_split = 1;
+    tp.offsets = h->ws.offsets;
+    tp.slot_token = h->ws.slot_token;
+    tp.slot_w = h->ws.slot_w;
+    tp.x = d_x;
+    tp.gu = h->gu;
+    tp.gu_stride = h->gu_stride;
+    tp.err = h->err;
+    PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
+  } else {
+    pw::SimpleParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.pt = pt;
+    sp.mode = 0;
+    sp.H = c.hidden;
+    sp.F = c.ffn;
+    sp.S = c.shared_ffn;
+    sp.E = c.n_experts;
+    sp.n_groups = h->G;
+    sp.offsets = h->ws.offsets;
+    sp.slot_token = h->ws.slot_token;
+    sp.slot_w = h->ws.slot_w;
+    sp.x = d_x;
+    sp.gu = h->gu;
+    sp.gu_stride = h->gu_stride;
+    const int rows = c.ffn > c.shared_ffn ? c.ffn : c.shared_ffn;
+    PW_CUDA(pw::launch_simple(sp, rows, s));
+  }
+  PW_CUDA(mark(2));
+  // down pass
+  int n_split = 1;
+  if (h->tc_down) {
+    n_split = down_splits(h, T);
+    pw::TcParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    tp.pt = pt;
+    tp.tmaps = h->d_tmaps;
+    tp.mode = pw::kTcDown;
+    tp.H = c.hidden;
+    tp.F = c.ffn;
+    tp.S = c.shared_ffn;
+    tp.E = c.n_experts;
+    tp.n_groups = h->G;
+    tp.n_split = n_split;
+    tp.offsets = h->ws.offsets;
+    tp.slot_token = h->ws.slot_token;
+    tp.slot_w = h->ws.slot_w;
+    tp.gu = h->gu;
+    tp.gu_stride = h->gu_stride;
+    tp.ysorted = h->ysorted;
+    tp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
+    tp.err = h->err;
+    PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
+  } else {
+    pw::SimpleParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.pt = pt;
+    sp.mode = 1;
+    sp.H = c.hidden;
+    sp.F = c.ffn;
+    sp.S = c.shared_ffn;
+    sp.E = c.n_experts;
+    sp.n_groups = h->G;
+    sp.offsets = h->ws.offsets;
+    sp.slot_token = h->ws.slot_token;
+    sp.slot_w = h->ws.slot_w;
+    sp.gu = h->gu;
+    sp.gu_stride = h->gu_stride;
+    sp.ysorted = h->ysorted;
+    PW_CUDA(pw::launch_simple(sp, c.hidden, s));
+  }
+  PW_CUDA(mark(3));
+  pw::CombineParams cp{};
+  cp.ysorted = h->ysorted;
+  cp.token_pos = h->ws.token_pos;
+  cp.y = d_y;
+  cp.T = T;
+  cp.H = c.hidden;
+  cp.k = c.top_k;
+  cp.has_shared = has_shared;
+  cp.n_split = n_split;
+  cp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
+  PW_CUDA(pw::launch_combine(cp, s));
+  PW_CUDA(mark(4));
+  if (h->profiling) h->ev_pending.push_back(evs);
+  PW_CUDA(cudaEventRecord(h->fwd_done, s));
+  h->any_forward = true;
+  return PW_OK;
+}
+
+pw_status_t pw_moe_forward(pw_moe_t* h, const uint16_t* d_x, int32_t T, const float* d_router_w,
+                           const float* d_router_bias, uint16_t* d_y, pw_stream_t stream) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  if (T < 0 || T > h->cfg.max_tokens)
+    return fail(PW_ERR_INVALID_ARG, "T = %d outside [0, max_tokens = %d]", T, h->cfg.max_tokens);
+  if (T > 0 && (!d_x || !d_router_w || !d_y)) return fail(PW_ERR_INVALID_ARG, "null buffer");
+  if ((d_x && !aligned16(d_x)) || (d_y && !aligned16(d_y)) ||
+      (d_router_w && !aligned16(d_router_w)))
+    return fail(PW_ERR_INVALID_ARG, "x, y and router weights must be 16-byte aligned");
+  return forward_impl(h, d_x, T, d_router_w, d_router_bias, d_y, static_cast<cudaStream_t>(stream));
+}
+
+pw_status_t pw_moe_forward_host(pw_moe_t* h, const uint16_t* x_host, int32_t T,
+                                const float* d_router_w, const float* d_router_bias,
+                                uint16_t* y_host, pw_stream_t stream) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  if (T < 0 || T > h->cfg.max_tokens)
+    return fail(PW_ERR_INVALID_ARG, "T = %d outside [0, max_tokens = %d]", T, h->cfg.max_tokens);
+  if (T > 0 && (!x_host || !y_host || !d_router_w)) return fail(PW_ERR_INVALID_ARG, "null buffer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(uint16_t) * static_cast<size_t>(T) * h->cfg.hidden;
+  if (T > 0) PW_CUDA(cudaMemcpyAsync(h->stage_x, x_host, bytes, cudaMemcpyHostToDevice, s));
+  pw_status_t st = forward_impl(h, h->stage_x, T, d_router_w, d_router_bias, h->stage_y, s);
+  if (st != PW_OK) return st;
+  if (T > 0) PW_CUDA(cudaMemcpyAsync(y_host, h->stage_y, bytes, cudaMemcpyDeviceToHost, s));
+  PW_CUDA(cudaStreamSynchronize(s));
+  return PW_OK;
+}
+
+pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t rows, int32_t cols,
+                      int32_t bits, const uint16_t* d_x, int32_t T, float* d_y,
+                      pw_stream_t stream) {
+  if (rows < 1 || cols < 1 || T < 0) return fail(PW_ERR_INVALID_ARG, "bad shape");
+  if (bits < 1 || bits > PW_MAX_BITS) return fail(PW_ERR_INVALID_ARG, "bits outside [1, 8]");
+  if (!d_planes || !d_lut || (T > 0 && (!d_x || !d_y))) return fail(PW_ERR_INVALID_ARG, "null buffer");
+  if (!aligned16(d_planes) || !aligned16(d_lut) || (d_x && !aligned16(d_x)))
+    return fail(PW_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  if (T == 0) return PW_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int dev = 0, n_sm = 0;
+  PW_CUDA(cudaGetDevice(&dev));
+  PW_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  if (tc_shape_ok(cols) && env_int("PW_FORCE_SIMPLE", 0) == 0) {
+    pw::TcParams tp;
+    std::memset(&tp, 0, sizeof(tp));
+    pw_status_t st = make_plane_map(&tp.lin_map, d_planes, bits, rows, cols);
+    if (st != PW_OK) return st;
+    tp.mode = pw::kTcLinear;
+    tp.n_groups = 1;
+    tp.n_split = 1;
+    tp.x = d_x;
+    tp.y = d_y;
+    tp.T = T;
+    tp.lin_rows = rows;
+    tp.lin_cols = cols;
+    tp.lin_bits = bits;
+    tp.lin_lut = d_lut;
+    tp.err = nullptr;
+    PW_CUDA(pw::launch_tc(tp, n_sm, s));
+  } else {
+    pw::SimpleParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.mode = 2;
+    sp.x = d_x;
+    sp.y = d_y;
+    sp.T = T;
+    sp.lin_rows = rows;
+    sp.lin_cols = cols;
+    sp.lin_bits = bits;
+    sp.lin_planes = d_planes;
+    sp.lin_lut = d_lut;
+    PW_CUDA(pw::launch_simple(sp, rows, s));
+  }
+  return PW_OK;
+}
+
+pw_status_t pw_get_routing(const pw_moe_t* h, int32_t* d_idx, float* d_w, pw_stream_t stream) {
+  if (!h || !d_idx || !d_w) return fail(PW_ERR_INVALID_ARG, "null argument");
+  const size_t n = static_cast<size_t>(h->last_T) * h->cfg.top_k;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n) {
+    PW_CUDA(cudaMemcpyAsync(d_idx, h->ws.topk_idx, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
+    PW_CUDA(cudaMemcpyAsync(d_w, h->ws.topk_w, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  }
+  return PW_OK;
+}
+
+pw_status_t pw_check_device_error(pw_moe_t* h) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  PW_CUDA(cudaDeviceSynchronize());
+  int e = 0;
+  PW_CUDA(cudaMemcpy(&e, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (e) {
+    PW_CUDA(cudaMemset(h->err, 0, sizeof(int)));
+    return fail(static_cast<pw_status_t>(e), "device-side wait gave up (error %d)", e);
+  }
+  return PW_OK;
+}
+
+pw_status_t pw_profile_enable(pw_moe_t* h, int32_t on) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  h->profiling = on != 0;
+  return PW_OK;
+}
+
+pw_status_t pw_profile_read(pw_moe_t* h, float* ms, int32_t n, int32_t* n_forwards) {
+  if (!h || !ms || n < 4) return fail(PW_ERR_INVALID_ARG, "need a handle and room for 4 floats");
+  for (int i = 0; i < n; ++i) ms[i] = 0.0f;
+  int count = 0;
+  for (auto& v : h->ev_pending) {
+    PW_CUDA(cudaEventSynchronize(v[4]));
+    for (int i = 0; i < 4; ++i) {
+      float t = 0.0f;
+      PW_CUDA(cudaEventElapsedTime(&t, v[i], v[i + 1]));
+      ms[i] += t;
+    }
+    for (auto e : v) h->ev_pool.push_back(e);
+    ++count;
+  }
+  h->ev_pending.clear();
+  if (n_forwards) *n_forwards = count;
+  return PW_OK;
+}
+
+int32_t pw_forward_launches(const pw_moe_t* h, int32_t T) {
+  if (!h) return 0;
+  return T > 0 ? 4 : 0;
+}
+
+pw_status_t pw_destroy(pw_moe_t* h) {
+  if (!h) return PW_OK;
+  pw_status_t st = PW_OK;
+  if (h->fwd_done && cudaEventSynchronize(h->fwd_done) != cudaSuccess)
+    st = fail(PW_ERR_CUDA, "waiting for the last forward failed");
+  for (auto& b : h->blk)
+    if (b.ready && cudaEventSynchronize(b.ready) != cudaSuccess)
+      st = fail(PW_ERR_CUDA, "waiting for a page move failed");
+  free_all(h);
+  return st;
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// pw_internal.h -- shared between the host side (pw_api.cu) and the kernels
+// of the B200 fused mixed-precision MoE library.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pw.h"
+
+namespace pw {
+
+constexpr int kMaxBlocks = 3 * (PW_MAX_EXPERTS + 1);
+constexpr int kMaxGroups = PW_MAX_EXPERTS + 1;  // routed experts + shared
+
+// Page-table entry of one linear-block as the kernels see it for one forward:
+// the plane buffer and the LUT slot that holds LUT_bits.  Passed by value in
+// the kernel parameters, so a forward keeps the table it was launched with
+// while the host moves on to the next one.
+struct BlockRef {
+  const uint32_t* planes;  // [n_max][rows][words]
+  const uint16_t* lut;     // [rows][2^bits] fp16 bits
+};
+
+struct PageTable {
+  BlockRef blk[kMaxBlocks];
+  uint8_t bits[kMaxBlocks];
+};
+
+// Routing results and per-group token lists, written by the route kernel.
+// "Group" g < E is routed expert g; g == E is the shared expert (all tokens).
+// Sorted positions: group g owns positions [offsets[g], offsets[g+1]); the
+// routed lists are ordered by token, the shared list is tokens 0..T-1.
+struct RouteWorkspace {
+  float* logits;        // [T][E]
+  int32_t* topk_idx;    // [T][k]
+  float* topk_w;        // [T][k]
+  int32_t* offsets;     // [G+1]
+  int32_t* slot_token;  // [P] token of each sorted position
+  float* slot_w;        // [P] routing weight of each sorted position
+  int32_t* token_pos;   // [T][k] (+ [T] shared) sorted position of (t, j)
+  uint32_t* ticket;     // last-block-done counter (self-resetting)
+};
+
+struct RouteParams {
+  const uint16_t* x;       // bf16 [T][H]
+  const float* wr;         // [E][H]
+  const float* bias;       // [E] or null
+  int T, H, E, k, renorm, has_shared;
+  RouteWorkspace ws;
+};
+
+struct CombineParams {
+  const float* ysorted;  // [P][H] routing-weighted expert outputs
+  const int32_t* token_pos;
+  uint16_t* y;           // bf16 [T][H]
+  int T, H, k, has_shared;
+  int n_split;           // partial sums per position (split-K of the down pass)
+  long long split_stride;  // floats between splits
+};
+
+// Expert pass over all groups on the CUDA-core (simple) path.
+struct SimpleParams {
+  PageTable pt;
+  int mode;        // 0 = gate/up -> gu, 1 = down -> ysorted, 2 = single linear
+  int H, F, S, E, n_groups;
+  const int32_t* offsets;
+  const int32_t* slot_token;
+  const float* slot_w;
+  const uint16_t* x;      // bf16 [T][H] (modes 0, 2)
+  float* gu;              // [P][2*Fmax] gate | up (mode 0 out, mode 1 in)
+  int gu_stride;          // floats per gu row
+  float* ysorted;         // [P][H] (mode 1 out)
+  float* y;               // [T][rows] (mode 2 out)
+  int T;                  // tokens (mode 2)
+  int lin_rows, lin_cols, lin_bits;  // mode 2 block
+  const uint32_t* lin_planes;
+  const uint16_t* lin_lut;
+};
+
+// Launchers (defined in the .cu files).
+cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
+cudaError_t launch_simple(const SimpleParams& p, int grid_rows, cudaStream_t s);
+
+}  // namespace pw

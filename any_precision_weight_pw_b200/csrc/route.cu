@@ -1,0 +1,204 @@
+// route.cu -- router GEMV, softmax/top-k and token->expert bucketing in one
+// launch, and the final combine.
+//
+// PagedWeight (legiblepapers summary, FAQ Q5): routing and output
+// accumulation are fused into the MoE kernel.  The pages give no routing
+// formula; the library's reading is the one stated in pw.h (logits in fp32
+// with the lane-butterfly order, ranking by logit with ties to the lower
+// expert, softmax over all experts, optional renormalisation).
+#include <cuda_bf16.h>
+
+#include "pw_internal.h"
+
+namespace pw {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kRouteThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// One launch.  Phase 1: every warp computes router logits for (token,
+// expert) pairs; lane j owns columns j, j+32, ... and fuses them in
+// ascending order, then the 32 partial sums meet in a xor butterfly
+// (16, 8, 4, 2, 1), so every lane ends with the same value.  Phase 2 runs in
+// the block that finishes last (a ticket counter, no waiting): top-k and
+// softmax per token, then per-expert token lists built with warp ballots and
+// prefix counts, ordered by token.
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams p) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int warps_per_block = kRouteThreads / 32;
+  const int E = p.E, H = p.H, T = p.T, k = p.k;
+  const RouteWorkspace& ws = p.ws;
+
+  const int total_pairs = T * E;
+  for (int pair = blockIdx.x * warps_per_block + warp; pair < total_pairs;
+       pair += gridDim.x * warps_per_block) {
+    const int t = pair / E;
+    const int e = pair - t * E;
+    const uint16_t* xr = p.x + static_cast<size_t>(t) * H;
+    const float* wr = p.wr + static_cast<size_t>(e) * H;
+    float s = 0.0f;
+    for (int i = lane; i < H; i += 32) s = __fmaf_rn(bf16_bits_to_f32(xr[i]), wr[i], s);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) s = s + __shfl_xor_sync(kFull, s, m);
+    if (lane == 0) ws.logits[pair] = p.bias ? s + p.bias[e] : s;
+  }
+
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(ws.ticket, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // ---- phase 2 (one block): top-k + softmax ------------------------------
+  for (int t = threadIdx.x; t < T; t += kRouteThreads) {
+    const float* l = ws.logits + static_cast<size_t>(t) * E;
+    int sel[PW_MAX_TOPK];
+    float lsel[PW_MAX_TOPK];
+    for (int j = 0; j < k; ++j) {
+      int bi = -1;
+      float best = 0.0f;
+      for (int e = 0; e < E; ++e) {
+        bool taken = false;
+        for (int q = 0; q < j; ++q) taken |= (sel[q] == e);
+        if (taken) continue;
+        const float v = __ldcg(l + e);
+        if (bi < 0 || v > best) {  // strict: equal logits keep the lower index
+          best = v;
+          bi = e;
+        }
+      }
+      sel[j] = bi;
+      lsel[j] = best;
+    }
+    const float mx = lsel[0];
+    float z = 0.0f;
+    for (int e = 0; e < E; ++e) z += expf(__ldcg(l + e) - mx);
+    float psel[PW_MAX_TOPK];
+    float ssum = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      psel[j] = expf(lsel[j] - mx) / z;
+      ssum += psel[j];
+    }
+    for (int j = 0; j < k; ++j) {
+      ws.topk_idx[t * k + j] = sel[j];
+      ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
+    }
+  }
+  __syncthreads();
+
+  // ---- bucketing: counts per expert with warp ballots ---------------------
+  __shared__ int s_cnt[kMaxGroups + 1];
+  __shared__ int s_off[kMaxGroups + 2];
+  for (int e = warp; e < E; e += warps_per_block) {
+    int cnt = 0;
+    for (int base = 0; base < T; base += 32) {
+      const int t = base + lane;
+      bool hit = false;
+      if (t < T)
+        for (int j = 0; j < k; ++j) hit |= (__ldcg(ws.topk_idx + t * k + j) == e);
+      cnt += __popc(__ballot_sync(kFull, hit));
+    }
+    if (lane == 0) s_cnt[e] = cnt;
+  }
+  __syncthreads();
+  const int G = E + (p.has_shared ? 1 : 0);
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = run;
+      run += s_cnt[e];
+    }
+    s_off[E] = run;
+    if (p.has_shared) {
+      s_cnt[E] = T;
+      s_off[E + 1] = run + T;
+    }
+    for (int g = 0; g <= G; ++g) ws.offsets[g] = s_off[g];
+    *ws.ticket = 0u;  // ready for the next forward (kernels on a stream do not overlap)
+  }
+  __syncthreads();
+
+  // ---- bucketing: lists ordered by token ----------------------------------
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int e = warp; e < E; e += warps_per_block) {
+    int run = s_off[e];
+    for (int base = 0; base < T; base += 32) {
+      const int t = base + lane;
+      int slot = -1;
+      if (t < T)
+        for (int j = 0; j < k; ++j)
+          if (__ldcg(ws.topk_idx + t * k + j) == e) slot = j;
+      const unsigned m = __ballot_sync(kFull, slot >= 0);
+      if (slot >= 0) {
+        const int pos = run + __popc(m & lt_mask);
+        ws.slot_token[pos] = t;
+        ws.slot_w[pos] = __ldcg(ws.topk_w + t * k + slot);
+        ws.token_pos[t * k + slot] = pos;
+      }
+      run += __popc(m);
+    }
+  }
+  if (p.has_shared) {
+    for (int t = threadIdx.x; t < T; t += kRouteThreads) {
+      const int pos = s_off[E] + t;
+      ws.slot_token[pos] = t;
+      ws.slot_w[pos] = 1.0f;
+      ws.token_pos[T * k + t] = pos;
+    }
+  }
+}
+
+// out[t] = sum_j ysorted[pos(t, j)] (+ shared) in slot order, summing the
+// split-K partials of each position in split order; fp32, rounded to bf16.
+__global__ void combine_kernel(const CombineParams p) {
+  const int t = blockIdx.y;
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (c >= p.H) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int nslots = p.k + (p.has_shared ? 1 : 0);
+  for (int j = 0; j < nslots; ++j) {
+    const int pos = (j < p.k) ? p.token_pos[t * p.k + j] : p.token_pos[p.T * p.k + t];
+    for (int s = 0; s < p.n_split; ++s) {
+      const float4 v = *reinterpret_cast<const float4*>(
+          p.ysorted + s * p.split_stride + static_cast<size_t>(pos) * p.H + c);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+  }
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 out;
+  out.x = *reinterpret_cast<uint32_t*>(&lo);
+  out.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(p.y + static_cast<size_t>(t) * p.H + c) = out;
+}
+
+}  // namespace
+
+cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s) {
+  const int pairs = p.T * p.E;
+  const int warps = kRouteThreads / 32;
+  int grid = (pairs + warps - 1) / warps;
+  if (grid > 4 * n_sm) grid = 4 * n_sm;
+  if (grid < 1) grid = 1;
+  route_kernel<<<grid, kRouteThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
+  const int threads = 128;
+  dim3 grid((p.H / 4 + threads - 1) / threads, p.T);
+  combine_kernel<<<grid, threads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace pw

@@ -1,0 +1,40 @@
+// tc.h -- parameters of the tensor-core dequant-GEMM kernel (tc.cu).
+#pragma once
+
+#include <cuda.h>
+
+#include "pw_internal.h"
+
+namespace pw {
+
+constexpr int kTcTokens = 32;  // token tile of one work item (MMA N <= 32)
+constexpr int kTcGateUp = 0;   // gate and up blocks of every group -> gu
+constexpr int kTcDown = 1;     // down blocks, B = silu(g) * u -> routing-weighted partials
+constexpr int kTcLinear = 2;   // one standalone block -> y
+
+struct TcParams {
+  CUtensorMap lin_map;           // plane tensor map of the standalone block (mode 2)
+  PageTable pt;                  // bits + active LUT slot per block (modes 0, 1)
+  const CUtensorMap* tmaps;      // plane tensor map per block id (modes 0, 1)
+  int mode;
+  int H, F, S, E, n_groups;
+  int n_split;                   // K ranges of the down pass (1 otherwise)
+  const int32_t* offsets;        // [G+1] sorted-position ranges per group
+  const int32_t* slot_token;
+  const float* slot_w;
+  const uint16_t* x;             // bf16 activations (modes 0, 2)
+  float* gu;                     // [P][gu_stride]: gate | up per sorted position
+  int gu_stride;
+  float* ysorted;                // [n_split][P][H]
+  long long split_stride;        // floats between split partial buffers
+  float* y;                      // [T][lin_rows] (mode 2)
+  int T;
+  int lin_rows, lin_cols, lin_bits;
+  const uint16_t* lin_lut;
+  int* err;                      // device error word (may be null)
+};
+
+size_t tc_smem_bytes();
+cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s);
+
+}  // namespace pw

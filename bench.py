@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the fused mixed-bitwidth MoE layer forward on B200.
+
+Metric: MoE-layer decode tokens/s and achieved HBM GB/s (fraction of the
+measured HBM copy bandwidth), on synthetic layers shaped like the models the
+PagedWeight pages evaluate (legiblepapers summary, FAQ Q6).  Headline
+workload: the Mixtral-8x7B-shaped layer (hidden 4096, 8 experts of FFN 14336,
+top-2, bitwidths drawn from {3, 4, 6}) at a decode batch of 16 tokens.  One
+step = one forward (router, top-k, bucketing, gate/up, SwiGLU, down,
+weighted combine) over a fresh token batch already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the layer on its
+own GPU (the layer does not shard: replicas only); value = all tokens / the
+slowest rank's time.  --impl reference times the CPU oracle (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of B200 roofline), 1 GPU"
+HEADLINE = ("mixtral_8x7b", 16)
+SWEEP = [("mixtral_8x7b", 1), ("mixtral_8x7b", 64), ("qwen15_moe_a27b", 1),
+         ("qwen15_moe_a27b", 8), ("qwen15_moe_a27b", 32)]
+N_BATCHES = 8  # distinct token batches cycled through the timed steps
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- bytes
+def block_bytes(layer, blk):
+    rows, cols = layer.shape(blk)
+    b = layer.bits[blk]
+    return b * rows * ((cols + 31) // 32) * 4 + rows * (1 << b) * 2
+
+
+def algorithmic_bytes(layer, idx):
+    """Bytes the method must move for one forward: the active planes and LUTs
+    of every expert with at least one routed token (plus the shared expert),
+    the router weights, the activations in and the output out."""
+    wl = layer.wl
+    T = idx.shape[0]
+    active = sorted(set(int(e) for e in np.unique(idx)))
+    if wl.shared_ffn > 0:
+        active.append(wl.n_experts)
+    gu = sum(block_bytes(layer, 3 * e + p) for e in active for p in (0, 1))
+    down = sum(block_bytes(layer, 3 * e + 2) for e in active)
+    router = wl.n_experts * wl.hidden * 4
+    act = 2 * T * wl.hidden * 2
+    return {"gu": gu + T * wl.hidden * 2, "down": down, "total": gu + down + router + act}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "bench_clocks_%d.csv" % os.getpid())
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self, t_begin=None, t_end=None):
+        """Samples taken between t_begin and t_end (host wall clock)."""
+        import datetime
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if t_begin is not None and not (t_begin - 0.15 <= ts <= t_end + 0.15):
+                    continue
+                rows.append((float(parts[1]), float(parts[2]), parts[5], parts[6], parts[7],
+                             parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from any_precision_weight_pw_b200 import binding, build, synth
+
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    hbm_peak, peak_kind = peaks()
+
+    def prepare_layer(name, seed):
+        layer = synth.Layer(synth.WORKLOADS[name], seed=seed)
+        d = binding.upload_synth_layer(layer, max_tokens=64)
+        wr = torch.from_numpy(layer.router_w).to(dev)
+        bias = None if layer.router_bias is None else torch.from_numpy(layer.router_bias).to(dev)
+        return layer, d, wr, bias
+
+    def prepare_batches(layer, d, wr, bias, T, seed):
+        xs_np = [synth.tokens(layer.wl, T, seed=seed, batch=b) for b in range(N_BATCHES)]
+        xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x in xs_np]
+        ys = [torch.empty_like(x) for x in xs]
+        bts = []  # routing of every batch (untimed) for the byte accounting
+        for x, y in zip(xs, ys):
+            d.forward(x, wr, bias, y)
+            idx, _ = d.routing(T)
+            bts.append(algorithmic_bytes(layer, idx.cpu().numpy()))
+        torch.cuda.synchronize()
+        d.check_device_error()
+        return xs, xs_np, ys, bts
+
+    name, T = HEADLINE
+    layer, d, wr, bias = prepare_layer(name, seed=rank)
+    xs, xs_np, ys, bts = prepare_batches(layer, d, wr, bias, T, seed=rank)
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        d.forward(xs[i % N_BATCHES], wr, bias, ys[i % N_BATCHES])
+    torch.cuda.synchronize()
+    d.profile(True)
+    d.profile_read()
+    with ClockSampler(local_rank) as clk:
+        time.sleep(1.0)  # let nvidia-smi start sampling
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t_begin = time.time()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            d.forward(xs[i % N_BATCHES], wr, bias, ys[i % N_BATCHES])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_end = time.time()
+        if world > 1:
+            torch.distributed.barrier()
+        ms = e0.elapsed_time(e1)
+    per_launch, n_fwd = d.profile_read()
+    d.profile(False)
+    d.check_device_error()
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    steps = args.steps
+    bytes_total = sum(bts[i % N_BATCHES]["total"] for i in range(steps))
+    bytes_gu = sum(bts[i % N_BATCHES]["gu"] for i in range(steps))
+    bytes_down = sum(bts[i % N_BATCHES]["down"] for i in range(steps))
+    tok_s = world * steps * T / (ms_max / 1e3)
+    fwd_gbs = bytes_total / (ms / 1e3) / 1e9
+    # dominant kernel: the tensor-core dequant-GEMM (its gate/up and down launches)
+    tc_ms = per_launch[1] + per_launch[2]
+    tc_gbs = (bytes_gu + bytes_down) / (tc_ms / 1e3) / 1e9 if tc_ms > 0 else None
+    traffic = None
+    prof_path = os.path.join(ROOT, "profiles", "traffic_per_forward.json")
+    if os.path.exists(prof_path):
+        tr = json.load(open(prof_path))
+        if tr.get("workload") == "%s T=%d" % HEADLINE:
+            traffic = tr.get("dram_bytes_per_forward")
+
+    # end to end: host activations in, host output out, through the C ABI
+    xh = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_np]
+    yh = torch.empty_like(xh[0]).pin_memory()
+    for i in range(min(3, args.warmup)):
+        d.forward_host(xh[i % N_BATCHES], wr, bias, yh)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for i in range(args.steps):
+        d.forward_host(xh[i % N_BATCHES], wr, bias, yh)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e2.elapsed_time(e3)
+    e2e_wall = time.perf_counter() - t0
+    e2e_tok_s = world * args.steps * T / (max(e2e_ms, e2e_wall * 1e3) / 1e3)
+
+    # decode sweep (other batch sizes and the Qwen-shaped layer); L2 flushed
+    # between timed forwards so small layers are not served from cache
+    sweep = []
+    if rank == 0 and not args.no_sweep:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        cur = (name, layer, d, wr, bias)
+        for (wname, wT) in SWEEP:
+            if wname != cur[0]:
+                cur[2].close()
+                cur = (wname,) + prepare_layer(wname, seed=rank)
+            _, lay, dd, wr2, b2 = cur
+            xs2, _, ys2, bts2 = prepare_batches(lay, dd, wr2, b2, wT, seed=rank)
+            times = []
+            for i in range(3 + 20):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                dd.forward(xs2[i % N_BATCHES], wr2, b2, ys2[i % N_BATCHES])
+                b.record(stream)
+                torch.cuda.synchronize()
+                if i >= 3:
+                    times.append(a.elapsed_time(b))
+            dd.check_device_error()
+            med = float(np.median(times))
+            mb = float(np.mean([bb["total"] for bb in bts2]))
+            sweep.append({"workload": wname, "tokens": wT, "ms_median": round(med, 4),
+                          "tokens_per_s": round(wT / (med / 1e3), 1),
+                          "gbs": round(mb / (med / 1e3) / 1e9, 1),
+                          "frac_of_measured_hbm": round(mb / (med / 1e3) / 1e9 / hbm_peak, 4),
+                          "bytes_alg": int(mb)})
+            del xs2, ys2
+        cur[2].close()
+        del flush
+    else:
+        d.close()
+
+    cpu = cpu_baseline(layer, xs_np[0], T) if (rank == 0 and world == 1 and not args.no_cpu) \
+        else None
+    if rank != 0:
+        return None
+    wl = layer.wl
+    launches = 4 * args.steps
+    out = {
+        "metric": METRIC,
+        "value": round(tok_s, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": "%s decode T=%d" % (name, T), "hidden": wl.hidden, "ffn": wl.ffn,
+                   "experts": wl.n_experts, "top_k": wl.top_k,
+                   "bits": sorted(set(layer.bits)),
+                   "l2": "inputs larger than L2 (active planes %.2f GB per forward, L2 126 MB)"
+                         % (bytes_total / steps / 1e9),
+                   "batches": N_BATCHES, "parallelism": "replicas" if world > 1 else "1 GPU"},
+        "hbm_gbs": round(fwd_gbs, 1),
+        "hbm_frac": round(fwd_gbs / hbm_peak, 4),
+        "hbm_peak": {"gbs": hbm_peak, "kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "tc_kernel (gate/up + down launches)",
+                     "achieved": round(tc_gbs, 1) if tc_gbs else None, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(tc_gbs / hbm_peak, 4) if tc_gbs else None,
+                     "traffic": traffic,
+                     "launch_ms_per_forward": [round(m / max(n_fwd, 1), 5) for m in per_launch]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_tok_s, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(T * wl.hidden * 2),
+                "d2h_bytes_per_step": int(T * wl.hidden * 2)},
+        "clocks": clk.summary(t_begin, t_end),
+        "gpu_launches": launches,
+        "sweep": sweep,
+    }
+    return out
+
+
+def cpu_baseline(layer, x_np, T, budget_s=12.0):
+    """The oracle as it stands, on this host's cores, one token at a time
+    until the time budget is spent (a bounded sample of the batch)."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from pw_testutil import oracle_layer
+    threads = oracle.default_threads()
+    L = oracle_layer(oracle, layer)
+    done = 0
+    t0 = time.perf_counter()
+    while done < T and (time.perf_counter() - t0) < budget_s:
+        L.forward(x_np[done:done + 1], layer.router_w, layer.router_bias, threads=threads)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(done / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of the %d tokens of one batch, one token per oracle call, %.1f s"
+                      % (done, T, dt)}
+
+
+def run_reference(args):
+    """The oracle timed as the reference arm, on the headline workload; each
+    step is a bounded sample: one token of a batch."""
+    from any_precision_weight_pw_b200 import synth
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from pw_testutil import oracle_layer
+    name, T = HEADLINE
+    layer = synth.Layer(synth.WORKLOADS[name], seed=0)
+    x = synth.tokens(layer.wl, T, seed=0, batch=0)
+    threads = oracle.default_threads()
+    L = oracle_layer(oracle, layer)
+    for i in range(args.warmup):
+        L.forward(x[i % T:i % T + 1], layer.router_w, layer.router_bias, threads=threads)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        L.forward(x[i % T:i % T + 1], layer.router_w, layer.router_bias, threads=threads)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "%s decode T=%d" % HEADLINE, "hidden": layer.wl.hidden,
+                       "ffn": layer.wl.ffn, "experts": layer.wl.n_experts,
+                       "top_k": layer.wl.top_k},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": "one token of the batch per step (%d steps)" % args.steps},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * pw.h -- C ABI of the B200 fused mixed-precision MoE layer (PagedWeight's
+ * hot path).
+ *
+ * What the library computes.  One Mixture-of-Experts FFN layer whose expert
+ * weights are stored as Any-Precision bit-plane pages plus per-row lookup
+ * tables, each linear-block (expert x projection) at its own bitwidth, with
+ * routing, expert activation and the weighted output sum fused into the same
+ * GPU pass:
+ *   - PagedWeight (arxivlens summary), abstract paragraph: a fused
+ *     mixed-precision MoE kernel processes AP bit-planes and LUTs of the
+ *     GPU-resident pages; page movement runs asynchronously, overlapped with
+ *     serving.
+ *   - PagedWeight (legiblepapers summary), "Key Takeaways" and FAQ Q5: the
+ *     kernel reads the bit-plane and LUT buffers directly, supports a
+ *     different bitwidth for every linear-block, and fuses routing, expert
+ *     activation and output accumulation.
+ *   - same summary, "Summary & Methodology Analysis": the bit-plane and LUT
+ *     buffers are GPU-resident pages that are reloaded or offloaded
+ *     asynchronously to hide latency.
+ *
+ * Definitions (readings where the pages are silent):
+ *   Linear-block W, rows x cols, applied as y = W x.  Routed expert e has
+ *   block ids 3e+0 (gate, F x H), 3e+1 (up, F x H), 3e+2 (down, H x F); the
+ *   shared expert (if any) has ids 3E+0..3E+2 with S in place of F.
+ *   Bit-planes: uint32 [n_max][rows][words], words = ceil(cols/32), plane 0
+ *   holds the MOST significant code bit; bit (i % 32) of word (i / 32) is
+ *   column i; pad bits are zero.  A b-bit view reads planes 0..b-1 only:
+ *   code_b = sum_{k<b} bit_k << (b-1-k) = code_{n_max} >> (n_max - b).
+ *   LUT of bitwidth b: fp16 [rows][2^b]; W[o][i] = LUT_b[o][code_b(o, i)].
+ *   Router: logit[t][e] = x_t . Wr_e (+ bias_e) in fp32; experts ranked by
+ *   logit, ties to the lower index; the first k are selected in that order;
+ *   p = softmax over all E logits; slot weight = p of the selected expert,
+ *   divided by the sum over the k selected when renorm_topk = 1.
+ *   Expert: h = silu(x Wg^T) * (x Wu^T), silu(g) = g / (1 + exp(-g));
+ *   y_e = h Wd^T.  Output: y_t = sum_j w_tj * y_{e_tj}(x_t) + shared(x_t)
+ *   (the shared expert is added with weight 1), rounded to bf16 (nearest
+ *   even); accumulation is fp32.
+ *
+ * Conventions.
+ *   Ownership: the caller owns every buffer it passes (device buffers and
+ *   pinned host copies) and keeps them alive and unmodified, except through
+ *   this library, until pw_destroy.  The library owns its handle, workspace
+ *   and events.
+ *   Streams: pw_stream_t is a cudaStream_t (NULL = the legacy default
+ *   stream).  Calls enqueue work and return without synchronising, except
+ *   pw_moe_forward_host, pw_check_device_error and pw_destroy.
+ *   Errors: every call returns a pw_status_t; nothing is thrown across the
+ *   ABI; pw_last_error() gives a message for the calling thread.  On an
+ *   error nothing has been enqueued, unless the status is PW_ERR_CUDA.
+ *   Threads: a handle is used by one host thread at a time.
+ *   Alignment: device buffers 16-byte aligned; x and y row-major, contiguous.
+ *   Kernels: a pass whose blocks have ceil(cols/32) % 4 == 0 and cols % 8 == 0
+ *   runs on the tensor-core kernel (TMA + tcgen05; activations are fed to it
+ *   as fp16, so |x| and |silu(g) u| must stay below 65504); other shapes run
+ *   on the CUDA-core kernel in fp32.
+ */
+#ifndef PW_H_
+#define PW_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PW_ABI_VERSION 1
+#define PW_MAX_BITS 8        /* n_max <= 8 */
+#define PW_MAX_EXPERTS 128   /* routed experts per layer */
+#define PW_MAX_TOPK 8
+
+typedef struct pw_moe pw_moe_t; /* opaque */
+typedef void* pw_stream_t;      /* cudaStream_t */
+
+typedef enum {
+  PW_OK = 0,
+  PW_ERR_INVALID_ARG = 1, /* a null pointer, a size out of range, misalignment */
+  PW_ERR_CUDA = 2,        /* a CUDA runtime call failed (message has the name) */
+  PW_ERR_OOM = 3,         /* workspace allocation failed */
+  PW_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up */
+  PW_ERR_STATE = 5,       /* call not valid now (e.g. a switch still pending) */
+  PW_ERR_UNSUPPORTED = 6  /* shape or device the kernels do not handle */
+} pw_status_t;
+
+typedef struct {
+  int32_t hidden;      /* H, multiple of 8 */
+  int32_t ffn;         /* F, routed expert FFN width, >= 1 */
+  int32_t n_experts;   /* E, 1..PW_MAX_EXPERTS */
+  int32_t top_k;       /* k, 1..min(E, PW_MAX_TOPK) */
+  int32_t shared_ffn;  /* S, shared expert FFN width, 0 = none */
+  int32_t n_max;       /* planes stored per block, 1..PW_MAX_BITS */
+  int32_t renorm_topk; /* 1 = selected weights renormalised to sum to one */
+  int32_t max_tokens;  /* largest T a forward may pass (sizes the workspace) */
+} pw_moe_config_t;
+
+/* One linear-block page (see "Definitions").  rows and cols follow from the
+ * block id and the config. */
+typedef struct {
+  uint32_t* d_planes;   /* device, [n_max][rows][words]; planes 0..bits-1 must
+                           be resident at create; the library writes planes
+                           bits..n_max-1 when a switch raises the bitwidth */
+  uint16_t* d_lut[2];   /* device, two LUT slots of rows * 2^n_max fp16 each;
+                           slot 0 holds LUT_bits at create; the library writes
+                           the idle slot when a switch changes the bitwidth */
+  const uint32_t* h_planes; /* host master copy of all n_max planes (pinned for
+                               overlap), or NULL if the block is never raised */
+  const uint16_t* h_lut[PW_MAX_BITS + 1]; /* host LUT_b at index b, [rows][2^b],
+                                             NULL where b is never used */
+  int32_t bits;         /* bitwidth at create, 1..n_max */
+} pw_block_desc_t;
+
+/* Create a layer over caller-owned pages.  blocks has 3*E (+3 if S > 0)
+ * entries in block-id order.  Allocates the workspace on the current device. */
+pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blocks,
+                          int32_t n_blocks, pw_moe_t** out);
+
+/* Change the bitwidth of one linear-block (an asynchronous page move).
+ * Enqueued on side_stream after the most recently issued forward ends:
+ * raising b -> b' copies planes b..b'-1 and LUT_b' from the host copies;
+ * lowering copies LUT_b' only (the top b' planes are already resident).  The
+ * LUT lands in the idle slot, so no forward ever reads memory being written.
+ * Lag: with N forwards issued, forward N still uses the old bitwidth and
+ * forward N+1 waits for the copy and uses the new one.  PW_ERR_STATE while an
+ * earlier change of the same block has not taken effect yet. */
+pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
+                              pw_stream_t side_stream);
+
+/* y = MoE(x): d_x bf16 [T][H], d_router_w fp32 [E][H], d_router_bias fp32
+ * [E] or NULL, d_y bf16 [T][H] (device).  0 <= T <= max_tokens. */
+pw_status_t pw_moe_forward(pw_moe_t* h, const uint16_t* d_x, int32_t T,
+                           const float* d_router_w, const float* d_router_bias,
+                           uint16_t* d_y, pw_stream_t stream);
+
+/* Free the workspace and events after all work of the handle has finished
+ * (synchronises on the handle's events).  NULL is accepted. */
+pw_status_t pw_destroy(pw_moe_t* h);
+
+/* ---- helpers beyond the four-call contract ---------------------------- */
+
+/* pw_moe_forward with HOST activations: copies x_host (bf16 [T][H]) in and
+ * y_host out through a library-owned device staging buffer, and returns
+ * after the stream has finished (pinned host buffers give full copy speed). */
+pw_status_t pw_moe_forward_host(pw_moe_t* h, const uint16_t* x_host, int32_t T,
+                                const float* d_router_w, const float* d_router_bias,
+                                uint16_t* y_host, pw_stream_t stream);
+
+/* One dequantised linear-block on its own: d_y[t][o] = sum_i W_b[o][i] x[t][i]
+ * with fp32 output.  d_planes [>=bits][rows][words], d_lut [rows][2^bits]
+ * fp16, d_x bf16 [T][cols], d_y fp32 [T][rows]; T >= 0, bits 1..8.  Uses the
+ * same dequantisation and contraction as the MoE experts. */
+pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t rows,
+                      int32_t cols, int32_t bits, const uint16_t* d_x, int32_t T,
+                      float* d_y, pw_stream_t stream);
+
+/* Bitwidth the next forward will use, and the pending one (0 if none). */
+pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_next,
+                              int32_t* bits_pending);
+
+/* Routing of the most recent forward: d_idx int32 [T][k] (selection order)
+ * and d_w fp32 [T][k], copied device-to-device on stream. */
+pw_status_t pw_get_routing(const pw_moe_t* h, int32_t* d_idx, float* d_w,
+                           pw_stream_t stream);
+
+/* Synchronises the device and reports a device-side error flag of the handle
+ * (PW_ERR_TIMEOUT if a bounded wait gave up) and clears it. */
+pw_status_t pw_check_device_error(pw_moe_t* h);
+
+/* Per-launch timing for benchmarks.  While enabled, every forward records
+ * CUDA events around each of its launches (route, gate/up, down, combine).
+ * pw_profile_read synchronises on them and writes, for each launch slot, the
+ * milliseconds summed over the forwards issued since the previous read (ms
+ * has room for n >= 4 floats); *n_forwards receives how many were summed. */
+pw_status_t pw_profile_enable(pw_moe_t* h, int32_t on);
+pw_status_t pw_profile_read(pw_moe_t* h, float* ms, int32_t n, int32_t* n_forwards);
+
+/* Number of kernel launches one forward of this handle issues for T tokens. */
+int32_t pw_forward_launches(const pw_moe_t* h, int32_t T);
+
+const char* pw_last_error(void);
+int32_t pw_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PW_H_ */

@@ -144,6 +144,7 @@ class Layer:
         # blocks: list of (planes [n_max][rows][words] uint32, lut [rows][2^b] uint16,
         #                  rows, cols, bits)
         self._keep = []
+        self.block_list = []
         arr = (_Block * len(blocks))()
         for j, (pl, lt, rows, cols, bits) in enumerate(blocks):
             pl = np.ascontiguousarray(pl, dtype=np.uint32)
@@ -152,6 +153,7 @@ class Layer:
             assert pl.shape[1] == rows and pl.shape[2] == (cols + 31) // 32
             assert bits <= pl.shape[0] <= 8
             self._keep += [pl, lt]
+            self.block_list.append((pl, lt, rows, cols, bits))
             arr[j] = _Block(pl.ctypes.data, lt.ctypes.data, rows, cols, bits)
         self._blocks = arr
         self.c = _Layer(hidden, ffn, n_experts, top_k, shared_ffn, n_max, renorm_topk,

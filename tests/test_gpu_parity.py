@@ -1,0 +1,263 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on
+the same seeded inputs.
+
+Bit-exact: unpacked codes (identity LUT with one-hot inputs returns every
+code), integer linear results, and the top-k expert indices and order.
+Floating point: the output tolerance of tests/pw_testutil.py.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from any_precision_weight_pw_b200 import synth
+from pw_testutil import assert_output_close, oracle_layer, output_errors
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def pw():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from any_precision_weight_pw_b200 import binding, build
+    build.build()
+    return binding
+
+
+def _dev_planes(planes):
+    return torch.from_numpy(np.ascontiguousarray(planes).view(np.int32)).cuda()
+
+
+def _dev_lut(lut):
+    return torch.from_numpy(np.ascontiguousarray(lut).view(np.int16)).cuda()
+
+
+def _dev_bf16(xbits):
+    return torch.from_numpy(np.ascontiguousarray(xbits).view(np.int16)).cuda()
+
+
+def _to_f32(y):
+    """bf16 device tensor (int16 storage) -> float32 numpy."""
+    return (y.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _identity_lut(rows, b):
+    return np.tile(np.arange(1 << b, dtype=np.float16), (rows, 1)).view(np.uint16)
+
+
+# ---------------------------------------------------------------- pw_linear
+
+LINEAR_SHAPES = [
+    (256, 256),   # tensor-core path, full tiles
+    (200, 384),   # tensor-core path, partial row tile, ragged K stage
+    (64, 40),     # CUDA-core path (ceil(40/32) = 2 words)
+]
+
+
+@pytest.mark.parametrize("rows,cols", LINEAR_SHAPES)
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_linear_unpacks_codes_bit_exactly(pw, oracle, rows, cols, b):
+    """Identity LUT and one-hot tokens: y[t][o] = code_b(o, t) for every column."""
+    rng = np.random.default_rng(rows * 100 + cols + b)
+    planes = synth.random_planes(rng, 8, rows, cols)
+    want = oracle.unpack_codes(planes, cols, b).astype(np.float32).T  # [cols][rows]
+    x = synth.to_bf16_bits(np.eye(cols, dtype=np.float32))
+    y = pw.linear(_dev_planes(planes), _dev_lut(_identity_lut(rows, b)), b, _dev_bf16(x))
+    np.testing.assert_array_equal(y.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("rows,cols", LINEAR_SHAPES)
+def test_linear_integer_exact(pw, oracle, rows, cols):
+    rng = np.random.default_rng(7)
+    planes = synth.random_planes(rng, 8, rows, cols)
+    for b in (3, 4, 6, 8):
+        x = rng.integers(-8, 9, size=(37, cols)).astype(np.float32)
+        codes = oracle.unpack_codes(planes, cols, b).astype(np.int64)
+        want = (x.astype(np.int64) @ codes.T).astype(np.float32)
+        y = pw.linear(_dev_planes(planes), _dev_lut(_identity_lut(rows, b)), b,
+                      _dev_bf16(synth.to_bf16_bits(x)))
+        np.testing.assert_array_equal(y.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("rows,cols", LINEAR_SHAPES + [(1408, 2048), (512, 1408)])
+def test_linear_random_matches_oracle(pw, oracle, rows, cols):
+    rng = np.random.default_rng(11)
+    planes = synth.random_planes(rng, 8, rows, cols)
+    for b in (3, 5, 8):
+        lut = synth.random_lut(rng, rows, b)
+        x = synth.to_bf16_bits(rng.normal(size=(5, cols)).astype(np.float32))
+        ref = oracle.linear(planes, lut, cols, b, synth.bf16_bits_to_float(x).astype(np.float64),
+                            threads=8)
+        y = pw.linear(_dev_planes(planes), _dev_lut(lut), b, _dev_bf16(x)).cpu().numpy()
+        scale = np.abs(ref).max()
+        assert np.abs(y - ref).max() <= 1e-5 * scale * max(1.0, cols / 1024)
+
+
+# ---------------------------------------------------------------- whole layer
+
+def _run_layer(pw, layer, T, batch=0, force_simple=False):
+    os.environ["PW_FORCE_SIMPLE"] = "1" if force_simple else "0"
+    try:
+        dev = pw.upload_synth_layer(layer, max_tokens=max(T, 1))
+    finally:
+        os.environ.pop("PW_FORCE_SIMPLE", None)
+    x = synth.tokens(layer.wl, T, seed=layer.seed, batch=batch)
+    xd = _dev_bf16(x)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    bias = None if layer.router_bias is None else torch.from_numpy(layer.router_bias).cuda()
+    y = dev.forward(xd, wr, bias)
+    idx, w = dev.routing(T)
+    torch.cuda.synchronize()
+    dev.check_device_error()
+    yf = _to_f32(y)
+    out = (yf, idx.cpu().numpy(), w.cpu().numpy(), x)
+    dev.close()
+    return out
+
+
+def _oracle_forward(oracle, layer, x, threads=16):
+    L = oracle_layer(oracle, layer)
+    return L.forward(x, layer.router_w, layer.router_bias, threads=threads)
+
+
+@pytest.mark.parametrize("force_simple", [False, True])
+def test_tiny_layer(pw, oracle, force_simple):
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=0)
+    y, idx, w, x = _run_layer(pw, layer, 16, force_simple=force_simple)
+    ref, ridx, rw = _oracle_forward(oracle, layer, x)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=2e-6, atol=1e-7)
+    assert_output_close(y, ref)
+
+
+def test_tiny_layer_many_tokens_one_expert(pw, oracle):
+    """A router bias sends every token to expert 3 first: 70 tokens -> three
+    token tiles for that expert; the second slot spreads over the rest."""
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=1)
+    layer.router_bias = np.zeros(8, np.float32)
+    layer.router_bias[3] = 50.0
+    y, idx, w, x = _run_layer(pw, layer, 70)
+    ref, ridx, rw = _oracle_forward(oracle, layer, x)
+    assert np.all(idx[:, 0] == 3)
+    np.testing.assert_array_equal(idx, ridx)
+    assert_output_close(y, ref)
+
+
+def test_hand_example_on_gpu(pw, oracle):
+    """The 2-expert, 4x32 hand example (CUDA-core path: 1-word rows)."""
+    from test_oracle_layer import _hand_layer
+    L, Wr, x = _hand_layer(oracle)
+    cfg = dict(hidden=32, ffn=4, n_experts=2, top_k=2, shared_ffn=0, n_max=3, renorm_topk=1,
+               max_tokens=3)
+    planes, slots, bits = [], [], []
+    for (pl, lt, rows, cols, b) in L.block_list:
+        planes.append(_dev_planes(pl))
+        s0 = torch.zeros(rows << 3, dtype=torch.int16, device="cuda")
+        s0[: lt.size].copy_(torch.from_numpy(lt.reshape(-1).view(np.int16)))
+        slots.append((s0, torch.zeros_like(s0)))
+        bits.append(b)
+    dev = pw.MoELayer(cfg, planes, slots, bits)
+    y = dev.forward(_dev_bf16(x), torch.from_numpy(Wr).cuda())
+    idx, w = dev.routing(3)
+    torch.cuda.synchronize()
+    assert idx.cpu().numpy().tolist() == [[0, 1], [1, 0], [0, 1]]
+    yf = _to_f32(y)
+    want = [[-0.9035184, -0.9142537, 0.3580196, 0.3472844],
+            [-0.6708742, -0.6615392, 0.5634112, 0.5727461],
+            [-0.9166429, -0.9241294, 0.4995289, 0.4920425]]
+    ref, _, _ = L.forward(x, Wr)
+    np.testing.assert_allclose(ref[:, :4], want, atol=6e-8)
+    assert_output_close(yf, ref)
+    dev.close()
+
+
+@pytest.mark.parametrize("T", [1, 8, 32])
+def test_qwen_shaped_layer(pw, oracle, T):
+    layer = synth.Layer(synth.WORKLOADS["qwen15_moe_a27b"], seed=0)
+    y, idx, w, x = _run_layer(pw, layer, T, batch=T)
+    ref, ridx, rw = _oracle_forward(oracle, layer, x)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=2e-6, atol=1e-7)
+    assert_output_close(y, ref)
+
+
+@pytest.mark.parametrize("T", [1, 16])
+def test_mixtral_shaped_layer(pw, oracle, T):
+    layer = synth.Layer(synth.WORKLOADS["mixtral_8x7b"], seed=0)
+    y, idx, w, x = _run_layer(pw, layer, T, batch=T)
+    ref, ridx, rw = _oracle_forward(oracle, layer, x, threads=32)
+    np.testing.assert_array_equal(idx, ridx)
+    assert_output_close(y, ref)
+
+
+def test_repeat_runs_are_bitwise_identical(pw):
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=2)
+    dev = pw.upload_synth_layer(layer, max_tokens=16)
+    x = _dev_bf16(synth.tokens(layer.wl, 16, seed=2))
+    wr = torch.from_numpy(layer.router_w).cuda()
+    a = dev.forward(x, wr).clone()
+    b = dev.forward(x, wr).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    dev.close()
+
+
+def test_zero_tokens_and_bad_T(pw):
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=0)
+    dev = pw.upload_synth_layer(layer, max_tokens=4)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    x = torch.zeros((0, 256), dtype=torch.int16, device="cuda")
+    y = dev.forward(x, wr)
+    assert y.shape == (0, 256)
+    with pytest.raises(pw.PwError):
+        dev.forward(torch.zeros((5, 256), dtype=torch.int16, device="cuda"), wr)
+    dev.close()
+
+
+def test_bitwidth_switch_lag_and_parity(pw, oracle):
+    """A switch requested after N forwards: forward N keeps the old widths,
+    forward N+1 uses the new ones; both match the oracle at those widths."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=3)
+    dev = pw.upload_synth_layer(layer, max_tokens=16, host_copies=True)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    side = torch.cuda.Stream()
+    changes = {0: 8, 4: 2, 5: 6, 11: 1, 23: 8}
+    x0 = synth.tokens(wl, 16, seed=3, batch=0)
+    dev.forward(_dev_bf16(x0), wr)                      # forward 0
+    old = list(layer.bits)
+    for blk, b in changes.items():
+        dev.set_block_bits(blk, b, side)
+        assert dev.get_block_bits(blk) == (old[blk], b)
+    with pytest.raises(pw.PwError):
+        dev.set_block_bits(0, 3, side)                  # still pending
+    new = list(old)
+    for blk, b in changes.items():
+        new[blk] = b
+    for f, bits in ((1, old), (2, new), (3, new)):
+        x = synth.tokens(wl, 16, seed=3, batch=f)
+        y = dev.forward(_dev_bf16(x), wr)
+        torch.cuda.synchronize()
+        yf = _to_f32(y)
+        ref, _, _ = oracle_layer(oracle, layer, bits).forward(x, layer.router_w, threads=8)
+        assert_output_close(yf, ref)
+        if f == 1:
+            for blk, b in changes.items():
+                assert dev.get_block_bits(blk) == (b, 0)
+    dev.check_device_error()
+    dev.close()
+
+
+def test_forward_host_matches_device(pw):
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=4)
+    dev = pw.upload_synth_layer(layer, max_tokens=16)
+    x = synth.tokens(layer.wl, 16, seed=4)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    yd = dev.forward(_dev_bf16(x), wr).cpu()
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    yh = dev.forward_host(xh, wr)
+    assert torch.equal(yd, yh)
+    dev.close()
