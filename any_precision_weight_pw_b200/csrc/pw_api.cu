@@ -68,12 +68,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // The tensor-core path stages planes with 3-D TMA tiles (words x rows x
-// plane), whose row pitch must be a multiple of 16 bytes, and reads its
-// activation rows with 16-byte vectors.
-bool tc_shape_ok(int cols) {
-  const int words = (cols + 31) / 32;
-  return words % 4 == 0 && cols % 8 == 0;
-}
+// plane), whose row pitch must be a multiple of 16 bytes, and permutes
+// activations in whole 32-column groups: it takes cols % 128 == 0.
+bool tc_shape_ok(int cols) { return cols % 128 == 0; }
 
 pw_status_t make_plane_map(CUtensorMap* m, const uint32_t* planes, int n_planes, int rows,
                            int cols) {
@@ -120,14 +117,17 @@ struct pw_moe {
   bool any_forward = false;
   // workspace
   pw::RouteWorkspace ws{};
-  float* gu = nullptr;
+  float* gu = nullptr;          // CUDA-core path: gate | up per sorted position
+  uint16_t* x_perm = nullptr;   // tensor-core path: fp16 activations, K-permuted
+  uint16_t* h_perm = nullptr;   // tensor-core path: fp16 silu(g) * u, K-permuted
+  int x_perm_ld = 0, h_perm_ld = 0;
   float* ysorted = nullptr;
   int* err = nullptr;
   CUtensorMap* d_tmaps = nullptr;
   uint16_t* stage_x = nullptr;
   uint16_t* stage_y = nullptr;
   int P_max = 0, gu_stride = 0, max_split = 8, last_T = 0;
-  bool tc_gu = false, tc_down = false;
+  bool tc = false;  // both expert passes on the tensor-core kernel
   void* ws_base = nullptr;
   // per-launch timing (pw_profile_*): 5 events per forward bracket 4 launches
   bool profiling = false;
@@ -251,9 +251,12 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const int S = c.shared_ffn;
   h->P_max = T * k + (S > 0 ? T : 0);
   const int Fmax = c.ffn > S ? c.ffn : S;
-  h->gu_stride = 2 * Fmax;
-  h->tc_gu = tc_shape_ok(c.hidden) && env_int("PW_FORCE_SIMPLE", 0) == 0;
-  h->tc_down = tc_shape_ok(c.ffn) && (S == 0 || tc_shape_ok(S)) && env_int("PW_FORCE_SIMPLE", 0) == 0;
+  h->tc = tc_shape_ok(c.hidden) && tc_shape_ok(c.ffn) && (S == 0 || tc_shape_ok(S)) &&
+          env_int("PW_FORCE_SIMPLE", 0) == 0;
+  h->gu_stride = h->tc ? 0 : 2 * Fmax;
+  // rows padded to whole 256-column stages, zero past the end
+  h->x_perm_ld = h->tc ? (c.hidden + 255) / 256 * 256 : 0;
+  h->h_perm_ld = h->tc ? (Fmax + 255) / 256 * 256 : 0;
   auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
   size_t off = 0;
   const size_t o_logits = off; off += al(sizeof(float) * T * E);
@@ -267,6 +270,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const size_t o_err = off; off += al(sizeof(int) * 4);
   const size_t o_tm = off; off += al(sizeof(CUtensorMap) * n_blocks);
   const size_t o_gu = off; off += al(sizeof(float) * size_t(h->P_max) * h->gu_stride);
+  const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(T) * h->x_perm_ld);
+  const size_t o_hp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->h_perm_ld);
   const size_t o_ys = off; off += al(sizeof(float) * size_t(h->max_split) * h->P_max * c.hidden);
   const size_t o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
   const size_t o_sy = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
@@ -286,15 +291,18 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->err = reinterpret_cast<int*>(w + o_err);
   h->d_tmaps = reinterpret_cast<CUtensorMap*>(w + o_tm);
   h->gu = reinterpret_cast<float*>(w + o_gu);
+  h->x_perm = reinterpret_cast<uint16_t*>(w + o_xp);
+  h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
   h->ysorted = reinterpret_cast<float*>(w + o_ys);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
   h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
-  if (cudaMemset(w + o_tk, 0, al(sizeof(uint32_t) * 4) + al(sizeof(int) * 4)) != cudaSuccess) {
+  if (cudaMemset(w + o_tk, 0, al(sizeof(uint32_t) * 4) + al(sizeof(int) * 4)) != cudaSuccess ||
+      cudaMemset(w + o_xp, 0, o_sx - o_xp) != cudaSuccess) {
     free_all(h);
     return fail(PW_ERR_CUDA, "cudaMemset failed");
   }
   // plane tensor maps for the tensor-core passes
-  if (h->tc_gu || h->tc_down) {
+  if (h->tc) {
     std::vector<CUtensorMap> maps(n_blocks);
     for (int i = 0; i < n_blocks; ++i) {
       std::memset(&maps[i], 0, sizeof(CUtensorMap));
@@ -414,12 +422,14 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   rp.k = c.top_k;
   rp.renorm = c.renorm_topk;
   rp.has_shared = has_shared;
+  rp.x_perm = h->tc ? h->x_perm : nullptr;
+  rp.x_perm_ld = h->x_perm_ld;
   rp.ws = h->ws;
   PW_CUDA(pw::launch_route(rp, h->n_sm, s));
   PW_CUDA(mark(1));
 
   // gate/up pass
-  if (h->tc_gu) {
+  if (h->tc) {
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
@@ -434,9 +444,10 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.offsets = h->ws.offsets;
     tp.slot_token = h->ws.slot_token;
     tp.slot_w = h->ws.slot_w;
-    tp.x = d_x;
-    tp.gu = h->gu;
-    tp.gu_stride = h->gu_stride;
+    tp.x_perm = h->x_perm;
+    tp.x_perm_ld = h->x_perm_ld;
+    tp.h_perm = h->h_perm;
+    tp.h_perm_ld = h->h_perm_ld;
     tp.err = h->err;
     PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
   } else {
@@ -461,7 +472,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   PW_CUDA(mark(2));
   // down pass
   int n_split = 1;
-  if (h->tc_down) {
+  if (h->tc) {
     n_split = down_splits(h, T);
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
@@ -477,8 +488,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.offsets = h->ws.offsets;
     tp.slot_token = h->ws.slot_token;
     tp.slot_w = h->ws.slot_w;
-    tp.gu = h->gu;
-    tp.gu_stride = h->gu_stride;
+    tp.h_perm = h->h_perm;
+    tp.h_perm_ld = h->h_perm_ld;
     tp.ysorted = h->ysorted;
     tp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
     tp.err = h->err;

@@ -43,6 +43,8 @@ struct RouteWorkspace {
 
 struct RouteParams {
   const uint16_t* x;       // bf16 [T][H]
+  uint16_t* x_perm;        // fp16 [T][x_perm_ld] in the tensor-core K order, or null
+  int x_perm_ld;
   const float* wr;         // [E][H]
   const float* bias;       // [E] or null
   int T, H, E, k, renorm, has_shared;

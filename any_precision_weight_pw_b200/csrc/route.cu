@@ -7,7 +7,9 @@
 // with the lane-butterfly order, ranking by logit with ties to the lower
 // expert, softmax over all experts, optional renormalisation).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
+#include "dequant.cuh"
 #include "pw_internal.h"
 
 namespace pw {
@@ -33,6 +35,41 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   const int warps_per_block = kRouteThreads / 32;
   const int E = p.E, H = p.H, T = p.T, k = p.k;
   const RouteWorkspace& ws = p.ws;
+
+  // fp16 copy of the activations in the tensor-core kernel's K order (each
+  // 32-column group permuted like the A operand), one 32-column group per
+  // thread; read by the gate/up pass.
+  if (p.x_perm) {
+    const int groups = T * (H >> 5);
+    for (int idx = blockIdx.x * kRouteThreads + threadIdx.x; idx < groups;
+         idx += gridDim.x * kRouteThreads) {
+      const int t = idx / (H >> 5), w = idx - t * (H >> 5);
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * H + 32 * w);
+      float v[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 r = src[q];
+        const uint32_t r4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * q + 2 * e] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] & 0xFFFFu));
+          v[8 * q + 2 * e + 1] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] >> 16));
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.x_perm + static_cast<size_t>(t) * p.x_perm_ld + 32 * w);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 h2 = __floats2half2_rn(v[dq::col_of_kpos(8 * q + 2 * e)],
+                                               v[dq::col_of_kpos(8 * q + 2 * e + 1)]);
+          o[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
 
   const int total_pairs = T * E;
   for (int pair = blockIdx.x * warps_per_block + warp; pair < total_pairs;

@@ -1,36 +1,47 @@
 // tc.cu -- tensor-core dequant-GEMM over Any-Precision bit-plane pages
-// (sm_100a: TMA + tcgen05 + TMEM).
+// (sm_100a: TMA + cp.async + tcgen05 + TMEM).
 //
 // PagedWeight (legiblepapers summary, FAQ Q5; arxivlens abstract): the fused
 // mixed-precision MoE kernel reads the AP bit-planes and per-row LUTs of the
-// resident pages directly, at a separate bitwidth for every linear-block.
+// resident pages directly, at a separate bitwidth for every linear-block, and
+// fuses the expert activation and the output accumulation.
 //
-// One persistent CTA per SM walks a list of work items.  An item is one
-// linear-block x 128 output rows x up to 32 tokens (x one K range when the
-// down pass is split).  Inside the CTA:
-//   warp 4      TMA producer: streams only the b active bit-planes of the
+// One persistent CTA per SM walks a list of work items.  An item is 128
+// output rows x up to 32 tokens of one expert, in one or two passes over K:
+// the gate/up item makes a gate pass and an up pass over the same rows (so
+// its epilogue can apply SwiGLU); the down item makes one pass (over one K
+// range when the down pass is split); a standalone linear makes one pass.
+//   warp 8      TMA producer: streams only the b active bit-planes of the
 //               block, 128 rows x 256 columns (8 words) per plane per stage,
 //               into a ring of 4 KB slots (32-byte swizzle, so that the
 //               thread-per-row reads below are bank-conflict free).
-//   warps 0-3   dequantisers, thread r <-> output row r <-> TMEM lane r: each
-//               thread unpacks its row's codes from the b plane words, looks
-//               them up in its row's LUT (shared memory, one bank per thread)
-//               and writes fp16 weights into a TMEM ring slot (the MMA's A
-//               operand); they also stage the token tile (the B operand) in
-//               shared memory: bf16 activations -> fp16 (gate/up pass) or
-//               silu(g)*u -> fp16 (down pass), in the K order the A slots use.
-//   warp 5      MMA issuer: tcgen05.mma kind::f16, M=128, N=16/32, K=16,
-//               fp32 accumulators in TMEM (two buffers, alternating items).
-//   warps 6-9   epilogue: tcgen05.ld the accumulators, write fp32 outputs
-//               (gate/up values, routing-weighted down partials, or the plain
-//               linear result).
-// Every wait is an mbarrier try_wait bounded by a global-timer deadline; a
-// timeout raises the CTA's abort flag and the device error word, and every
-// role drains what it has in flight before the CTA frees its TMEM and exits.
+//   warp 10     token-tile loader: cp.async copies of the stage's 256
+//               columns of every token row (fp16, already in the A operand's
+//               K order) into a 4-deep ring, in the K-major 128-byte swizzle
+//               layout of the MMA's B operand; two stages in flight.
+//   warps 0-7   dequantisers in two K halves: warps q and q+4 both own rows
+//               32q..32q+31 (thread <-> output row <-> TMEM lane); the first
+//               group takes columns 0-127 of every stage, the second
+//               columns 128-255.  Each thread unpacks its row's codes from the
+//               b plane words, looks them up in its row's LUT (registers for
+//               b <= 3, else a shared-memory table with one bank per thread;
+//               see dequant.cuh) and writes fp16 weights into a TMEM ring
+//               slot (the MMA's A operand).
+//   warp 9      MMA issuer: tcgen05.mma kind::f16, M=128, N=16/32, K=16,
+//               fp32 accumulators in TMEM (two buffers, alternating items;
+//               gate and up accumulate side by side).
+//   warps 11-14 epilogue: tcgen05.ld the accumulators; write h = silu(g)*u
+//               as fp16 in the down pass's K order (gate/up), the routing-
+//               weighted fp32 partials (down), or the fp32 result (linear).
+// Every wait is an mbarrier try_wait (with a suspend hint, so waiting warps
+// do not spin) bounded by a global-timer deadline; a timeout raises the CTA's
+// abort flag and the device error word, and every role drains what it has in
+// flight before the CTA frees its TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "dequant.cuh"
 #include "pw_internal.h"
 #include "tc.h"
 
@@ -43,22 +54,28 @@ constexpr int kSlotBytes = kTileRows * kStageWords * 4;  // 4 KB
 constexpr int kNSlot = 16;
 constexpr int kNT = kTcTokens;                 // token tile (MMA N <= 32)
 constexpr int kBStageBytes = kNT * 256 * 2;    // 32 rows x 256 K fp16 = 16 KB
+constexpr int kNB = 4;                         // token-tile ring depth
 constexpr int kNA = 6;                         // TMEM A ring slots (128 K each)
 constexpr int kAColsPerSlot = 64;
 constexpr int kAColBase = 128;
-constexpr int kDColsPerBuf = 64;
+constexpr int kDColsPerBuf = 64;               // gate at +0, up at +32
 constexpr int kTmemCols = 512;
-constexpr int kLutWords = kTileRows * 128;     // 128 rows x 256 fp16
-constexpr int kThreads = 320;
+constexpr int kDqThreads = 256;                // 8 dequantiser warps
+constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpLoader = 10;
+constexpr int kThreads = 15 * 32;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
-constexpr size_t kSmemSlots = size_t(kNSlot) * kSlotBytes;
-constexpr size_t kSmemB = 2 * size_t(kBStageBytes);
-constexpr size_t kSmemLut = size_t(kLutWords) * 4;
-constexpr size_t kNumBars = 2 * kNSlot + 4 + 2 * kNA + 4 + 1;
-constexpr size_t kSmemBars = kNumBars * 8;
-constexpr size_t kSmemMisc = 16 + 4 * (kMaxGroups + 2) + 16;
-constexpr size_t kSmemTotal = 1024 + kSmemSlots + kSmemB + kSmemLut + kSmemBars + kSmemMisc;
+// Shared memory (offsets from a 1024-byte aligned base; compile-time so the
+// table lookups fold the base into the load's immediate offset).
+constexpr uint32_t kOffLut = 0;                // 128 rows x 128 words x 4 B
+constexpr uint32_t kLutBytes = 128u * 128u * 4u;
+constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
+constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
+constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
+constexpr uint32_t kNumBars = 2 * kNSlot + 2 * kNB + 2 * kNA + 4 + 2;
+constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
+constexpr uint32_t kSmemTotal = kOffMisc + 16 + 4 * (kMaxGroups + 2);
+static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -80,13 +97,14 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, uint32_t bytes) {
                "r"(bytes)
                : "memory");
 }
+// Test (and, for up to the suspend hint in ns, sleep until) completion of a phase.
 __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       "selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_addr(b)), "r"(parity)
+      : "r"(smem_addr(b)), "r"(parity), "r"(100000u)
       : "memory");
   return ok != 0;
 }
@@ -123,15 +141,24 @@ __device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
     if (global_ns() - t0 > 200000000ull) return;
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1,
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
       : "memory");
 }
-
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -153,7 +180,6 @@ __device__ __forceinline__ void tc_mma(uint32_t d, uint32_t a, uint64_t bdesc, u
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
       "r"(a), "l"(bdesc), "r"(idesc), "r"(acc));
 }
-
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -211,264 +237,274 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Byte offset of 16-byte chunk c16 (0..31) of token row n in a B stage
+// (K-major, 128-byte swizzle: 64 columns per 128-byte atom row).
+__device__ __forceinline__ uint32_t b_chunk_off(int n, int c16) {
+  const int atom = c16 >> 3, c = c16 & 7;
+  return atom * (kNT * 128) + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
+}
+
 // ---------------------------------------------------------------- work items
-struct Item {
-  int g, proj, row0, tok0, ntok, pos0, split;
-  int blk, rows, cols, words, bits, s_begin, s_end;
+struct Pass {
+  int blk, bits;
   const uint16_t* lut;
   const CUtensorMap* tmap;
+};
+struct Item {
+  int g, row0, tok0, ntok, pos0, split, rows, cols, npass, s_begin, s_end;
+  Pass pass[2];
 };
 
 __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix, int G,
                                             int i, Item& it) {
   int g = 0;
   while (g + 1 < G && s_prefix[g + 1] <= i) ++g;
-  int local = i - s_prefix[g];
-  int rows, cols, nproj, n, pos0;
+  const int local = i - s_prefix[g];
+  int n, pos0;
   if (p.mode == kTcLinear) {
-    rows = p.lin_rows;
-    cols = p.lin_cols;
-    nproj = 1;
+    it.rows = p.lin_rows;
+    it.cols = p.lin_cols;
     n = p.T;
     pos0 = 0;
   } else {
     const int Fg = (g == p.E) ? p.S : p.F;
-    nproj = (p.mode == kTcGateUp) ? 2 : 1;
-    rows = (p.mode == kTcGateUp) ? Fg : p.H;
-    cols = (p.mode == kTcGateUp) ? p.H : Fg;
+    it.rows = (p.mode == kTcGateUp) ? Fg : p.H;
+    it.cols = (p.mode == kTcGateUp) ? p.H : Fg;
     pos0 = p.offsets[g];
     n = p.offsets[g + 1] - pos0;
   }
-  const int rt = (rows + kTileRows - 1) / kTileRows;
+  const int rt = (it.rows + kTileRows - 1) / kTileRows;
   const int ns = p.n_split;
-  const int per_tt = nproj * rt * ns;
+  const int per_tt = rt * ns;
   const int tt = local / per_tt;
-  int r = local - tt * per_tt;
-  const int proj = r / (rt * ns);
-  r -= proj * rt * ns;
+  const int r = local - tt * per_tt;
   const int row_tile = r / ns;
-  const int split = r - row_tile * ns;
+  it.split = r - row_tile * ns;
   it.g = g;
-  it.proj = (p.mode == kTcGateUp) ? proj : 2;
   it.row0 = row_tile * kTileRows;
   it.tok0 = tt * kNT;
   it.ntok = min(kNT, n - it.tok0);
   it.pos0 = pos0 + it.tok0;
-  it.split = split;
-  it.rows = rows;
-  it.cols = cols;
-  it.words = (cols + 31) >> 5;
-  const int stages = (it.words + kStageWords - 1) / kStageWords;
-  it.s_begin = static_cast<int>((static_cast<long long>(stages) * split) / ns);
-  it.s_end = static_cast<int>((static_cast<long long>(stages) * (split + 1)) / ns);
+  const int stages = (((it.cols + 31) >> 5) + kStageWords - 1) / kStageWords;
+  it.s_begin = static_cast<int>((static_cast<long long>(stages) * it.split) / ns);
+  it.s_end = static_cast<int>((static_cast<long long>(stages) * (it.split + 1)) / ns);
   if (p.mode == kTcLinear) {
-    it.blk = -1;
-    it.bits = p.lin_bits;
-    it.lut = p.lin_lut;
-    it.tmap = &p.lin_map;
+    it.npass = 1;
+    it.pass[0] = Pass{-1, p.lin_bits, p.lin_lut, &p.lin_map};
   } else {
-    it.blk = 3 * g + it.proj;
-    it.bits = p.pt.bits[it.blk];
-    it.lut = p.pt.blk[it.blk].lut;
-    it.tmap = p.tmaps + it.blk;
+    it.npass = (p.mode == kTcGateUp) ? 2 : 1;
+    for (int q = 0; q < it.npass; ++q) {
+      const int blk = 3 * g + ((p.mode == kTcGateUp) ? q : 2);
+      it.pass[q] = Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.tmaps + blk};
+    }
   }
-}
-
-// Column (0..31 of a word) held at position q of the K order of a TMEM A
-// slot: pair register pr = 4m + j holds columns (8j + m, 8j + m + 4).
-__host__ __device__ constexpr int col_of_kpos(int q) {
-  return 8 * ((q >> 1) & 3) + (q >> 3) + 4 * (q & 1);
 }
 
 // ---------------------------------------------------------------- dequant
-// Thread-private LUT: row r's entries (2j, 2j+1) packed in word j*128 + r,
-// so the 32 threads of a warp always hit 32 different banks.
-template <int B>
-__device__ __forceinline__ uint32_t lut_get(const uint32_t* lrow, uint32_t v) {
-  const uint32_t w = lrow[(v >> 1) * kTileRows];
-  return (v & 1u) ? (w >> 16) : (w & 0xFFFFu);
+extern __shared__ __align__(1024) uint8_t pw_tc_smem[];
+
+// Read this thread's 4 words (one 16-byte chunk) of a plane slot: chunk
+// `half` of row r (32-byte swizzle: chunk index xor bit 2 of the row).
+__device__ __forceinline__ uint4 read_plane_chunk(uint32_t slot_off, int r, int half) {
+  const uint32_t off = slot_off + r * 32 + ((half ^ ((r >> 2) & 1)) << 4);
+  return *reinterpret_cast<const uint4*>(pw_tc_smem + off);
 }
 
-// 32 columns of one row: P[k] is plane k's word (k = 0 is the MSB plane).
-// out[pr] = fp16 pair (col 8j+m, col 8j+m+4), pr = 4m + j.
-template <int B>
-__device__ __forceinline__ void dequant_word(const uint32_t (&P)[B], const uint32_t* lrow,
-                                             uint32_t* out) {
-  uint32_t S[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    uint32_t s = 0;
-#pragma unroll
-    for (int k = 0; k < B; ++k) s |= ((P[k] >> m) & 0x01010101u) << (B - 1 - k);
-    S[m] = s;  // byte n = b-bit code of column 8n + m
-  }
-#pragma unroll
-  for (int pr = 0; pr < 16; ++pr) {
-    const int m = pr >> 2, j = pr & 3;
-    const uint32_t v0 = (S[m] >> (8 * j)) & 0xFFu;
-    const uint32_t v1 = (S[m + 4] >> (8 * j)) & 0xFFu;
-    out[pr] = lut_get<B>(lrow, v0) | (lut_get<B>(lrow, v1) << 16);
-  }
-}
-
-// Read this thread's 4 words (one 16-byte chunk) of plane slot `slot` for
-// sub-chunk `sub` (32-byte swizzle: chunk index xor bit 2 of the row).
-__device__ __forceinline__ uint4 read_plane_chunk(const uint8_t* slot, int r, int sub) {
-  const int off = r * 32 + ((sub ^ ((r >> 2) & 1)) << 4);
-  return *reinterpret_cast<const uint4*>(slot + off);
+// All dequantiser threads meet (a bounded wait, unlike a hardware barrier,
+// so a warp that gave up cannot leave the others blocked).
+__device__ __forceinline__ bool dq_sync(uint64_t* bar, uint32_t& phase, const Ctl& ctl) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait_warp(bar, phase, ctl);
+  phase ^= 1u;
+  return ok;
 }
 
 struct DequantState {
-  uint32_t slot_ctr, a_ctr, b_ctr;
+  uint32_t slot_ctr;  // plane slots consumed
+  uint32_t a_ctr;     // stages processed by this K half
 };
 
-// Stage the token tile of stage s (256 K) into B buffer `buf`, K-major in
-// the 128-byte swizzle layout, columns permuted into the A slot order.
-__device__ void fill_b(const TcParams& p, const Item& it, int s, uint8_t* buf, int tid) {
-  const int total = it.ntok * kStageWords;
-  for (int idx = tid; idx < total; idx += 128) {
-    const int n = idx >> 3, w = idx & 7;
-    const int col0 = s * 256 + 32 * w;
-    float v[32];
-    if (p.mode == kTcDown) {
-      const int Fg = it.cols;
-      const float* gr = p.gu + static_cast<size_t>(it.pos0 + n) * p.gu_stride;
-      const float* ur = gr + Fg;
-      if (col0 + 32 <= it.cols) {
+// b = 8 tables are packed two entries per word: word (v >> 1) * 128 + r.
+// The offset of the entry for byte n of x (an 8-bit code) is
+// ((v >> 1) << 9) | ((v & 1) << 1) | 4r.
+template <int N>
+__device__ __forceinline__ uint32_t byte_addr8(uint32_t x, uint32_t r4) {
+  const uint32_t a = (dq::shl<8 - 8 * N>(x) & 0xFE00u) | r4;
+  return (dq::shl<1 - 8 * N>(x) & 2u) | a;
+}
+__device__ __forceinline__ void dq_word8(const uint32_t (&P)[8], uint32_t r4, uint32_t* out) {
+  uint32_t X[8];
+  dq::transpose_codes<8>(P, X);
+  auto lds = [](uint32_t x) -> uint32_t {
+    return *reinterpret_cast<const uint16_t*>(pw_tc_smem + kOffLut + x);
+  };
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 g4 = *reinterpret_cast<const float4*>(gr + col0 + 4 * q);
-          const float4 u4 = *reinterpret_cast<const float4*>(ur + col0 + 4 * q);
-          v[4 * q + 0] = g4.x / (1.0f + expf(-g4.x)) * u4.x;
-          v[4 * q + 1] = g4.y / (1.0f + expf(-g4.y)) * u4.y;
-          v[4 * q + 2] = g4.z / (1.0f + expf(-g4.z)) * u4.z;
-          v[4 * q + 3] = g4.w / (1.0f + expf(-g4.w)) * u4.w;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = col0 + c;
-          if (col < it.cols) {
-            const float gv = gr[col];
-            v[c] = gv / (1.0f + expf(-gv)) * ur[col];
-          } else {
-            v[c] = 0.0f;
-          }
-        }
-      }
-    } else {
-      const int t = (p.mode == kTcGateUp) ? p.slot_token[it.pos0 + n] : it.tok0 + n;
-      const int ld = (p.mode == kTcGateUp) ? p.H : p.lin_cols;
-      const uint16_t* src = p.x + static_cast<size_t>(t) * ld;
-      if (col0 + 32 <= it.cols && (ld & 7) == 0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + col0 + 8 * q);
-          const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[8 * q + 2 * e] = bf16f(static_cast<uint16_t>(r4[e] & 0xFFFFu));
-            v[8 * q + 2 * e + 1] = bf16f(static_cast<uint16_t>(r4[e] >> 16));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = col0 + c;
-          v[c] = (col < it.cols) ? bf16f(src[col]) : 0.0f;
-        }
-      }
-    }
-    uint32_t q16[16];
-#pragma unroll
-    for (int pr = 0; pr < 16; ++pr) q16[pr] = pack_h2(v[col_of_kpos(2 * pr)], v[col_of_kpos(2 * pr + 1)]);
-    const int atom = w >> 1;
-    uint8_t* rowp = buf + atom * (kNT * 128) + (n >> 3) * 1024 + (n & 7) * 128;
-#pragma unroll
-    for (int qc = 0; qc < 4; ++qc) {
-      const int c16 = (w & 1) * 4 + qc;
-      *reinterpret_cast<uint4*>(rowp + ((c16 ^ (n & 7)) << 4)) =
-          make_uint4(q16[4 * qc], q16[4 * qc + 1], q16[4 * qc + 2], q16[4 * qc + 3]);
-    }
+  for (int m = 0; m < 4; ++m) {
+    out[4 * m + 0] = dq::pack16(lds(byte_addr8<0>(X[m], r4)), lds(byte_addr8<0>(X[m + 4], r4)));
+    out[4 * m + 1] = dq::pack16(lds(byte_addr8<1>(X[m], r4)), lds(byte_addr8<1>(X[m + 4], r4)));
+    out[4 * m + 2] = dq::pack16(lds(byte_addr8<2>(X[m], r4)), lds(byte_addr8<2>(X[m + 4], r4)));
+    out[4 * m + 3] = dq::pack16(lds(byte_addr8<3>(X[m], r4)), lds(byte_addr8<3>(X[m + 4], r4)));
   }
 }
 
 template <int B>
-__device__ bool dequant_stages(const TcParams& p, const Item& it, uint8_t* slots, uint8_t* bbuf,
-                               const uint32_t* lrow, uint64_t* pf, uint64_t* pe, uint64_t* bfull,
-                               uint64_t* bempty, uint64_t* af, uint64_t* ae, uint32_t tmem_a_lane,
-                               DequantState& st, const Ctl& ctl) {
-  const int r = threadIdx.x;
+__device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegLut& L,
+                               uint64_t* pf, uint64_t* pe, uint64_t* af, uint64_t* ae,
+                               uint32_t tmem_base, DequantState& st, const Ctl& ctl) {
+  const int lane = threadIdx.x & 31;
+  const int r = 32 * quad + lane;
+  const uint32_t r4 = 4u * static_cast<uint32_t>(r);
+  const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * quad) << 16);
+  auto lds = [](uint32_t x) -> uint32_t {
+    return *reinterpret_cast<const uint16_t*>(pw_tc_smem + kOffLut + x);
+  };
   for (int s = it.s_begin; s < it.s_end; ++s) {
-    // token tile for this stage
-    const uint32_t jb = st.b_ctr & 1u;
-    if (!mbar_wait_warp(&bempty[jb], ((st.b_ctr >> 1) & 1u) ^ 1u, ctl)) return false;
-    fill_b(p, it, s, bbuf + jb * kBStageBytes, r);
-    fence_proxy_async();
-    mbar_arrive(&bfull[jb]);
-    st.b_ctr++;
-    // planes of this stage
+    uint32_t P[4][B];
 #pragma unroll
     for (int k = 0; k < B; ++k) {
       const uint32_t c = st.slot_ctr + k;
       if (!mbar_wait_warp(&pf[c % kNSlot], (c / kNSlot) & 1u, ctl)) return false;
+      const uint4 q4 = read_plane_chunk(kOffSlots + (c % kNSlot) * kSlotBytes, r, grp);
+      P[0][k] = q4.x;
+      P[1][k] = q4.y;
+      P[2][k] = q4.z;
+      P[3][k] = q4.w;
     }
-#pragma unroll 1
-    for (int sub = 0; sub < 2; ++sub) {
-      uint32_t P[4][B];
 #pragma unroll
-      for (int k = 0; k < B; ++k) {
-        const uint4 q = read_plane_chunk(slots + ((st.slot_ctr + k) % kNSlot) * kSlotBytes, r, sub);
-        P[0][k] = q.x;
-        P[1][k] = q.y;
-        P[2][k] = q.z;
-        P[3][k] = q.w;
-      }
-      if (sub == 1) {
+    for (int k = 0; k < B; ++k) mbar_arrive(&pe[(st.slot_ctr + k) % kNSlot]);
+    const uint32_t a_idx = 2u * st.a_ctr + static_cast<uint32_t>(grp);
+    const uint32_t qa = a_idx % kNA;
+    if (!mbar_wait_warp(&ae[qa], ((a_idx / kNA) & 1u) ^ 1u, ctl)) return false;
+    const uint32_t tcol = tmem_lane + kAColBase + qa * kAColsPerSlot;
 #pragma unroll
-        for (int k = 0; k < B; ++k) mbar_arrive(&pe[(st.slot_ctr + k) % kNSlot]);
+    for (int h = 0; h < 2; ++h) {
+      uint32_t out[32];
+      if constexpr (B <= 3) {
+        dq::dq_word_reg<B>(P[2 * h], L, out);
+        dq::dq_word_reg<B>(P[2 * h + 1], L, out + 16);
+      } else if constexpr (B <= 7) {
+        dq::dq_word_smem<B>(P[2 * h], r4, lds, out);
+        dq::dq_word_smem<B>(P[2 * h + 1], r4, lds, out + 16);
+      } else {
+        dq_word8(P[2 * h], r4, out);
+        dq_word8(P[2 * h + 1], r4, out + 16);
       }
-      const uint32_t qa = st.a_ctr % kNA;
-      if (!mbar_wait_warp(&ae[qa], ((st.a_ctr / kNA) & 1u) ^ 1u, ctl)) return false;
-      const uint32_t tcol = tmem_a_lane + kAColBase + qa * kAColsPerSlot;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t out[32];
-        dequant_word<B>(P[2 * half], lrow, out);
-        dequant_word<B>(P[2 * half + 1], lrow, out + 16);
-        tmem_st32(tcol + 32 * half, out);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&af[qa]);
-      st.a_ctr++;
+      tmem_st32(tcol + 32 * h, out);
     }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&af[qa]);
+    st.a_ctr++;
     st.slot_ctr += B;
   }
   return true;
 }
 
+// This thread's share of a pass's LUT: b <= 3 goes to registers (both
+// threads of a row load it), wider tables to shared memory, each of the two
+// threads of a row writing half of the words.
+__device__ void load_lut(const Item& it, const Pass& ps, int grp, int r, dq::RegLut& L) {
+  const int o = it.row0 + r;
+  if (o >= it.rows) return;
+  const int b = ps.bits;
+  const uint16_t* row = ps.lut + (static_cast<size_t>(o) << b);
+  if (b <= 3) {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(row);
+    for (int i = 0; i < (1 << b) / 2; ++i) w[i] = src[i];
+    L = dq::make_reg_lut<3>(w);
+    return;
+  }
+  uint32_t* dst = reinterpret_cast<uint32_t*>(pw_tc_smem + kOffLut + 4u * r);
+  if (b == 8) {
+    // packed: word j (entries 2j, 2j+1) at (j << 9) | 4r; this thread's 64 words
+    const uint4* src = reinterpret_cast<const uint4*>(row) + grp * 16;
+    for (int i = 0; i < 16; ++i) {
+      const uint4 v = src[i];
+      const uint32_t j = static_cast<uint32_t>(grp * 64 + 4 * i);
+      dst[(j + 0) * 128] = v.x;
+      dst[(j + 1) * 128] = v.y;
+      dst[(j + 2) * 128] = v.z;
+      dst[(j + 3) * 128] = v.w;
+    }
+    return;
+  }
+  const int half = 1 << (b - 1);
+  const uint4* src = reinterpret_cast<const uint4*>(row + grp * half);
+  for (int i = 0; i < half / 8; ++i) {
+    const uint4 v = src[i];
+    const uint32_t e4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t ent = (e & 1) ? (e4[e >> 1] >> 16) : (e4[e >> 1] & 0xFFFFu);
+      dst[(grp * half + 8 * i + e) * 128] = ent;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- token tiles
+// Linear mode: the activations are bf16 in natural column order; convert,
+// permute into the A slots' K order and store (generic stores; the caller
+// fences).  Stage s, token rows 0..ntok-1, this lane's share.
+__device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t buf, int lane) {
+  for (int idx = lane; idx < it.ntok * kStageWords; idx += 32) {
+    const int n = idx >> 3, w = idx & 7;
+    const int col0 = s * 256 + 32 * w;
+    const uint16_t* src = p.x + static_cast<size_t>(it.tok0 + n) * p.lin_cols;
+    float v[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const int col = col0 + c;
+      v[c] = (col < it.cols) ? bf16f(src[col]) : 0.0f;
+    }
+    uint32_t q16[16];
+#pragma unroll
+    for (int pr = 0; pr < 16; ++pr)
+      q16[pr] = pack_h2(v[dq::col_of_kpos(2 * pr)], v[dq::col_of_kpos(2 * pr + 1)]);
+#pragma unroll
+    for (int qc = 0; qc < 4; ++qc) {
+      const uint32_t dst = buf + b_chunk_off(n, 4 * w + qc);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(q16[4 * qc]),
+                   "r"(q16[4 * qc + 1]), "r"(q16[4 * qc + 2]), "r"(q16[4 * qc + 3])
+                   : "memory");
+    }
+  }
+}
+
+// Gate/up and down modes: rows are fp16 in the A slots' K order already
+// (x_perm by token, h_perm by sorted position), zero past the row's end;
+// copy the stage's 512 bytes of every token row asynchronously.
+__device__ void issue_b_copies(const TcParams& p, const Item& it, int s, uint32_t buf, int lane) {
+  const int chunks = it.ntok * 32;
+  for (int idx = lane; idx < chunks; idx += 32) {
+    const int n = idx >> 5, c16 = idx & 31;
+    const uint16_t* row;
+    if (p.mode == kTcGateUp) {
+      row = p.x_perm + static_cast<size_t>(p.slot_token[it.pos0 + n]) * p.x_perm_ld;
+    } else {
+      row = p.h_perm + static_cast<size_t>(it.pos0 + n) * p.h_perm_ld;
+    }
+    cp_async16(buf + b_chunk_off(n, c16), row + s * 256 + c16 * 8);
+  }
+}
+
 // ---------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__ TcParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* slots = base;
-  uint8_t* bbuf = slots + kSmemSlots;
-  uint32_t* lut = reinterpret_cast<uint32_t*>(bbuf + kSmemB);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(lut) + kSmemLut);
+  uint8_t* smem = pw_tc_smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* pf = bars;
   uint64_t* pe = pf + kNSlot;
   uint64_t* bfull = pe + kNSlot;
-  uint64_t* bempty = bfull + 2;
-  uint64_t* af = bempty + 2;
+  uint64_t* bempty = bfull + kNB;
+  uint64_t* af = bempty + kNB;
   uint64_t* ae = af + kNA;
   uint64_t* df = ae + kNA;
   uint64_t* de = df + 2;
   uint64_t* drain = de + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* s_prefix = reinterpret_cast<int*>(tmem_holder + 4);
+  uint64_t* dqbar = drain + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  int* s_prefix = reinterpret_cast<int*>(smem + kOffMisc + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -477,11 +513,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNSlot; ++i) {
       mbar_init(&pf[i], 1);
-      mbar_init(&pe[i], 128);
+      mbar_init(&pe[i], kDqThreads);
+    }
+    for (int i = 0; i < kNB; ++i) {
+      mbar_init(&bfull[i], 32);
+      mbar_init(&bempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bfull[i], 128);
-      mbar_init(&bempty[i], 1);
       mbar_init(&df[i], 1);
       mbar_init(&de[i], 128);
     }
@@ -490,24 +528,25 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       mbar_init(&ae[i], 1);
     }
     mbar_init(drain, 1);
-    *s_abort = 0;
-    // items per group: projections x row tiles x token tiles x K splits
+    mbar_init(dqbar, kDqThreads);
+    // the table offsets assume a 1024-byte aligned dynamic shared memory base
+    *s_abort = (smem_addr(smem) & 1023u) ? 1 : 0;
+    if (*s_abort && p.err) atomicExch(p.err, PW_ERR_UNSUPPORTED);
+    // items per group: row tiles x token tiles x K splits
     int acc = 0;
     for (int g = 0; g < G; ++g) {
       s_prefix[g] = acc;
-      int rows, n, nproj;
+      int rows, n;
       if (p.mode == kTcLinear) {
         rows = p.lin_rows;
         n = p.T;
-        nproj = 1;
       } else {
         const int Fg = (g == p.E) ? p.S : p.F;
         rows = (p.mode == kTcGateUp) ? Fg : p.H;
-        nproj = (p.mode == kTcGateUp) ? 2 : 1;
         n = p.offsets[g + 1] - p.offsets[g];
       }
       const int tt = (n + kNT - 1) / kNT;
-      acc += nproj * ((rows + kTileRows - 1) / kTileRows) * tt * p.n_split;
+      acc += ((rows + kTileRows - 1) / kTileRows) * tt * p.n_split;
     }
     s_prefix[G] = acc;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -522,58 +561,66 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int total = s_prefix[G];
+  const int total = *s_abort ? 0 : s_prefix[G];
   const Ctl ctl{s_abort, p.err};
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------ dequantisers
-    DequantState st{0u, 0u, 0u};
-    const int r = threadIdx.x;
-    const uint32_t* lrow = lut + r;
-    const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
-    for (int i = blockIdx.x; i < total && !__any_sync(0xffffffffu, *s_abort != 0);
-         i += gridDim.x) {
+    DequantState st{0u, 0u};
+    const int grp = warp >> 2, quad = warp & 3;
+    const int r = 32 * quad + lane;
+    uint32_t sync_phase = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
       Item it;
       decode_item(p, s_prefix, G, i, it);
-      // this thread's LUT row
-      const int o = it.row0 + r;
-      if (o < it.rows) {
-        const uint32_t* src = reinterpret_cast<const uint32_t*>(it.lut) +
-                              (static_cast<size_t>(o) << (it.bits - 1));
-        const int nw = 1 << (it.bits - 1);
-        for (int j = 0; j < nw; ++j) lut[j * kTileRows + r] = src[j];
+      for (int q = 0; q < it.npass && ok; ++q) {
+        const Pass& ps = it.pass[q];
+        // every thread is done with the previous pass's table before it changes
+        if (!dq_sync(dqbar, sync_phase, ctl)) {
+          ok = false;
+          break;
+        }
+        dq::RegLut L{0u, 0u, 0u, 0u};
+        load_lut(it, ps, grp, r, L);
+        if (!dq_sync(dqbar, sync_phase, ctl)) {
+          ok = false;
+          break;
+        }
+        switch (ps.bits) {
+          case 1: ok = dequant_stages<1>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          case 2: ok = dequant_stages<2>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          case 3: ok = dequant_stages<3>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          case 4: ok = dequant_stages<4>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          case 5: ok = dequant_stages<5>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          case 6: ok = dequant_stages<6>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          case 7: ok = dequant_stages<7>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+          default: ok = dequant_stages<8>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        }
       }
-      bool ok = true;
-      switch (it.bits) {
-        case 1: ok = dequant_stages<1>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        case 2: ok = dequant_stages<2>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        case 3: ok = dequant_stages<3>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        case 4: ok = dequant_stages<4>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        case 5: ok = dequant_stages<5>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        case 6: ok = dequant_stages<6>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        case 7: ok = dequant_stages<7>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-        default: ok = dequant_stages<8>(p, it, slots, bbuf, lrow, pf, pe, bfull, bempty, af, ae, tmem_lane, st, ctl); break;
-      }
-      if (!ok) break;
     }
-  } else if (warp == 4) {
-    // ------------------------------------------------ TMA producer
+  } else if (warp == kWarpProducer) {
+    // ------------------------------------------------ TMA producer (planes)
     if (lane == 0) {
       uint32_t slot_ctr = 0;
       bool ok = true;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
         decode_item(p, s_prefix, G, i, it);
-        for (int s = it.s_begin; s < it.s_end && ok; ++s) {
-          for (int k = 0; k < it.bits; ++k) {
-            const uint32_t sl = slot_ctr % kNSlot;
-            if (!mbar_wait(&pe[sl], ((slot_ctr / kNSlot) & 1u) ^ 1u, ctl)) {
-              ok = false;
-              break;
+        for (int q = 0; q < it.npass && ok; ++q) {
+          const Pass& ps = it.pass[q];
+          for (int s = it.s_begin; s < it.s_end && ok; ++s) {
+            for (int k = 0; k < ps.bits; ++k) {
+              const uint32_t sl = slot_ctr % kNSlot;
+              if (!mbar_wait(&pe[sl], ((slot_ctr / kNSlot) & 1u) ^ 1u, ctl)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_tx(&pf[sl], kSlotBytes);
+              tma_load_3d(smem_addr(smem + kOffSlots + sl * kSlotBytes), ps.tmap,
+                          s * kStageWords, it.row0, k, &pf[sl]);
+              slot_ctr++;
             }
-            mbar_arrive_tx(&pf[sl], kSlotBytes);
-            tma_load_3d(slots + sl * kSlotBytes, it.tmap, s * kStageWords, it.row0, k, &pf[sl]);
-            slot_ctr++;
           }
         }
       }
@@ -583,7 +630,47 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         for (uint32_t c = lo; c < slot_ctr; ++c) mbar_drain(&pf[c % kNSlot], (c / kNSlot) & 1u);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpLoader) {
+    // ------------------------------------------------ token-tile loader
+    // Each stage's copies are committed as one group; a stage is published
+    // (its group complete, a proxy fence, an arrive) once the next stage has
+    // been issued, so two stages are in flight.
+    uint32_t b_ctr = 0, pending = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+      Item it;
+      decode_item(p, s_prefix, G, i, it);
+      for (int q = 0; q < it.npass && ok; ++q) {
+        for (int s = it.s_begin; s < it.s_end; ++s) {
+          const uint32_t jb = b_ctr % kNB;
+          if (!mbar_wait_warp(&bempty[jb], ((b_ctr / kNB) & 1u) ^ 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t buf = smem_addr(smem + kOffB + jb * kBStageBytes);
+          if (p.mode == kTcLinear) {
+            fill_b_linear(p, it, s, buf, lane);
+          } else {
+            issue_b_copies(p, it, s, buf, lane);
+          }
+          cp_async_commit();
+          b_ctr++;
+          pending++;
+          if (pending == 2) {
+            cp_async_wait<1>();
+            fence_proxy_async();
+            mbar_arrive(&bfull[(b_ctr - 2) % kNB]);
+            pending = 1;
+          }
+        }
+      }
+    }
+    cp_async_wait<0>();
+    if (pending == 1) {
+      fence_proxy_async();
+      mbar_arrive(&bfull[(b_ctr - 1) % kNB]);
+    }
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t a_ctr = 0, b_ctr = 0, d_ctr = 0;
@@ -596,37 +683,39 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         const uint32_t jd = d_ctr & 1u;
         if (!mbar_wait(&de[jd], ((d_ctr >> 1) & 1u) ^ 1u, ctl)) break;
         tc_fence_after();
-        const uint32_t dt = tmem_base + jd * kDColsPerBuf;
-        uint32_t accum = 0;
-        for (int s = it.s_begin; s < it.s_end && ok; ++s) {
-          const uint32_t jb = b_ctr & 1u;
-          if (!mbar_wait(&bfull[jb], (b_ctr >> 1) & 1u, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t bbase = smem_addr(bbuf + jb * kBStageBytes);
-          for (int sub = 0; sub < 2; ++sub) {
-            const uint32_t qa = a_ctr % kNA;
-            if (!mbar_wait(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
+        for (int q = 0; q < it.npass && ok; ++q) {
+          const uint32_t dt = tmem_base + jd * kDColsPerBuf + 32 * q;
+          uint32_t accum = 0;
+          for (int s = it.s_begin; s < it.s_end && ok; ++s) {
+            const uint32_t jb = b_ctr % kNB;
+            if (!mbar_wait(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t at = tmem_base + kAColBase + qa * kAColsPerSlot;
+            const uint32_t bbase = smem_addr(smem + kOffB + jb * kBStageBytes);
+            for (int sub = 0; sub < 2; ++sub) {
+              const uint32_t qa = a_ctr % kNA;
+              if (!mbar_wait(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t at = tmem_base + kAColBase + qa * kAColsPerSlot;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const int kp = sub * 128 + kk * 16;
-              const uint32_t baddr = bbase + (kp >> 6) * (kNT * 128) + (kp & 63) * 2;
-              tc_mma(dt, at + kk * 8, smem_desc_sw128(baddr), idesc, accum);
-              accum = 1;
+              for (int kk = 0; kk < 8; ++kk) {
+                const int kp = sub * 128 + kk * 16;
+                const uint32_t baddr = bbase + (kp >> 6) * (kNT * 128) + (kp & 63) * 2;
+                tc_mma(dt, at + kk * 8, smem_desc_sw128(baddr), idesc, accum);
+                accum = 1;
+              }
+              tc_commit(&ae[qa]);
+              a_ctr++;
             }
-            tc_commit(&ae[qa]);
-            a_ctr++;
+            if (!ok) break;
+            tc_commit(&bempty[jb]);
+            b_ctr++;
           }
-          if (!ok) break;
-          tc_commit(&bempty[jb]);
-          b_ctr++;
         }
         if (!ok) break;
         tc_commit(&df[jd]);
@@ -647,23 +736,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       const uint32_t jd = d_ctr & 1u;
       if (!mbar_wait_warp(&df[jd], (d_ctr >> 1) & 1u, ctl)) break;
       tc_fence_after();
-      uint32_t v[32];
+      uint32_t v[32], u[32];
       tmem_ld32(tmem_lane + jd * kDColsPerBuf, v);
+      if (it.npass == 2) tmem_ld32(tmem_lane + jd * kDColsPerBuf + 32, u);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&de[jd]);
       d_ctr++;
       const int o = it.row0 + 32 * qd + lane;
       if (o < it.rows) {
-        for (int n = 0; n < it.ntok; ++n) {
-          const float acc = __uint_as_float(v[n]);
-          if (p.mode == kTcGateUp) {
-            p.gu[static_cast<size_t>(it.pos0 + n) * p.gu_stride + it.proj * it.rows + o] = acc;
-          } else if (p.mode == kTcDown) {
+        if (p.mode == kTcGateUp) {
+          // h = silu(g) * u, fp16, at o's position in the down pass's K order
+          const size_t col = static_cast<size_t>(o & ~31) + dq::kpos_of_col(o & 31);
+#pragma unroll
+          for (int n = 0; n < kNT; ++n) {
+            if (n >= it.ntok) break;
+            const float g = __uint_as_float(v[n]);
+            const float h = g / (1.0f + expf(-g)) * __uint_as_float(u[n]);
+            p.h_perm[static_cast<size_t>(it.pos0 + n) * p.h_perm_ld + col] =
+                __half_as_ushort(__float2half_rn(h));
+          }
+        } else if (p.mode == kTcDown) {
+#pragma unroll
+          for (int n = 0; n < kNT; ++n) {
+            if (n >= it.ntok) break;
             p.ysorted[it.split * p.split_stride + static_cast<size_t>(it.pos0 + n) * p.H + o] =
-                p.slot_w[it.pos0 + n] * acc;
-          } else {
-            p.y[static_cast<size_t>(it.tok0 + n) * it.rows + o] = acc;
+                p.slot_w[it.pos0 + n] * __uint_as_float(v[n]);
+          }
+        } else {
+#pragma unroll
+          for (int n = 0; n < kNT; ++n) {
+            if (n >= it.ntok) break;
+            p.y[static_cast<size_t>(it.tok0 + n) * it.rows + o] = __uint_as_float(v[n]);
           }
         }
       }

@@ -8,8 +8,8 @@
 namespace pw {
 
 constexpr int kTcTokens = 32;  // token tile of one work item (MMA N <= 32)
-constexpr int kTcGateUp = 0;   // gate and up blocks of every group -> gu
-constexpr int kTcDown = 1;     // down blocks, B = silu(g) * u -> routing-weighted partials
+constexpr int kTcGateUp = 0;   // gate and up blocks of every group -> h = silu(g) * u
+constexpr int kTcDown = 1;     // down blocks, B = h -> routing-weighted partials
 constexpr int kTcLinear = 2;   // one standalone block -> y
 
 struct TcParams {
@@ -22,9 +22,11 @@ struct TcParams {
   const int32_t* offsets;        // [G+1] sorted-position ranges per group
   const int32_t* slot_token;
   const float* slot_w;
-  const uint16_t* x;             // bf16 activations (modes 0, 2)
-  float* gu;                     // [P][gu_stride]: gate | up per sorted position
-  int gu_stride;
+  const uint16_t* x;             // bf16 activations [T][lin_cols] (mode 2)
+  const uint16_t* x_perm;        // fp16 activations in the A K order, [T][x_perm_ld] (mode 0)
+  int x_perm_ld;
+  uint16_t* h_perm;              // fp16 silu(g)*u in the A K order, [P][h_perm_ld]
+  int h_perm_ld;                 // (written by mode 0, read by mode 1; zero past F)
   float* ysorted;                // [n_split][P][H]
   long long split_stride;        // floats between split partial buffers
   float* y;                      // [T][lin_rows] (mode 2)

@@ -50,10 +50,11 @@
  *   error nothing has been enqueued, unless the status is PW_ERR_CUDA.
  *   Threads: a handle is used by one host thread at a time.
  *   Alignment: device buffers 16-byte aligned; x and y row-major, contiguous.
- *   Kernels: a pass whose blocks have ceil(cols/32) % 4 == 0 and cols % 8 == 0
- *   runs on the tensor-core kernel (TMA + tcgen05; activations are fed to it
- *   as fp16, so |x| and |silu(g) u| must stay below 65504); other shapes run
- *   on the CUDA-core kernel in fp32.
+ *   Kernels: when H, F and S are multiples of 128 the expert passes run on the
+ *   tensor-core kernel (TMA + tcgen05; activations are fed to it as fp16, so
+ *   |x| and |silu(g) u| must stay below 65504); other shapes run on the
+ *   CUDA-core kernel in fp32.  pw_linear takes the tensor-core kernel when
+ *   cols is a multiple of 128.
  */
 #ifndef PW_H_
 #define PW_H_
