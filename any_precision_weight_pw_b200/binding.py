@@ -22,7 +22,8 @@ STATUS = {0: "PW_OK", 1: "PW_ERR_INVALID_ARG", 2: "PW_ERR_CUDA", 3: "PW_ERR_OOM"
 EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy",
             "pw_moe_forward_host", "pw_linear", "pw_get_block_bits", "pw_get_routing",
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
-            "pw_forward_launches", "pw_last_error", "pw_abi_version"]
+            "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_last_error",
+            "pw_abi_version"]
 
 
 class PwError(RuntimeError):
@@ -67,10 +68,14 @@ def lib():
         L.pw_profile_read.argtypes = [P, C.POINTER(C.c_float), i32, C.POINTER(i32)]
         L.pw_forward_launches.argtypes = [P, i32]
         L.pw_forward_launches.restype = i32
+        L.pw_plane_bytes.argtypes = [i32, i32]
+        L.pw_plane_bytes.restype = C.c_int64
+        L.pw_repack_planes.argtypes = [P, P, i32, i32, i32, P]
         L.pw_last_error.restype = C.c_char_p
         L.pw_abi_version.restype = i32
         for name in EXPORTED:
-            if name not in ("pw_forward_launches", "pw_last_error", "pw_abi_version"):
+            if name not in ("pw_forward_launches", "pw_last_error", "pw_abi_version",
+                            "pw_plane_bytes"):
                 getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -91,12 +96,26 @@ def _stream(stream) -> Optional[int]:
     return s.cuda_stream
 
 
-def linear(planes, lut, bits: int, x, y=None, stream=None):
-    """y[t][o] = sum_i W_b[o][i] x[t][i] for one block.  planes: int32 tensor
-    [>=bits][rows][words] (uint32 bit patterns); lut: int16 [rows][2^bits]
-    (fp16 bit patterns); x: bf16 [T][cols].  Returns fp32 [T][rows]."""
+def plane_bytes(rows: int, cols: int) -> int:
+    """Bytes of one plane page of a rows x cols block."""
+    return int(lib().pw_plane_bytes(rows, cols))
+
+
+def repack_planes(planes, cols: int, stream=None):
+    """Row-major planes (int32 device tensor [n][rows][ceil(cols/32)], uint32
+    bit patterns) -> plane pages (int32 device tensor [n][plane_bytes / 4])."""
     import torch
-    rows = planes.shape[1]
+    n, rows, _ = planes.shape
+    out = torch.empty((n, plane_bytes(rows, cols) // 4), dtype=torch.int32, device=planes.device)
+    check(lib().pw_repack_planes(_ptr(planes), _ptr(out), rows, cols, n, _stream(stream)))
+    return out
+
+
+def linear(planes, lut, bits: int, x, rows: int, y=None, stream=None):
+    """y[t][o] = sum_i W_b[o][i] x[t][i] for one block.  planes: plane pages
+    (repack_planes) of at least `bits` planes; lut: int16 [rows][2^bits] (fp16
+    bit patterns); x: bf16 [T][cols].  Returns fp32 [T][rows]."""
+    import torch
     T, cols = x.shape
     if y is None:
         y = torch.empty((T, rows), dtype=torch.float32, device=x.device)
@@ -202,16 +221,17 @@ def upload_synth_layer(layer, max_tokens: int, host_copies: bool = False,
     wl = layer.wl
     planes, slots, hp, hl = [], [], [], []
     for blk in range(wl.n_blocks):
-        rows, _ = layer.shape(blk)
+        rows, cols = layer.shape(blk)
         pl = layer.planes(blk)
-        planes.append(torch.from_numpy(pl.view(np.int32)).to(device))
+        paged = repack_planes(torch.from_numpy(pl.view(np.int32)).to(device), cols)
+        planes.append(paged)
         s0 = torch.zeros(rows << wl.n_max, dtype=torch.int16, device=device)
         s1 = torch.zeros(rows << wl.n_max, dtype=torch.int16, device=device)
         lt = layer.lut(blk, layer.bits[blk])
         s0[: lt.size].copy_(torch.from_numpy(lt.reshape(-1).view(np.int16)))
         slots.append((s0, s1))
         if host_copies:
-            hp.append(torch.from_numpy(pl.view(np.int32)).pin_memory())
+            hp.append(paged.cpu().pin_memory())
             hl.append({b: torch.from_numpy(layer.lut(blk, b).reshape(-1).view(np.int16)).pin_memory()
                        for b in range(1, wl.n_max + 1)})
     cfg = dict(hidden=wl.hidden, ffn=wl.ffn, n_experts=wl.n_experts, top_k=wl.top_k,

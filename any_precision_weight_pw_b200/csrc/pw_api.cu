@@ -18,6 +18,7 @@
 #include <string>
 #include <vector>
 
+#include "pages.h"
 #include "pw_internal.h"
 #include "tc.h"
 
@@ -72,21 +73,19 @@ EncodeTiledFn encode_fn() {
 // activations in whole 32-column groups: it takes cols % 128 == 0.
 bool tc_shape_ok(int cols) { return cols % 128 == 0; }
 
-pw_status_t make_plane_map(CUtensorMap* m, const uint32_t* planes, int n_planes, int rows,
-                           int cols) {
+// 2-D map over an fp16 row buffer [rows][ld] for the token tiles: boxes of
+// 64 columns x 8 rows with the 128-byte swizzle of the MMA's K-major operand.
+pw_status_t make_row_map(CUtensorMap* m, const uint16_t* base, int ld, int rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const int words = (cols + 31) / 32;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(n_planes)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(words) * 4,
-                           static_cast<cuuint64_t>(words) * 4 * rows};
-  cuuint32_t box[3] = {8, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(planes), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, 8};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled (rows) failed (%d)", (int)r);
   return PW_OK;
 }
 
@@ -118,12 +117,12 @@ struct pw_moe {
   // workspace
   pw::RouteWorkspace ws{};
   float* gu = nullptr;          // CUDA-core path: gate | up per sorted position
-  uint16_t* x_perm = nullptr;   // tensor-core path: fp16 activations, K-permuted
+  uint16_t* x_sorted = nullptr; // tensor-core path: gathered fp16 activations, K-permuted
   uint16_t* h_perm = nullptr;   // tensor-core path: fp16 silu(g) * u, K-permuted
-  int x_perm_ld = 0, h_perm_ld = 0;
+  int x_ld = 0, h_perm_ld = 0;
+  CUtensorMap x_map, h_map;     // 2-D TMA maps over x_sorted and h_perm
   float* ysorted = nullptr;
   int* err = nullptr;
-  CUtensorMap* d_tmaps = nullptr;
   uint16_t* stage_x = nullptr;
   uint16_t* stage_y = nullptr;
   int P_max = 0, gu_stride = 0, max_split = 8, last_T = 0;
@@ -255,7 +254,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
           env_int("PW_FORCE_SIMPLE", 0) == 0;
   h->gu_stride = h->tc ? 0 : 2 * Fmax;
   // rows padded to whole 256-column stages, zero past the end
-  h->x_perm_ld = h->tc ? (c.hidden + 255) / 256 * 256 : 0;
+  h->x_ld = h->tc ? (c.hidden + 255) / 256 * 256 : 0;
   h->h_perm_ld = h->tc ? (Fmax + 255) / 256 * 256 : 0;
   auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
   size_t off = 0;
@@ -268,9 +267,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const size_t o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
   const size_t o_tk = off; off += al(sizeof(uint32_t) * 4);
   const size_t o_err = off; off += al(sizeof(int) * 4);
-  const size_t o_tm = off; off += al(sizeof(CUtensorMap) * n_blocks);
   const size_t o_gu = off; off += al(sizeof(float) * size_t(h->P_max) * h->gu_stride);
-  const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(T) * h->x_perm_ld);
+  const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->x_ld);
   const size_t o_hp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->h_perm_ld);
   const size_t o_ys = off; off += al(sizeof(float) * size_t(h->max_split) * h->P_max * c.hidden);
   const size_t o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
@@ -289,9 +287,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->ws.token_pos = reinterpret_cast<int32_t*>(w + o_tp);
   h->ws.ticket = reinterpret_cast<uint32_t*>(w + o_tk);
   h->err = reinterpret_cast<int*>(w + o_err);
-  h->d_tmaps = reinterpret_cast<CUtensorMap*>(w + o_tm);
   h->gu = reinterpret_cast<float*>(w + o_gu);
-  h->x_perm = reinterpret_cast<uint16_t*>(w + o_xp);
+  h->x_sorted = reinterpret_cast<uint16_t*>(w + o_xp);
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
   h->ysorted = reinterpret_cast<float*>(w + o_ys);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
@@ -301,23 +298,13 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
     free_all(h);
     return fail(PW_ERR_CUDA, "cudaMemset failed");
   }
-  // plane tensor maps for the tensor-core passes
+  // token-tile tensor maps for the tensor-core passes
   if (h->tc) {
-    std::vector<CUtensorMap> maps(n_blocks);
-    for (int i = 0; i < n_blocks; ++i) {
-      std::memset(&maps[i], 0, sizeof(CUtensorMap));
-      if (!tc_shape_ok(h->blk[i].cols)) continue;
-      pw_status_t st = make_plane_map(&maps[i], h->blk[i].d_planes, c.n_max, h->blk[i].rows,
-                                      h->blk[i].cols);
-      if (st != PW_OK) {
-        free_all(h);
-        return st;
-      }
-    }
-    if (cudaMemcpy(h->d_tmaps, maps.data(), sizeof(CUtensorMap) * n_blocks,
-                   cudaMemcpyHostToDevice) != cudaSuccess) {
+    pw_status_t st = make_row_map(&h->x_map, h->x_sorted, h->x_ld, h->P_max);
+    if (st == PW_OK) st = make_row_map(&h->h_map, h->h_perm, h->h_perm_ld, h->P_max);
+    if (st != PW_OK) {
       free_all(h);
-      return fail(PW_ERR_CUDA, "tensor map upload failed");
+      return st;
     }
   }
   *out = h;
@@ -340,7 +327,7 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
     return fail(PW_ERR_INVALID_ARG, "block %d: raising bits needs the host planes", block_id);
   cudaStream_t s = static_cast<cudaStream_t>(side_stream);
   if (h->any_forward) PW_CUDA(cudaStreamWaitEvent(s, h->fwd_done, 0));
-  const size_t plane_elems = static_cast<size_t>(b.rows) * ((b.cols + 31) / 32);
+  const size_t plane_elems = static_cast<size_t>(pw::pages::plane_words(b.rows, b.cols));
   if (new_bits > b.bits) {
     PW_CUDA(cudaMemcpyAsync(b.d_planes + b.bits * plane_elems, b.h_planes + b.bits * plane_elems,
                             sizeof(uint32_t) * plane_elems * (new_bits - b.bits),
@@ -422,18 +409,24 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   rp.k = c.top_k;
   rp.renorm = c.renorm_topk;
   rp.has_shared = has_shared;
-  rp.x_perm = h->tc ? h->x_perm : nullptr;
-  rp.x_perm_ld = h->x_perm_ld;
   rp.ws = h->ws;
   PW_CUDA(pw::launch_route(rp, h->n_sm, s));
   PW_CUDA(mark(1));
 
   // gate/up pass
   if (h->tc) {
+    pw::GatherParams gp{};
+    gp.x = d_x;
+    gp.offsets = h->ws.offsets;
+    gp.slot_token = h->ws.slot_token;
+    gp.x_sorted = h->x_sorted;
+    gp.H = c.hidden;
+    gp.ld = h->x_ld;
+    gp.n_groups = h->G;
+    PW_CUDA(pw::launch_gather(gp, T * c.top_k + (c.shared_ffn > 0 ? T : 0), h->n_sm, s));
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
-    tp.tmaps = h->d_tmaps;
     tp.mode = pw::kTcGateUp;
     tp.H = c.hidden;
     tp.F = c.ffn;
@@ -444,8 +437,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.offsets = h->ws.offsets;
     tp.slot_token = h->ws.slot_token;
     tp.slot_w = h->ws.slot_w;
-    tp.x_perm = h->x_perm;
-    tp.x_perm_ld = h->x_perm_ld;
+    tp.b_map = h->x_map;
     tp.h_perm = h->h_perm;
     tp.h_perm_ld = h->h_perm_ld;
     tp.err = h->err;
@@ -477,7 +469,6 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
-    tp.tmaps = h->d_tmaps;
     tp.mode = pw::kTcDown;
     tp.H = c.hidden;
     tp.F = c.ffn;
@@ -488,6 +479,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.offsets = h->ws.offsets;
     tp.slot_token = h->ws.slot_token;
     tp.slot_w = h->ws.slot_w;
+    tp.b_map = h->h_map;
     tp.h_perm = h->h_perm;
     tp.h_perm_ld = h->h_perm_ld;
     tp.ysorted = h->ysorted;
@@ -576,8 +568,6 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
   if (tc_shape_ok(cols) && env_int("PW_FORCE_SIMPLE", 0) == 0) {
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
-    pw_status_t st = make_plane_map(&tp.lin_map, d_planes, bits, rows, cols);
-    if (st != PW_OK) return st;
     tp.mode = pw::kTcLinear;
     tp.n_groups = 1;
     tp.n_split = 1;
@@ -588,6 +578,7 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
     tp.lin_cols = cols;
     tp.lin_bits = bits;
     tp.lin_lut = d_lut;
+    tp.lin_planes = d_planes;
     tp.err = nullptr;
     PW_CUDA(pw::launch_tc(tp, n_sm, s));
   } else {
@@ -604,6 +595,21 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
     sp.lin_lut = d_lut;
     PW_CUDA(pw::launch_simple(sp, rows, s));
   }
+  return PW_OK;
+}
+
+int64_t pw_plane_bytes(int32_t rows, int32_t cols) {
+  if (rows < 1 || cols < 1) return 0;
+  return pw::pages::plane_words(rows, cols) * 4;
+}
+
+pw_status_t pw_repack_planes(const uint32_t* d_src, uint32_t* d_dst, int32_t rows, int32_t cols,
+                             int32_t n_planes, pw_stream_t stream) {
+  if (!d_src || !d_dst || rows < 1 || cols < 1 || n_planes < 1 || n_planes > PW_MAX_BITS)
+    return fail(PW_ERR_INVALID_ARG, "bad repack arguments");
+  if (!aligned16(d_src) || !aligned16(d_dst))
+    return fail(PW_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+  PW_CUDA(pw::launch_repack(d_src, d_dst, rows, cols, n_planes, static_cast<cudaStream_t>(stream)));
   return PW_OK;
 }
 
@@ -657,7 +663,7 @@ pw_status_t pw_profile_read(pw_moe_t* h, float* ms, int32_t n, int32_t* n_forwar
 
 int32_t pw_forward_launches(const pw_moe_t* h, int32_t T) {
   if (!h) return 0;
-  return T > 0 ? 4 : 0;
+  return T > 0 ? (h->tc ? 5 : 4) : 0;
 }
 
 pw_status_t pw_destroy(pw_moe_t* h) {

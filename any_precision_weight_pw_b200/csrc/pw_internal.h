@@ -17,7 +17,7 @@ constexpr int kMaxGroups = PW_MAX_EXPERTS + 1;  // routed experts + shared
 // the kernel parameters, so a forward keeps the table it was launched with
 // while the host moves on to the next one.
 struct BlockRef {
-  const uint32_t* planes;  // [n_max][rows][words]
+  const uint32_t* planes;  // n_max plane pages (layout: pages.h)
   const uint16_t* lut;     // [rows][2^bits] fp16 bits
 };
 
@@ -43,12 +43,18 @@ struct RouteWorkspace {
 
 struct RouteParams {
   const uint16_t* x;       // bf16 [T][H]
-  uint16_t* x_perm;        // fp16 [T][x_perm_ld] in the tensor-core K order, or null
-  int x_perm_ld;
   const float* wr;         // [E][H]
   const float* bias;       // [E] or null
   int T, H, E, k, renorm, has_shared;
   RouteWorkspace ws;
+};
+
+struct GatherParams {
+  const uint16_t* x;         // bf16 [T][H]
+  const int32_t* offsets;    // [n_groups+1]
+  const int32_t* slot_token; // [P]
+  uint16_t* x_sorted;        // fp16 [P][ld], tensor-core K order
+  int H, ld, n_groups;
 };
 
 struct CombineParams {
@@ -81,6 +87,9 @@ struct SimpleParams {
 
 // Launchers (defined in the .cu files).
 cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s);
+cudaError_t launch_repack(const uint32_t* src, uint32_t* dst, int rows, int cols, int n_planes,
+                          cudaStream_t s);
+cudaError_t launch_gather(const GatherParams& p, int max_rows, int n_sm, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_simple(const SimpleParams& p, int grid_rows, cudaStream_t s);
 

@@ -36,41 +36,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   const int E = p.E, H = p.H, T = p.T, k = p.k;
   const RouteWorkspace& ws = p.ws;
 
-  // fp16 copy of the activations in the tensor-core kernel's K order (each
-  // 32-column group permuted like the A operand), one 32-column group per
-  // thread; read by the gate/up pass.
-  if (p.x_perm) {
-    const int groups = T * (H >> 5);
-    for (int idx = blockIdx.x * kRouteThreads + threadIdx.x; idx < groups;
-         idx += gridDim.x * kRouteThreads) {
-      const int t = idx / (H >> 5), w = idx - t * (H >> 5);
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * H + 32 * w);
-      float v[32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 r = src[q];
-        const uint32_t r4[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[8 * q + 2 * e] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] & 0xFFFFu));
-          v[8 * q + 2 * e + 1] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] >> 16));
-        }
-      }
-      uint4* dst = reinterpret_cast<uint4*>(p.x_perm + static_cast<size_t>(t) * p.x_perm_ld + 32 * w);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __half2 h2 = __floats2half2_rn(v[dq::col_of_kpos(8 * q + 2 * e)],
-                                               v[dq::col_of_kpos(8 * q + 2 * e + 1)]);
-          o[e] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
-  }
-
   const int total_pairs = T * E;
   for (int pair = blockIdx.x * warps_per_block + warp; pair < total_pairs;
        pair += gridDim.x * warps_per_block) {
@@ -192,6 +157,44 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   }
 }
 
+// x_sorted[pos] = the activations of token slot_token[pos] as fp16, each
+// 32-column group permuted into the tensor-core kernel's K order; rows are the
+// sorted positions of all groups, so every expert's token tile is contiguous.
+// One 32-column group per thread.
+__global__ void gather_kernel(const GatherParams p) {
+  const int P = p.offsets[p.n_groups];
+  const int wpr = p.H >> 5;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < P * wpr;
+       idx += gridDim.x * blockDim.x) {
+    const int pos = idx / wpr, w = idx - pos * wpr;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        p.x + static_cast<size_t>(p.slot_token[pos]) * p.H + 32 * w);
+    float v[32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 r = src[q];
+      const uint32_t r4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * q + 2 * e] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] & 0xFFFFu));
+        v[8 * q + 2 * e + 1] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] >> 16));
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.x_sorted + static_cast<size_t>(pos) * p.ld + 32 * w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 h2 = __floats2half2_rn(v[dq::col_of_kpos(8 * q + 2 * e)],
+                                             v[dq::col_of_kpos(8 * q + 2 * e + 1)]);
+        o[e] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 // out[t] = sum_j ysorted[pos(t, j)] (+ shared) in slot order, summing the
 // split-K partials of each position in split order; fp32, rounded to bf16.
 __global__ void combine_kernel(const CombineParams p) {
@@ -228,6 +231,15 @@ cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s) {
   if (grid > 4 * n_sm) grid = 4 * n_sm;
   if (grid < 1) grid = 1;
   route_kernel<<<grid, kRouteThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherParams& p, int max_rows, int n_sm, cudaStream_t s) {
+  const int threads = 256;
+  int grid = (max_rows * (p.H >> 5) + threads - 1) / threads;
+  if (grid > 4 * n_sm) grid = 4 * n_sm;
+  if (grid < 1) grid = 1;
+  gather_kernel<<<grid, threads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

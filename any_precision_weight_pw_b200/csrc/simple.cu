@@ -3,14 +3,15 @@
 // One warp per output row: the lanes split the row's 32-column words, unpack
 // the b-bit codes from the top b bit-planes, gather the row's LUT entries and
 // accumulate in fp32 for up to 8 tokens at a time, then reduce across the
-// warp.  This path handles every shape (including blocks whose word count is
-// not a multiple of 4, which the tensor-core path's TMA tiles cannot
-// address) and serves as a second GPU implementation in the tests.
+// warp.  This path handles every shape (the tensor-core path needs widths
+// that are multiples of 128) and serves as a second GPU implementation in the
+// tests.
 //
 // PagedWeight (legiblepapers summary, FAQ Q5): the kernel reads bit-planes
 // and lookup tables directly, with a different bitwidth per linear-block.
 #include <cuda_fp16.h>
 
+#include "pages.h"
 #include "pw_internal.h"
 
 namespace pw {
@@ -76,7 +77,6 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
   const int row0 = blockIdx.x * kRowsPerCta;
   if (row0 >= rows || n_tok <= 0) return;
   const int words = (cols + 31) >> 5;
-  const size_t plane_stride = static_cast<size_t>(rows) * words;
   const int Fg = (mode == 1) ? cols : rows;
 
   for (int tb = 0; tb < n_tok; tb += kTok) {
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
       const uint16_t* lrow = lut + (static_cast<size_t>(o) << bits);
       for (int w = lane; w < words; w += 32) {
         uint32_t pw_[PW_MAX_BITS];
-        for (int k = 0; k < bits; ++k) pw_[k] = planes[k * plane_stride + static_cast<size_t>(o) * words + w];
+        for (int k = 0; k < bits; ++k) pw_[k] = planes[pages::word_index(k, o, w, rows, cols)];
         const int cmax = min(32, cols - 32 * w);
         for (int c = 0; c < cmax; ++c) {
           int code = 0;

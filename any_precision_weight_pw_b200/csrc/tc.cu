@@ -1,5 +1,5 @@
 // tc.cu -- tensor-core dequant-GEMM over Any-Precision bit-plane pages
-// (sm_100a: TMA + cp.async + tcgen05 + TMEM).
+// (sm_100a: TMA + tcgen05 + TMEM).
 //
 // PagedWeight (legiblepapers summary, FAQ Q5; arxivlens abstract): the fused
 // mixed-precision MoE kernel reads the AP bit-planes and per-row LUTs of the
@@ -11,14 +11,19 @@
 // the gate/up item makes a gate pass and an up pass over the same rows (so
 // its epilogue can apply SwiGLU); the down item makes one pass (over one K
 // range when the down pass is split); a standalone linear makes one pass.
-//   warp 8      TMA producer: streams only the b active bit-planes of the
-//               block, 128 rows x 256 columns (8 words) per plane per stage,
-//               into a ring of 4 KB slots (32-byte swizzle, so that the
-//               thread-per-row reads below are bank-conflict free).
-//   warp 10     token-tile loader: cp.async copies of the stage's 256
-//               columns of every token row (fp16, already in the A operand's
-//               K order) into a 4-deep ring, in the K-major 128-byte swizzle
-//               layout of the MMA's B operand; two stages in flight.
+//   warp 8      producer: streams only the b active bit-planes of the block,
+//               128 rows x 256 columns (8 words) per plane per stage, each a
+//               contiguous 4 KB tile of the paged layout (pages.h) moved by
+//               one bulk copy into a ring of 4 KB slots; the tile arrives with
+//               its rows' halves already swizzled, so the thread-per-row reads
+//               below are bank-conflict free.
+//   warp 10     token-tile loader: the item's token rows are contiguous in an
+//               fp16 buffer already in the A operand's K order (the gathered
+//               activations for gate/up, h = silu(g)*u for down), so one lane
+//               streams each stage's 256 columns with 2-D TMA boxes (64
+//               columns x 8 rows, 128-byte swizzle = the MMA's K-major B
+//               layout) into a 4-deep ring.  A standalone linear converts its
+//               bf16 rows with all 32 lanes instead.
 //   warps 0-7   dequantisers in two K halves: warps q and q+4 both own rows
 //               32q..32q+31 (thread <-> output row <-> TMEM lane); the first
 //               group takes columns 0-127 of every stage, the second
@@ -42,6 +47,7 @@
 #include <cuda_fp16.h>
 
 #include "dequant.cuh"
+#include "pages.h"
 #include "pw_internal.h"
 #include "tc.h"
 
@@ -115,8 +121,7 @@ struct Ctl {
 };
 
 // Wait for the phase with the given parity; false on timeout or abort.
-__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const Ctl& c) {
-  if (mbar_try(b, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, const Ctl& c) {
   const unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try(b, parity)) return true;
@@ -127,6 +132,9 @@ __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const Ctl& 
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, const Ctl& c) {
+  return mbar_try(b, parity) || mbar_wait_slow(b, parity, c);
 }
 // The same wait for a whole warp: every lane gets the same answer, so the
 // warp-collective tcgen05 instructions that follow never run on a partial warp.
@@ -141,23 +149,21 @@ __device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
     if (global_ns() - t0 > 200000000ull) return;
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, uint64_t* bar) {
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -248,11 +254,10 @@ __device__ __forceinline__ uint32_t b_chunk_off(int n, int c16) {
 struct Pass {
   int blk, bits;
   const uint16_t* lut;
-  const CUtensorMap* tmap;
+  const uint32_t* planes;  // plane pages (pages.h)
 };
 struct Item {
   int g, row0, tok0, ntok, pos0, split, rows, cols, npass, s_begin, s_end;
-  Pass pass[2];
 };
 
 __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix, int G,
@@ -288,16 +293,14 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
   const int stages = (((it.cols + 31) >> 5) + kStageWords - 1) / kStageWords;
   it.s_begin = static_cast<int>((static_cast<long long>(stages) * it.split) / ns);
   it.s_end = static_cast<int>((static_cast<long long>(stages) * (it.split + 1)) / ns);
-  if (p.mode == kTcLinear) {
-    it.npass = 1;
-    it.pass[0] = Pass{-1, p.lin_bits, p.lin_lut, &p.lin_map};
-  } else {
-    it.npass = (p.mode == kTcGateUp) ? 2 : 1;
-    for (int q = 0; q < it.npass; ++q) {
-      const int blk = 3 * g + ((p.mode == kTcGateUp) ? q : 2);
-      it.pass[q] = Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.tmaps + blk};
-    }
-  }
+  it.npass = (p.mode == kTcGateUp) ? 2 : 1;
+}
+
+// Block, bitwidth, LUT and plane tensor map of pass q of an item.
+__device__ __forceinline__ Pass get_pass(const TcParams& p, const Item& it, int q) {
+  if (p.mode == kTcLinear) return Pass{-1, p.lin_bits, p.lin_lut, p.lin_planes};
+  const int blk = 3 * it.g + ((p.mode == kTcGateUp) ? q : 2);
+  return Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.pt.blk[blk].planes};
 }
 
 // ---------------------------------------------------------------- dequant
@@ -400,22 +403,64 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegL
   return true;
 }
 
-// This thread's share of a pass's LUT: b <= 3 goes to registers (both
-// threads of a row load it), wider tables to shared memory, each of the two
-// threads of a row writing half of the words.
-__device__ void load_lut(const Item& it, const Pass& ps, int grp, int r, dq::RegLut& L) {
+// This thread's share of a pass's LUT.  b <= 3 goes to registers (both
+// threads of a row load the whole row), wider tables to shared memory, each of
+// the two threads of a row writing half of the words.  For b <= 6 the global
+// loads are issued one pass ahead (prefetch) and installed when the pass
+// starts, so their latency hides behind the previous pass; b = 7, 8 tables
+// load when the pass starts.
+struct LutPrefetch {
+  uint4 v[4];
+  int bits;
+  bool live;  // this thread's row exists
+};
+
+__device__ __forceinline__ void lut_prefetch(const Item& it, const Pass& ps, int grp, int r,
+                                             LutPrefetch& f) {
   const int o = it.row0 + r;
-  if (o >= it.rows) return;
+  f.bits = ps.bits;
+  f.live = o < it.rows;
+  if (!f.live || ps.bits > 6) return;
   const int b = ps.bits;
   const uint16_t* row = ps.lut + (static_cast<size_t>(o) << b);
   if (b <= 3) {
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
     const uint32_t* src = reinterpret_cast<const uint32_t*>(row);
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
     for (int i = 0; i < (1 << b) / 2; ++i) w[i] = src[i];
+    f.v[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(row + grp * (1 << (b - 1)));
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (i < (1 << (b - 4))) f.v[i] = src[i];
+}
+
+__device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int grp, int r,
+                                            const LutPrefetch& f, dq::RegLut& L) {
+  if (!f.live) return;
+  const int b = ps.bits;
+  uint32_t* dst = reinterpret_cast<uint32_t*>(pw_tc_smem + kOffLut + 4u * r);
+  if (b <= 3) {
+    const uint32_t w[4] = {f.v[0].x, f.v[0].y, f.v[0].z, f.v[0].w};
     L = dq::make_reg_lut<3>(w);
     return;
   }
-  uint32_t* dst = reinterpret_cast<uint32_t*>(pw_tc_smem + kOffLut + 4u * r);
+  const int half = 1 << (b - 1);
+  if (b <= 6) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i >= (1 << (b - 4))) break;
+      const uint32_t e4[4] = {f.v[i].x, f.v[i].y, f.v[i].z, f.v[i].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t ent = (e & 1) ? (e4[e >> 1] >> 16) : (e4[e >> 1] & 0xFFFFu);
+        dst[(grp * half + 8 * i + e) * 128] = ent;
+      }
+    }
+    return;
+  }
+  const uint16_t* row = ps.lut + (static_cast<size_t>(it.row0 + r) << b);
   if (b == 8) {
     // packed: word j (entries 2j, 2j+1) at (j << 9) | 4r; this thread's 64 words
     const uint4* src = reinterpret_cast<const uint4*>(row) + grp * 16;
@@ -429,7 +474,6 @@ __device__ void load_lut(const Item& it, const Pass& ps, int grp, int r, dq::Reg
     }
     return;
   }
-  const int half = 1 << (b - 1);
   const uint4* src = reinterpret_cast<const uint4*>(row + grp * half);
   for (int i = 0; i < half / 8; ++i) {
     const uint4 v = src[i];
@@ -450,12 +494,23 @@ __device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t
   for (int idx = lane; idx < it.ntok * kStageWords; idx += 32) {
     const int n = idx >> 3, w = idx & 7;
     const int col0 = s * 256 + 32 * w;
-    const uint16_t* src = p.x + static_cast<size_t>(it.tok0 + n) * p.lin_cols;
     float v[32];
+    if (col0 < it.cols) {  // cols is a multiple of 128: whole 32-column groups
+      const uint4* src = reinterpret_cast<const uint4*>(
+          p.x + static_cast<size_t>(it.tok0 + n) * p.lin_cols + col0);
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const int col = col0 + c;
-      v[c] = (col < it.cols) ? bf16f(src[col]) : 0.0f;
+      for (int q = 0; q < 4; ++q) {
+        const uint4 r4 = src[q];
+        const uint32_t e4[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * q + 2 * e] = bf16f(static_cast<uint16_t>(e4[e] & 0xFFFFu));
+          v[8 * q + 2 * e + 1] = bf16f(static_cast<uint16_t>(e4[e] >> 16));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] = 0.0f;
     }
     uint32_t q16[16];
 #pragma unroll
@@ -468,23 +523,6 @@ __device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t
                    "r"(q16[4 * qc + 1]), "r"(q16[4 * qc + 2]), "r"(q16[4 * qc + 3])
                    : "memory");
     }
-  }
-}
-
-// Gate/up and down modes: rows are fp16 in the A slots' K order already
-// (x_perm by token, h_perm by sorted position), zero past the row's end;
-// copy the stage's 512 bytes of every token row asynchronously.
-__device__ void issue_b_copies(const TcParams& p, const Item& it, int s, uint32_t buf, int lane) {
-  const int chunks = it.ntok * 32;
-  for (int idx = lane; idx < chunks; idx += 32) {
-    const int n = idx >> 5, c16 = idx & 31;
-    const uint16_t* row;
-    if (p.mode == kTcGateUp) {
-      row = p.x_perm + static_cast<size_t>(p.slot_token[it.pos0 + n]) * p.x_perm_ld;
-    } else {
-      row = p.h_perm + static_cast<size_t>(it.pos0 + n) * p.h_perm_ld;
-    }
-    cp_async16(buf + b_chunk_off(n, c16), row + s * 256 + c16 * 8);
   }
 }
 
@@ -516,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       mbar_init(&pe[i], kDqThreads);
     }
     for (int i = 0; i < kNB; ++i) {
-      mbar_init(&bfull[i], 32);
+      mbar_init(&bfull[i], p.mode == kTcLinear ? 32 : 1);
       mbar_init(&bempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -571,33 +609,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     const int r = 32 * quad + lane;
     uint32_t sync_phase = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-      Item it;
+    // walk (item, pass) pairs; the next pass's LUT loads are issued before
+    // the current pass's stages
+    int i = blockIdx.x, q = 0;
+    Item it;
+    LutPrefetch pre;
+    if (i < total) {
       decode_item(p, s_prefix, G, i, it);
-      for (int q = 0; q < it.npass && ok; ++q) {
-        const Pass& ps = it.pass[q];
-        // every thread is done with the previous pass's table before it changes
-        if (!dq_sync(dqbar, sync_phase, ctl)) {
-          ok = false;
-          break;
-        }
-        dq::RegLut L{0u, 0u, 0u, 0u};
-        load_lut(it, ps, grp, r, L);
-        if (!dq_sync(dqbar, sync_phase, ctl)) {
-          ok = false;
-          break;
-        }
-        switch (ps.bits) {
-          case 1: ok = dequant_stages<1>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          case 2: ok = dequant_stages<2>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          case 3: ok = dequant_stages<3>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          case 4: ok = dequant_stages<4>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          case 5: ok = dequant_stages<5>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          case 6: ok = dequant_stages<6>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          case 7: ok = dequant_stages<7>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-          default: ok = dequant_stages<8>(it, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        }
+      lut_prefetch(it, get_pass(p, it, 0), grp, r, pre);
+    }
+    while (i < total && ok) {
+      const Pass ps = get_pass(p, it, q);
+      // every thread is done with the previous pass's table before it changes
+      if (!dq_sync(dqbar, sync_phase, ctl)) break;
+      dq::RegLut L{0u, 0u, 0u, 0u};
+      lut_install(it, ps, grp, r, pre, L);
+      if (!dq_sync(dqbar, sync_phase, ctl)) break;
+      const Item cur = it;
+      int ni = i, nq = q + 1;
+      if (nq >= it.npass) {
+        ni = i + gridDim.x;
+        nq = 0;
+        if (ni < total) decode_item(p, s_prefix, G, ni, it);
       }
+      if (ni < total) lut_prefetch(it, get_pass(p, it, nq), grp, r, pre);
+      switch (ps.bits) {
+        case 1: ok = dequant_stages<1>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 2: ok = dequant_stages<2>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 3: ok = dequant_stages<3>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 4: ok = dequant_stages<4>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 5: ok = dequant_stages<5>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 6: ok = dequant_stages<6>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 7: ok = dequant_stages<7>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        default: ok = dequant_stages<8>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+      }
+      i = ni;
+      q = nq;
     }
   } else if (warp == kWarpProducer) {
     // ------------------------------------------------ TMA producer (planes)
@@ -607,8 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
         decode_item(p, s_prefix, G, i, it);
+        const int n_rt = pages::row_tiles(it.rows), n_kt = pages::k_tiles(it.cols);
+        const int rt = it.row0 / kTileRows;
         for (int q = 0; q < it.npass && ok; ++q) {
-          const Pass& ps = it.pass[q];
+          const Pass ps = get_pass(p, it, q);
           for (int s = it.s_begin; s < it.s_end && ok; ++s) {
             for (int k = 0; k < ps.bits; ++k) {
               const uint32_t sl = slot_ctr % kNSlot;
@@ -616,9 +665,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
                 ok = false;
                 break;
               }
+              const int64_t tile = (static_cast<int64_t>(k) * n_rt + rt) * n_kt + s;
               mbar_arrive_tx(&pf[sl], kSlotBytes);
-              tma_load_3d(smem_addr(smem + kOffSlots + sl * kSlotBytes), ps.tmap,
-                          s * kStageWords, it.row0, k, &pf[sl]);
+              bulk_load(smem_addr(smem + kOffSlots + sl * kSlotBytes),
+                        ps.planes + tile * (kSlotBytes / 4), kSlotBytes, &pf[sl]);
               slot_ctr++;
             }
           }
@@ -632,14 +682,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     }
   } else if (warp == kWarpLoader) {
     // ------------------------------------------------ token-tile loader
-    // Each stage's copies are committed as one group; a stage is published
-    // (its group complete, a proxy fence, an arrive) once the next stage has
-    // been issued, so two stages are in flight.
-    uint32_t b_ctr = 0, pending = 0;
+    uint32_t b_ctr = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
       Item it;
       decode_item(p, s_prefix, G, i, it);
+      const int ngrp = (it.ntok + 7) >> 3;  // 8-row groups of the tile
       for (int q = 0; q < it.npass && ok; ++q) {
         for (int s = it.s_begin; s < it.s_end; ++s) {
           const uint32_t jb = b_ctr % kNB;
@@ -650,25 +698,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
           const uint32_t buf = smem_addr(smem + kOffB + jb * kBStageBytes);
           if (p.mode == kTcLinear) {
             fill_b_linear(p, it, s, buf, lane);
-          } else {
-            issue_b_copies(p, it, s, buf, lane);
-          }
-          cp_async_commit();
-          b_ctr++;
-          pending++;
-          if (pending == 2) {
-            cp_async_wait<1>();
             fence_proxy_async();
-            mbar_arrive(&bfull[(b_ctr - 2) % kNB]);
-            pending = 1;
+            mbar_arrive(&bfull[jb]);
+          } else if (lane == 0) {
+            mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(ngrp) * 4u * 1024u);
+            for (int a = 0; a < 4; ++a)
+              for (int j = 0; j < ngrp; ++j)
+                tma_load_2d(buf + a * (kNT * 128) + j * 1024, &p.b_map, s * 256 + a * 64,
+                            it.pos0 + 8 * j, &bfull[jb]);
           }
+          b_ctr++;
         }
       }
     }
-    cp_async_wait<0>();
-    if (pending == 1) {
-      fence_proxy_async();
-      mbar_arrive(&bfull[(b_ctr - 1) % kNB]);
+    if (!ok && lane == 0 && p.mode != kTcLinear) {
+      // let issued copies land before the CTA's shared memory goes away
+      const uint32_t lo = b_ctr > kNB ? b_ctr - kNB : 0u;
+      for (uint32_t c = lo; c < b_ctr; ++c) mbar_drain(&bfull[c % kNB], (c / kNB) & 1u);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------ MMA issuer

@@ -13,9 +13,9 @@ constexpr int kTcDown = 1;     // down blocks, B = h -> routing-weighted partial
 constexpr int kTcLinear = 2;   // one standalone block -> y
 
 struct TcParams {
-  CUtensorMap lin_map;           // plane tensor map of the standalone block (mode 2)
-  PageTable pt;                  // bits + active LUT slot per block (modes 0, 1)
-  const CUtensorMap* tmaps;      // plane tensor map per block id (modes 0, 1)
+  CUtensorMap b_map;             // token-tile source (modes 0, 1): x_sorted or h_perm,
+                                 // fp16 [rows][ld], 64 x 8 boxes, 128-byte swizzle
+  PageTable pt;                  // planes, bits, active LUT slot per block (modes 0, 1)
   int mode;
   int H, F, S, E, n_groups;
   int n_split;                   // K ranges of the down pass (1 otherwise)
@@ -23,8 +23,6 @@ struct TcParams {
   const int32_t* slot_token;
   const float* slot_w;
   const uint16_t* x;             // bf16 activations [T][lin_cols] (mode 2)
-  const uint16_t* x_perm;        // fp16 activations in the A K order, [T][x_perm_ld] (mode 0)
-  int x_perm_ld;
   uint16_t* h_perm;              // fp16 silu(g)*u in the A K order, [P][h_perm_ld]
   int h_perm_ld;                 // (written by mode 0, read by mode 1; zero past F)
   float* ysorted;                // [n_split][P][H]
@@ -33,6 +31,7 @@ struct TcParams {
   int T;
   int lin_rows, lin_cols, lin_bits;
   const uint16_t* lin_lut;
+  const uint32_t* lin_planes;    // plane pages of the standalone block (mode 2)
   int* err;                      // device error word (may be null)
 };
 

@@ -23,10 +23,15 @@
  *   Linear-block W, rows x cols, applied as y = W x.  Routed expert e has
  *   block ids 3e+0 (gate, F x H), 3e+1 (up, F x H), 3e+2 (down, H x F); the
  *   shared expert (if any) has ids 3E+0..3E+2 with S in place of F.
- *   Bit-planes: uint32 [n_max][rows][words], words = ceil(cols/32), plane 0
- *   holds the MOST significant code bit; bit (i % 32) of word (i / 32) is
- *   column i; pad bits are zero.  A b-bit view reads planes 0..b-1 only:
+ *   Bit-planes: plane 0 holds the MOST significant code bit; in the word
+ *   covering columns 32w..32w+31 of a row, bit (i % 32) is column i; pad bits
+ *   are zero.  A b-bit view reads planes 0..b-1 only:
  *   code_b = sum_{k<b} bit_k << (b-1-k) = code_{n_max} >> (n_max - b).
+ *   Pages: each plane is one page; the library reads pages in its paged
+ *   layout, plane-major, each plane pw_plane_bytes(rows, cols) bytes of 4 KB
+ *   tiles (128 rows x 8 words, rows' 16-byte halves swapped on rows with bit
+ *   2 set; see csrc/pages.h).  pw_repack_planes converts the row-major layout
+ *   [plane][rows][words] into it.
  *   LUT of bitwidth b: fp16 [rows][2^b]; W[o][i] = LUT_b[o][code_b(o, i)].
  *   Router: logit[t][e] = x_t . Wr_e (+ bias_e) in fp32; experts ranked by
  *   logit, ties to the lower index; the first k are selected in that order;
@@ -97,14 +102,14 @@ typedef struct {
 /* One linear-block page (see "Definitions").  rows and cols follow from the
  * block id and the config. */
 typedef struct {
-  uint32_t* d_planes;   /* device, [n_max][rows][words]; planes 0..bits-1 must
+  uint32_t* d_planes;   /* device, n_max plane pages; planes 0..bits-1 must
                            be resident at create; the library writes planes
                            bits..n_max-1 when a switch raises the bitwidth */
   uint16_t* d_lut[2];   /* device, two LUT slots of rows * 2^n_max fp16 each;
                            slot 0 holds LUT_bits at create; the library writes
                            the idle slot when a switch changes the bitwidth */
-  const uint32_t* h_planes; /* host master copy of all n_max planes (pinned for
-                               overlap), or NULL if the block is never raised */
+  const uint32_t* h_planes; /* host master copy of all n_max plane pages (pinned
+                               for overlap), or NULL if the block is never raised */
   const uint16_t* h_lut[PW_MAX_BITS + 1]; /* host LUT_b at index b, [rows][2^b],
                                              NULL where b is never used */
   int32_t bits;         /* bitwidth at create, 1..n_max */
@@ -145,8 +150,16 @@ pw_status_t pw_moe_forward_host(pw_moe_t* h, const uint16_t* x_host, int32_t T,
                                 const float* d_router_w, const float* d_router_bias,
                                 uint16_t* y_host, pw_stream_t stream);
 
+/* Bytes of one plane page of a rows x cols block (0 for a bad shape). */
+int64_t pw_plane_bytes(int32_t rows, int32_t cols);
+
+/* Convert n_planes row-major planes d_src [n_planes][rows][ceil(cols/32)]
+ * into plane pages d_dst (n_planes * pw_plane_bytes bytes), on stream. */
+pw_status_t pw_repack_planes(const uint32_t* d_src, uint32_t* d_dst, int32_t rows, int32_t cols,
+                             int32_t n_planes, pw_stream_t stream);
+
 /* One dequantised linear-block on its own: d_y[t][o] = sum_i W_b[o][i] x[t][i]
- * with fp32 output.  d_planes [>=bits][rows][words], d_lut [rows][2^bits]
+ * with fp32 output.  d_planes: >= bits plane pages, d_lut [rows][2^bits]
  * fp16, d_x bf16 [T][cols], d_y fp32 [T][rows]; T >= 0, bits 1..8.  Uses the
  * same dequantisation and contraction as the MoE experts. */
 pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t rows,

@@ -94,3 +94,15 @@ def test_linear_rejects_bad_args(pwlib):
     assert L.pw_linear(None, 4096, 8, 32, 4, 4096, 1, 4096, None) == 1      # null planes
     assert L.pw_linear(4100, 4096, 8, 32, 4, 4096, 1, 4096, None) == 1      # misaligned
     assert L.pw_linear(4096, 4096, 8, 32, 4, None, 0, None, None) == 0      # T = 0: nothing to do
+    assert L.pw_repack_planes(None, 4096, 8, 32, 1, None) == 1
+    assert L.pw_repack_planes(4096, 4096, 8, 32, 9, None) == 1
+
+
+def test_plane_bytes(pwlib):
+    L = pwlib.lib()
+    # 128 rows x 8 words per 4 KB tile
+    assert L.pw_plane_bytes(128, 256) == 4096
+    assert L.pw_plane_bytes(129, 256) == 8192
+    assert L.pw_plane_bytes(128, 257) == 8192
+    assert L.pw_plane_bytes(14336, 4096) == 14336 * 4096 // 8
+    assert L.pw_plane_bytes(0, 32) == 0

@@ -27,8 +27,10 @@ def pw():
     return binding
 
 
-def _dev_planes(planes):
-    return torch.from_numpy(np.ascontiguousarray(planes).view(np.int32)).cuda()
+def _dev_planes(planes, cols, pw):
+    """Row-major planes -> plane pages on the device (the library's layout)."""
+    dev = torch.from_numpy(np.ascontiguousarray(planes).view(np.int32)).cuda()
+    return pw.repack_planes(dev, cols)
 
 
 def _dev_lut(lut):
@@ -48,6 +50,37 @@ def _identity_lut(rows, b):
     return np.tile(np.arange(1 << b, dtype=np.float16), (rows, 1)).view(np.uint16)
 
 
+# ---------------------------------------------------------------- page layout
+
+def _paged_reference(planes, cols):
+    """The plane-page layout written out from its definition: plane k, tile
+    (rt, kt) of 128 rows x 8 words at ((k n_rt + rt) n_kt + kt) * 1024 words;
+    row r at 8r words, its two 4-word halves swapped when bit 2 of r is set."""
+    n, rows, words = planes.shape
+    n_rt, n_kt = -(-rows // 128), -(-words // 8)
+    out = np.zeros((n, n_rt, n_kt, 128, 8), np.uint32)
+    padded = np.zeros((n, n_rt * 128, n_kt * 8), np.uint32)
+    padded[:, :rows, :words] = planes
+    for rt in range(n_rt):
+        for kt in range(n_kt):
+            tile = padded[:, rt * 128:(rt + 1) * 128, kt * 8:(kt + 1) * 8]
+            for r in range(128):
+                if (r >> 2) & 1:
+                    out[:, rt, kt, r, :] = np.concatenate([tile[:, r, 4:], tile[:, r, :4]], axis=1)
+                else:
+                    out[:, rt, kt, r, :] = tile[:, r, :]
+    return out.reshape(n, -1)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 256), (200, 300), (5, 33), (300, 1408)])
+def test_repack_matches_page_layout(pw, rows, cols):
+    rng = np.random.default_rng(rows + cols)
+    planes = synth.random_planes(rng, 3, rows, cols)
+    got = _dev_planes(planes, cols, pw).cpu().numpy().view(np.uint32)
+    assert got.shape[1] * 4 == pw.plane_bytes(rows, cols)
+    np.testing.assert_array_equal(got, _paged_reference(planes, cols))
+
+
 # ---------------------------------------------------------------- pw_linear
 
 LINEAR_SHAPES = [
@@ -65,7 +98,8 @@ def test_linear_unpacks_codes_bit_exactly(pw, oracle, rows, cols, b):
     planes = synth.random_planes(rng, 8, rows, cols)
     want = oracle.unpack_codes(planes, cols, b).astype(np.float32).T  # [cols][rows]
     x = synth.to_bf16_bits(np.eye(cols, dtype=np.float32))
-    y = pw.linear(_dev_planes(planes), _dev_lut(_identity_lut(rows, b)), b, _dev_bf16(x))
+    y = pw.linear(_dev_planes(planes, cols, pw), _dev_lut(_identity_lut(rows, b)), b, _dev_bf16(x),
+                  rows)
     np.testing.assert_array_equal(y.cpu().numpy(), want)
 
 
@@ -77,8 +111,8 @@ def test_linear_integer_exact(pw, oracle, rows, cols):
         x = rng.integers(-8, 9, size=(37, cols)).astype(np.float32)
         codes = oracle.unpack_codes(planes, cols, b).astype(np.int64)
         want = (x.astype(np.int64) @ codes.T).astype(np.float32)
-        y = pw.linear(_dev_planes(planes), _dev_lut(_identity_lut(rows, b)), b,
-                      _dev_bf16(synth.to_bf16_bits(x)))
+        y = pw.linear(_dev_planes(planes, cols, pw), _dev_lut(_identity_lut(rows, b)), b,
+                      _dev_bf16(synth.to_bf16_bits(x)), rows)
         np.testing.assert_array_equal(y.cpu().numpy(), want)
 
 
@@ -91,7 +125,8 @@ def test_linear_random_matches_oracle(pw, oracle, rows, cols):
         x = synth.to_bf16_bits(rng.normal(size=(5, cols)).astype(np.float32))
         ref = oracle.linear(planes, lut, cols, b, synth.bf16_bits_to_float(x).astype(np.float64),
                             threads=8)
-        y = pw.linear(_dev_planes(planes), _dev_lut(lut), b, _dev_bf16(x)).cpu().numpy()
+        y = pw.linear(_dev_planes(planes, cols, pw), _dev_lut(lut), b, _dev_bf16(x),
+                      rows).cpu().numpy()
         scale = np.abs(ref).max()
         assert np.abs(y - ref).max() <= 1e-5 * scale * max(1.0, cols / 1024)
 
@@ -154,7 +189,7 @@ def test_hand_example_on_gpu(pw, oracle):
                max_tokens=3)
     planes, slots, bits = [], [], []
     for (pl, lt, rows, cols, b) in L.block_list:
-        planes.append(_dev_planes(pl))
+        planes.append(_dev_planes(pl, cols, pw))
         s0 = torch.zeros(rows << 3, dtype=torch.int16, device="cuda")
         s0[: lt.size].copy_(torch.from_numpy(lt.reshape(-1).view(np.int16)))
         slots.append((s0, torch.zeros_like(s0)))
