@@ -60,7 +60,7 @@ def lib():
         L.pw_moe_forward.argtypes = [P, P, i32, P, P, P, P]
         L.pw_destroy.argtypes = [P]
         L.pw_moe_forward_host.argtypes = [P, P, i32, P, P, P, P]
-        L.pw_linear.argtypes = [P, P, i32, i32, i32, P, i32, P, P]
+        L.pw_linear.argtypes = [P, P, i32, i32, i32, i32, P, i32, P, P]
         L.pw_get_block_bits.argtypes = [P, i32, C.POINTER(i32), C.POINTER(i32)]
         L.pw_get_routing.argtypes = [P, P, P, P]
         L.pw_check_device_error.argtypes = [P]
@@ -103,23 +103,26 @@ def plane_bytes(rows: int, cols: int) -> int:
 
 def repack_planes(planes, cols: int, stream=None):
     """Row-major planes (int32 device tensor [n][rows][ceil(cols/32)], uint32
-    bit patterns) -> plane pages (int32 device tensor [n][plane_bytes / 4])."""
+    bit patterns) -> the paged layout of an n-plane block (flat int32 device
+    tensor of n * plane_bytes / 4 words)."""
     import torch
     n, rows, _ = planes.shape
-    out = torch.empty((n, plane_bytes(rows, cols) // 4), dtype=torch.int32, device=planes.device)
+    out = torch.empty(n * plane_bytes(rows, cols) // 4, dtype=torch.int32, device=planes.device)
     check(lib().pw_repack_planes(_ptr(planes), _ptr(out), rows, cols, n, _stream(stream)))
     return out
 
 
 def linear(planes, lut, bits: int, x, rows: int, y=None, stream=None):
-    """y[t][o] = sum_i W_b[o][i] x[t][i] for one block.  planes: plane pages
-    (repack_planes) of at least `bits` planes; lut: int16 [rows][2^bits] (fp16
-    bit patterns); x: bf16 [T][cols].  Returns fp32 [T][rows]."""
+    """y[t][o] = sum_i W_b[o][i] x[t][i] for one block.  planes: a block in
+    the paged layout (repack_planes; its plane count follows from its size);
+    lut: int16 [rows][2^bits] (fp16 bit patterns); x: bf16 [T][cols].
+    Returns fp32 [T][rows]."""
     import torch
     T, cols = x.shape
+    n_max = planes.numel() * 4 // plane_bytes(rows, cols)
     if y is None:
         y = torch.empty((T, rows), dtype=torch.float32, device=x.device)
-    check(lib().pw_linear(_ptr(planes), _ptr(lut), rows, cols, bits, _ptr(x), T, _ptr(y),
+    check(lib().pw_linear(_ptr(planes), _ptr(lut), rows, cols, n_max, bits, _ptr(x), T, _ptr(y),
                           _stream(stream)))
     return y
 

@@ -73,19 +73,23 @@ EncodeTiledFn encode_fn() {
 // activations in whole 32-column groups: it takes cols % 128 == 0.
 bool tc_shape_ok(int cols) { return cols % 128 == 0; }
 
-// 2-D map over an fp16 row buffer [rows][ld] for the token tiles: boxes of
-// 64 columns x 8 rows with the 128-byte swizzle of the MMA's K-major operand.
-pw_status_t make_row_map(CUtensorMap* m, const uint16_t* base, int ld, int rows) {
+// Maps over an atom-major fp16 buffer [ld / 64][rows][64] for the token
+// tiles, as {64 columns, rows, atoms}: box i loads 8(i+1) rows x 4 atoms with
+// the 128-byte swizzle of the MMA's K-major operand, one copy per stage.
+pw_status_t make_row_maps(CUtensorMap* m, const uint16_t* base, int ld, int rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[2] = {64, 8};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(base), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled (rows) failed (%d)", (int)r);
+  for (int i = 0; i < 4; ++i) {
+    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(ld / 64)};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(rows) * 128};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(8 * (i + 1)), 4};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled (token rows) failed (%d)", (int)r);
+  }
   return PW_OK;
 }
 
@@ -120,7 +124,7 @@ struct pw_moe {
   uint16_t* x_sorted = nullptr; // tensor-core path: gathered fp16 activations, K-permuted
   uint16_t* h_perm = nullptr;   // tensor-core path: fp16 silu(g) * u, K-permuted
   int x_ld = 0, h_perm_ld = 0;
-  CUtensorMap x_map, h_map;     // 2-D TMA maps over x_sorted and h_perm
+  CUtensorMap x_maps[4], h_maps[4];  // token-tile maps over x_sorted and h_perm
   float* ysorted = nullptr;
   int* err = nullptr;
   uint16_t* stage_x = nullptr;
@@ -300,8 +304,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   }
   // token-tile tensor maps for the tensor-core passes
   if (h->tc) {
-    pw_status_t st = make_row_map(&h->x_map, h->x_sorted, h->x_ld, h->P_max);
-    if (st == PW_OK) st = make_row_map(&h->h_map, h->h_perm, h->h_perm_ld, h->P_max);
+    pw_status_t st = make_row_maps(h->x_maps, h->x_sorted, h->x_ld, h->P_max);
+    if (st == PW_OK) st = make_row_maps(h->h_maps, h->h_perm, h->h_perm_ld, h->P_max);
     if (st != PW_OK) {
       free_all(h);
       return st;
@@ -327,11 +331,14 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
     return fail(PW_ERR_INVALID_ARG, "block %d: raising bits needs the host planes", block_id);
   cudaStream_t s = static_cast<cudaStream_t>(side_stream);
   if (h->any_forward) PW_CUDA(cudaStreamWaitEvent(s, h->fwd_done, 0));
-  const size_t plane_elems = static_cast<size_t>(pw::pages::plane_words(b.rows, b.cols));
   if (new_bits > b.bits) {
-    PW_CUDA(cudaMemcpyAsync(b.d_planes + b.bits * plane_elems, b.h_planes + b.bits * plane_elems,
-                            sizeof(uint32_t) * plane_elems * (new_bits - b.bits),
-                            cudaMemcpyHostToDevice, s));
+    // planes b.bits .. new_bits-1 are tiles b.bits.. of every tile group
+    const size_t pitch = static_cast<size_t>(h->cfg.n_max) * pw::pages::kTileBytes;
+    const size_t groups = static_cast<size_t>(pw::pages::groups_of(b.rows, b.cols));
+    const size_t off = static_cast<size_t>(b.bits) * (pw::pages::kTileBytes / 4);
+    PW_CUDA(cudaMemcpy2DAsync(b.d_planes + off, pitch, b.h_planes + off, pitch,
+                              static_cast<size_t>(new_bits - b.bits) * pw::pages::kTileBytes,
+                              groups, cudaMemcpyHostToDevice, s));
   }
   PW_CUDA(cudaMemcpyAsync(b.d_lut[b.slot ^ 1], b.h_lut[new_bits],
                           sizeof(uint16_t) * static_cast<size_t>(b.rows) << new_bits,
@@ -422,6 +429,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     gp.x_sorted = h->x_sorted;
     gp.H = c.hidden;
     gp.ld = h->x_ld;
+    gp.rows = h->P_max;
     gp.n_groups = h->G;
     PW_CUDA(pw::launch_gather(gp, T * c.top_k + (c.shared_ffn > 0 ? T : 0), h->n_sm, s));
     pw::TcParams tp;
@@ -437,9 +445,11 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.offsets = h->ws.offsets;
     tp.slot_token = h->ws.slot_token;
     tp.slot_w = h->ws.slot_w;
-    tp.b_map = h->x_map;
+    for (int i = 0; i < 4; ++i) tp.b_maps[i] = h->x_maps[i];
+    tp.n_max = c.n_max;
     tp.h_perm = h->h_perm;
     tp.h_perm_ld = h->h_perm_ld;
+    tp.h_rows = h->P_max;
     tp.err = h->err;
     PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
   } else {
@@ -447,6 +457,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     std::memset(&sp, 0, sizeof(sp));
     sp.pt = pt;
     sp.mode = 0;
+    sp.n_max = c.n_max;
     sp.H = c.hidden;
     sp.F = c.ffn;
     sp.S = c.shared_ffn;
@@ -479,7 +490,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.offsets = h->ws.offsets;
     tp.slot_token = h->ws.slot_token;
     tp.slot_w = h->ws.slot_w;
-    tp.b_map = h->h_map;
+    for (int i = 0; i < 4; ++i) tp.b_maps[i] = h->h_maps[i];
+    tp.n_max = c.n_max;
     tp.h_perm = h->h_perm;
     tp.h_perm_ld = h->h_perm_ld;
     tp.ysorted = h->ysorted;
@@ -491,6 +503,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     std::memset(&sp, 0, sizeof(sp));
     sp.pt = pt;
     sp.mode = 1;
+    sp.n_max = c.n_max;
     sp.H = c.hidden;
     sp.F = c.ffn;
     sp.S = c.shared_ffn;
@@ -553,10 +566,11 @@ pw_status_t pw_moe_forward_host(pw_moe_t* h, const uint16_t* x_host, int32_t T,
 }
 
 pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t rows, int32_t cols,
-                      int32_t bits, const uint16_t* d_x, int32_t T, float* d_y,
+                      int32_t n_max, int32_t bits, const uint16_t* d_x, int32_t T, float* d_y,
                       pw_stream_t stream) {
   if (rows < 1 || cols < 1 || T < 0) return fail(PW_ERR_INVALID_ARG, "bad shape");
-  if (bits < 1 || bits > PW_MAX_BITS) return fail(PW_ERR_INVALID_ARG, "bits outside [1, 8]");
+  if (n_max < 1 || n_max > PW_MAX_BITS || bits < 1 || bits > n_max)
+    return fail(PW_ERR_INVALID_ARG, "need 1 <= bits <= n_max <= 8");
   if (!d_planes || !d_lut || (T > 0 && (!d_x || !d_y))) return fail(PW_ERR_INVALID_ARG, "null buffer");
   if (!aligned16(d_planes) || !aligned16(d_lut) || (d_x && !aligned16(d_x)))
     return fail(PW_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
@@ -579,6 +593,7 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
     tp.lin_bits = bits;
     tp.lin_lut = d_lut;
     tp.lin_planes = d_planes;
+    tp.lin_n_max = n_max;
     tp.err = nullptr;
     PW_CUDA(pw::launch_tc(tp, n_sm, s));
   } else {
@@ -591,6 +606,7 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
     sp.lin_rows = rows;
     sp.lin_cols = cols;
     sp.lin_bits = bits;
+    sp.lin_n_max = n_max;
     sp.lin_planes = d_planes;
     sp.lin_lut = d_lut;
     PW_CUDA(pw::launch_simple(sp, rows, s));

@@ -53,8 +53,8 @@ struct GatherParams {
   const uint16_t* x;         // bf16 [T][H]
   const int32_t* offsets;    // [n_groups+1]
   const int32_t* slot_token; // [P]
-  uint16_t* x_sorted;        // fp16 [P][ld], tensor-core K order
-  int H, ld, n_groups;
+  uint16_t* x_sorted;        // fp16 atom-major [ld/64][rows][64], tensor-core K order
+  int H, ld, rows, n_groups;
 };
 
 struct CombineParams {
@@ -80,7 +80,8 @@ struct SimpleParams {
   float* ysorted;         // [P][H] (mode 1 out)
   float* y;               // [T][rows] (mode 2 out)
   int T;                  // tokens (mode 2)
-  int lin_rows, lin_cols, lin_bits;  // mode 2 block
+  int lin_rows, lin_cols, lin_bits, lin_n_max;  // mode 2 block
+  int n_max;                         // planes per block (modes 0, 1)
   const uint32_t* lin_planes;
   const uint16_t* lin_lut;
 };

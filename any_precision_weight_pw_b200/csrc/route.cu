@@ -157,9 +157,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   }
 }
 
-// x_sorted[pos] = the activations of token slot_token[pos] as fp16, each
+// x_sorted row pos = the activations of token slot_token[pos] as fp16, each
 // 32-column group permuted into the tensor-core kernel's K order; rows are the
 // sorted positions of all groups, so every expert's token tile is contiguous.
+// Stored atom-major, [ld / 64][rows][64], so one 3-D copy fetches a stage.
 // One 32-column group per thread.
 __global__ void gather_kernel(const GatherParams p) {
   const int P = p.offsets[p.n_groups];
@@ -180,7 +181,8 @@ __global__ void gather_kernel(const GatherParams p) {
         v[8 * q + 2 * e + 1] = bf16_bits_to_f32(static_cast<uint16_t>(r4[e] >> 16));
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(p.x_sorted + static_cast<size_t>(pos) * p.ld + 32 * w);
+    uint4* dst = reinterpret_cast<uint4*>(
+        p.x_sorted + (static_cast<size_t>(w >> 1) * p.rows + pos) * 64 + 32 * (w & 1));
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t o[4];

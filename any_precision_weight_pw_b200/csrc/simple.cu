@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
   const int mode = p.mode;
 
   // Which block, rows, cols and token range this CTA serves.
-  int blk = 0, rows, cols, bits, pos0, n_tok;
+  int blk = 0, rows, cols, bits, pos0, n_tok, n_max;
   const uint32_t* planes;
   const uint16_t* lut;
   int group = 0, proj = 0;
@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
     rows = p.lin_rows;
     cols = p.lin_cols;
     bits = p.lin_bits;
+    n_max = p.lin_n_max;
     planes = p.lin_planes;
     lut = p.lin_lut;
     pos0 = 0;
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
     rows = (proj < 2) ? Fg : p.H;
     cols = (proj < 2) ? p.H : Fg;
     bits = p.pt.bits[blk];
+    n_max = p.n_max;
     planes = p.pt.blk[blk].planes;
     lut = p.pt.blk[blk].lut;
     pos0 = p.offsets[group];
@@ -103,7 +105,8 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
       const uint16_t* lrow = lut + (static_cast<size_t>(o) << bits);
       for (int w = lane; w < words; w += 32) {
         uint32_t pw_[PW_MAX_BITS];
-        for (int k = 0; k < bits; ++k) pw_[k] = planes[pages::word_index(k, o, w, rows, cols)];
+        for (int k = 0; k < bits; ++k)
+          pw_[k] = planes[pages::word_index(k, o, w, rows, cols, n_max)];
         const int cmax = min(32, cols - 32 * w);
         for (int c = 0; c < cmax; ++c) {
           int code = 0;

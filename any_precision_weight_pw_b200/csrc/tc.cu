@@ -12,18 +12,19 @@
 // its epilogue can apply SwiGLU); the down item makes one pass (over one K
 // range when the down pass is split); a standalone linear makes one pass.
 //   warp 8      producer: streams only the b active bit-planes of the block,
-//               128 rows x 256 columns (8 words) per plane per stage, each a
-//               contiguous 4 KB tile of the paged layout (pages.h) moved by
-//               one bulk copy into a ring of 4 KB slots; the tile arrives with
-//               its rows' halves already swizzled, so the thread-per-row reads
-//               below are bank-conflict free.
+//               128 rows x 256 columns (8 words) per stage: in the paged
+//               layout (pages.h) the b tiles are one contiguous b * 4 KB run,
+//               moved by ONE bulk copy into a ring of 4 KB slots (stages take
+//               b consecutive slots, so the ring holds more stages at low b);
+//               the tiles arrive with their rows' halves already swizzled, so
+//               the thread-per-row reads below are bank-conflict free.
 //   warp 10     token-tile loader: the item's token rows are contiguous in an
 //               fp16 buffer already in the A operand's K order (the gathered
 //               activations for gate/up, h = silu(g)*u for down), so one lane
-//               streams each stage's 256 columns with 2-D TMA boxes (64
-//               columns x 8 rows, 128-byte swizzle = the MMA's K-major B
-//               layout) into a 4-deep ring.  A standalone linear converts its
-//               bf16 rows with all 32 lanes instead.
+//               moves each stage's tile with ONE 3-D TMA box (4 atoms of 64
+//               columns x 8, 16, 24 or 32 rows, 128-byte swizzle = the MMA's
+//               K-major B layout) into a 4-deep ring.  A standalone linear
+//               converts its bf16 rows with all 32 lanes instead.
 //   warps 0-7   dequantisers in two K halves: warps q and q+4 both own rows
 //               32q..32q+31 (thread <-> output row <-> TMEM lane); the first
 //               group takes columns 0-127 of every stage, the second
@@ -56,8 +57,9 @@ namespace {
 
 constexpr int kTileRows = 128;
 constexpr int kStageWords = 8;                 // 256 columns per stage
-constexpr int kSlotBytes = kTileRows * kStageWords * 4;  // 4 KB
-constexpr int kNSlot = 16;
+constexpr int kSlotBytes = kTileRows * kStageWords * 4;  // 4 KB: one plane of a stage
+constexpr int kNSlot = 20;                     // plane slots (80 KB)
+constexpr int kNS = 8;                         // plane stages in flight (barrier pairs)
 constexpr int kNT = kTcTokens;                 // token tile (MMA N <= 32)
 constexpr int kBStageBytes = kNT * 256 * 2;    // 32 rows x 256 K fp16 = 16 KB
 constexpr int kNB = 4;                         // token-tile ring depth
@@ -78,10 +80,19 @@ constexpr uint32_t kLutBytes = 128u * 128u * 4u;
 constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
 constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
 constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
-constexpr uint32_t kNumBars = 2 * kNSlot + 2 * kNB + 2 * kNA + 4 + 2;
+constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 4 + 2;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
 constexpr uint32_t kSmemTotal = kOffMisc + 16 + 4 * (kMaxGroups + 2);
 static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
+
+// Plane stages take `bits` consecutive slots of the ring; a stage that would
+// run past the end starts again at slot 0.  Producer and dequantisers walk
+// the same sequence of stages, so both derive the same placement.
+__device__ __forceinline__ uint32_t place_stage(uint32_t& ring_end, int bits) {
+  const uint32_t start = (ring_end + bits <= static_cast<uint32_t>(kNSlot)) ? ring_end : 0u;
+  ring_end = start + bits;
+  return start;
+}
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -157,12 +168,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint64_t* bar) {
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
       : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() {
@@ -243,12 +254,15 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Byte offset of 16-byte chunk c16 (0..31) of token row n in a B stage
-// (K-major, 128-byte swizzle: 64 columns per 128-byte atom row).
-__device__ __forceinline__ uint32_t b_chunk_off(int n, int c16) {
+// Byte offset of 16-byte chunk c16 (0..31) of token row n in a B stage of
+// `rows` rows (K-major, 128-byte swizzle: 64 columns per 128-byte atom row,
+// atoms of `rows` rows one after the other).
+__device__ __forceinline__ uint32_t b_chunk_off(int n, int c16, int rows) {
   const int atom = c16 >> 3, c = c16 & 7;
-  return atom * (kNT * 128) + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
+  return atom * (rows * 128) + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
 }
+// Rows of a token tile as loaded: whole 8-row groups covering ntok.
+__device__ __forceinline__ int tile_rows(int ntok) { return ((ntok + 7) >> 3) << 3; }
 
 // ---------------------------------------------------------------- work items
 struct Pass {
@@ -323,8 +337,9 @@ __device__ __forceinline__ bool dq_sync(uint64_t* bar, uint32_t& phase, const Ct
 }
 
 struct DequantState {
-  uint32_t slot_ctr;  // plane slots consumed
-  uint32_t a_ctr;     // stages processed by this K half
+  uint32_t stage_ctr;  // plane stages consumed
+  uint32_t ring_end;   // plane-slot placement (place_stage)
+  uint32_t a_ctr;      // stages processed by this K half
 };
 
 // b = 8 tables are packed two entries per word: word (v >> 1) * 128 + r.
@@ -352,7 +367,7 @@ __device__ __forceinline__ void dq_word8(const uint32_t (&P)[8], uint32_t r4, ui
 
 template <int B>
 __device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegLut& L,
-                               uint64_t* pf, uint64_t* pe, uint64_t* af, uint64_t* ae,
+                               uint64_t* sf, uint64_t* se, uint64_t* af, uint64_t* ae,
                                uint32_t tmem_base, DequantState& st, const Ctl& ctl) {
   const int lane = threadIdx.x & 31;
   const int r = 32 * quad + lane;
@@ -363,18 +378,19 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegL
   };
   for (int s = it.s_begin; s < it.s_end; ++s) {
     uint32_t P[4][B];
+    const uint32_t e = st.stage_ctr % kNS;
+    const uint32_t slot0 = place_stage(st.ring_end, B);
+    if (!mbar_wait_warp(&sf[e], (st.stage_ctr / kNS) & 1u, ctl)) return false;
 #pragma unroll
     for (int k = 0; k < B; ++k) {
-      const uint32_t c = st.slot_ctr + k;
-      if (!mbar_wait_warp(&pf[c % kNSlot], (c / kNSlot) & 1u, ctl)) return false;
-      const uint4 q4 = read_plane_chunk(kOffSlots + (c % kNSlot) * kSlotBytes, r, grp);
+      const uint4 q4 = read_plane_chunk(kOffSlots + (slot0 + k) * kSlotBytes, r, grp);
       P[0][k] = q4.x;
       P[1][k] = q4.y;
       P[2][k] = q4.z;
       P[3][k] = q4.w;
     }
-#pragma unroll
-    for (int k = 0; k < B; ++k) mbar_arrive(&pe[(st.slot_ctr + k) % kNSlot]);
+    mbar_arrive(&se[e]);
+    st.stage_ctr++;
     const uint32_t a_idx = 2u * st.a_ctr + static_cast<uint32_t>(grp);
     const uint32_t qa = a_idx % kNA;
     if (!mbar_wait_warp(&ae[qa], ((a_idx / kNA) & 1u) ^ 1u, ctl)) return false;
@@ -398,7 +414,6 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegL
     tc_fence_before();
     mbar_arrive(&af[qa]);
     st.a_ctr++;
-    st.slot_ctr += B;
   }
   return true;
 }
@@ -518,7 +533,7 @@ __device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t
       q16[pr] = pack_h2(v[dq::col_of_kpos(2 * pr)], v[dq::col_of_kpos(2 * pr + 1)]);
 #pragma unroll
     for (int qc = 0; qc < 4; ++qc) {
-      const uint32_t dst = buf + b_chunk_off(n, 4 * w + qc);
+      const uint32_t dst = buf + b_chunk_off(n, 4 * w + qc, tile_rows(it.ntok));
       asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(q16[4 * qc]),
                    "r"(q16[4 * qc + 1]), "r"(q16[4 * qc + 2]), "r"(q16[4 * qc + 3])
                    : "memory");
@@ -530,9 +545,9 @@ __device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t
 __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__ TcParams p) {
   uint8_t* smem = pw_tc_smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
-  uint64_t* pf = bars;
-  uint64_t* pe = pf + kNSlot;
-  uint64_t* bfull = pe + kNSlot;
+  uint64_t* sf = bars;      // plane stage full (bulk copy landed)
+  uint64_t* se = sf + kNS;  // plane stage empty (all dequantisers read it)
+  uint64_t* bfull = se + kNS;
   uint64_t* bempty = bfull + kNB;
   uint64_t* af = bempty + kNB;
   uint64_t* ae = af + kNA;
@@ -549,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   const int G = (p.mode == kTcLinear) ? 1 : p.n_groups;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNSlot; ++i) {
-      mbar_init(&pf[i], 1);
-      mbar_init(&pe[i], kDqThreads);
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&sf[i], 1);
+      mbar_init(&se[i], kDqThreads);
     }
     for (int i = 0; i < kNB; ++i) {
       mbar_init(&bfull[i], p.mode == kTcLinear ? 32 : 1);
@@ -604,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
 
   if (warp < 8) {
     // ------------------------------------------------ dequantisers
-    DequantState st{0u, 0u};
+    DequantState st{0u, 0u, 0u};
     const int grp = warp >> 2, quad = warp & 3;
     const int r = 32 * quad + lane;
     uint32_t sync_phase = 0;
@@ -634,50 +649,64 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       }
       if (ni < total) lut_prefetch(it, get_pass(p, it, nq), grp, r, pre);
       switch (ps.bits) {
-        case 1: ok = dequant_stages<1>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        case 2: ok = dequant_stages<2>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        case 3: ok = dequant_stages<3>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        case 4: ok = dequant_stages<4>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        case 5: ok = dequant_stages<5>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        case 6: ok = dequant_stages<6>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        case 7: ok = dequant_stages<7>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
-        default: ok = dequant_stages<8>(cur, grp, quad, L, pf, pe, af, ae, tmem_base, st, ctl); break;
+        case 1: ok = dequant_stages<1>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 2: ok = dequant_stages<2>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 3: ok = dequant_stages<3>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 4: ok = dequant_stages<4>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 5: ok = dequant_stages<5>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 6: ok = dequant_stages<6>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 7: ok = dequant_stages<7>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        default: ok = dequant_stages<8>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
       }
       i = ni;
       q = nq;
     }
   } else if (warp == kWarpProducer) {
-    // ------------------------------------------------ TMA producer (planes)
+    // ------------------------------------------------ producer (planes)
     if (lane == 0) {
-      uint32_t slot_ctr = 0;
+      uint32_t t = 0, ring_end = 0;
+      uint32_t rs[kNS], re[kNS];  // slot range of each stage in flight
       bool ok = true;
+      const int n_max = (p.mode == kTcLinear) ? p.lin_n_max : p.n_max;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
         decode_item(p, s_prefix, G, i, it);
-        const int n_rt = pages::row_tiles(it.rows), n_kt = pages::k_tiles(it.cols);
+        const int n_kt = pages::k_tiles(it.cols);
         const int rt = it.row0 / kTileRows;
         for (int q = 0; q < it.npass && ok; ++q) {
           const Pass ps = get_pass(p, it, q);
-          for (int s = it.s_begin; s < it.s_end && ok; ++s) {
-            for (int k = 0; k < ps.bits; ++k) {
-              const uint32_t sl = slot_ctr % kNSlot;
-              if (!mbar_wait(&pe[sl], ((slot_ctr / kNSlot) & 1u) ^ 1u, ctl)) {
-                ok = false;
+          for (int s = it.s_begin; s < it.s_end; ++s, ++t) {
+            const uint32_t e = t % kNS;
+            const uint32_t start = place_stage(ring_end, ps.bits);
+            // the barrier pair of stage t - kNS is free ...
+            if (!mbar_wait(&se[e], ((t / kNS) & 1u) ^ 1u, ctl)) {
+              ok = false;
+              break;
+            }
+            // ... and so are the slots: wait for the latest earlier stage
+            // still holding any of them (stages are released in order)
+            for (uint32_t j = 1; j < kNS && j <= t; ++j) {
+              const uint32_t u = t - j;
+              if (rs[u % kNS] < start + ps.bits && start < re[u % kNS]) {
+                if (!mbar_wait(&se[u % kNS], (u / kNS) & 1u, ctl)) ok = false;
                 break;
               }
-              const int64_t tile = (static_cast<int64_t>(k) * n_rt + rt) * n_kt + s;
-              mbar_arrive_tx(&pf[sl], kSlotBytes);
-              bulk_load(smem_addr(smem + kOffSlots + sl * kSlotBytes),
-                        ps.planes + tile * (kSlotBytes / 4), kSlotBytes, &pf[sl]);
-              slot_ctr++;
             }
+            if (!ok) break;
+            rs[e] = start;
+            re[e] = start + ps.bits;
+            const int64_t grp_idx = static_cast<int64_t>(rt) * n_kt + s;
+            const uint32_t bytes = static_cast<uint32_t>(ps.bits) * kSlotBytes;
+            mbar_arrive_tx(&sf[e], bytes);
+            bulk_load(smem_addr(smem + kOffSlots + start * kSlotBytes),
+                      ps.planes + grp_idx * n_max * (kSlotBytes / 4), bytes, &sf[e]);
           }
         }
       }
       if (!ok) {
         // let every issued copy land before the CTA's shared memory goes away
-        const uint32_t lo = slot_ctr > kNSlot ? slot_ctr - kNSlot : 0u;
-        for (uint32_t c = lo; c < slot_ctr; ++c) mbar_drain(&pf[c % kNSlot], (c / kNSlot) & 1u);
+        const uint32_t lo = t > kNS ? t - kNS : 0u;
+        for (uint32_t c = lo; c < t; ++c) mbar_drain(&sf[c % kNS], (c / kNS) & 1u);
       }
     }
   } else if (warp == kWarpLoader) {
@@ -687,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
       Item it;
       decode_item(p, s_prefix, G, i, it);
-      const int ngrp = (it.ntok + 7) >> 3;  // 8-row groups of the tile
+      const int rows_b = tile_rows(it.ntok);  // token rows loaded per stage
       for (int q = 0; q < it.npass && ok; ++q) {
         for (int s = it.s_begin; s < it.s_end; ++s) {
           const uint32_t jb = b_ctr % kNB;
@@ -701,11 +730,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             fence_proxy_async();
             mbar_arrive(&bfull[jb]);
           } else if (lane == 0) {
-            mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(ngrp) * 4u * 1024u);
-            for (int a = 0; a < 4; ++a)
-              for (int j = 0; j < ngrp; ++j)
-                tma_load_2d(buf + a * (kNT * 128) + j * 1024, &p.b_map, s * 256 + a * 64,
-                            it.pos0 + 8 * j, &bfull[jb]);
+            // {64 columns, rows_b rows, 4 atoms} starting at column 256 s
+            mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(rows_b) * 4u * 128u);
+            tma_load_3d(buf, &p.b_maps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s, &bfull[jb]);
           }
           b_ctr++;
         }
@@ -726,6 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         decode_item(p, s_prefix, G, i, it);
         const int n = it.ntok <= 16 ? 16 : 32;
         const uint32_t idesc = mma_idesc(n);
+        const uint32_t atom_bytes = static_cast<uint32_t>(tile_rows(it.ntok)) * 128u;
         const uint32_t jd = d_ctr & 1u;
         if (!mbar_wait(&de[jd], ((d_ctr >> 1) & 1u) ^ 1u, ctl)) break;
         tc_fence_after();
@@ -751,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
                 const int kp = sub * 128 + kk * 16;
-                const uint32_t baddr = bbase + (kp >> 6) * (kNT * 128) + (kp & 63) * 2;
+                const uint32_t baddr = bbase + (kp >> 6) * atom_bytes + (kp & 63) * 2;
                 tc_mma(dt, at + kk * 8, smem_desc_sw128(baddr), idesc, accum);
                 accum = 1;
               }
@@ -793,14 +821,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       if (o < it.rows) {
         if (p.mode == kTcGateUp) {
           // h = silu(g) * u, fp16, at o's position in the down pass's K order
-          const size_t col = static_cast<size_t>(o & ~31) + dq::kpos_of_col(o & 31);
+          // atom-major [ld/64][rows][64]: column col of row pos at
+          // ((col / 64) * rows + pos) * 64 + col % 64
+          const int col = (o & ~31) + dq::kpos_of_col(o & 31);
+          uint16_t* hp = p.h_perm + static_cast<size_t>(col >> 6) * p.h_rows * 64 + (col & 63);
 #pragma unroll
           for (int n = 0; n < kNT; ++n) {
             if (n >= it.ntok) break;
             const float g = __uint_as_float(v[n]);
             const float h = g / (1.0f + expf(-g)) * __uint_as_float(u[n]);
-            p.h_perm[static_cast<size_t>(it.pos0 + n) * p.h_perm_ld + col] =
-                __half_as_ushort(__float2half_rn(h));
+            hp[static_cast<size_t>(it.pos0 + n) * 64] = __half_as_ushort(__float2half_rn(h));
           }
         } else if (p.mode == kTcDown) {
 #pragma unroll

@@ -13,23 +13,25 @@ constexpr int kTcDown = 1;     // down blocks, B = h -> routing-weighted partial
 constexpr int kTcLinear = 2;   // one standalone block -> y
 
 struct TcParams {
-  CUtensorMap b_map;             // token-tile source (modes 0, 1): x_sorted or h_perm,
-                                 // fp16 [rows][ld], 64 x 8 boxes, 128-byte swizzle
+  CUtensorMap b_maps[4];         // token-tile source (modes 0, 1): x_sorted or h_perm
+                                 // as {64 columns, rows, atoms}; box i holds 8(i+1)
+                                 // rows x 4 atoms, 128-byte swizzle
   PageTable pt;                  // planes, bits, active LUT slot per block (modes 0, 1)
   int mode;
-  int H, F, S, E, n_groups;
+  int H, F, S, E, n_groups, n_max;
   int n_split;                   // K ranges of the down pass (1 otherwise)
   const int32_t* offsets;        // [G+1] sorted-position ranges per group
   const int32_t* slot_token;
   const float* slot_w;
   const uint16_t* x;             // bf16 activations [T][lin_cols] (mode 2)
-  uint16_t* h_perm;              // fp16 silu(g)*u in the A K order, [P][h_perm_ld]
-  int h_perm_ld;                 // (written by mode 0, read by mode 1; zero past F)
+  uint16_t* h_perm;              // fp16 silu(g)*u in the A K order, atom-major
+  int h_perm_ld, h_rows;         // [h_perm_ld/64][h_rows][64] (written by mode 0,
+                                 // read by mode 1; zero past F)
   float* ysorted;                // [n_split][P][H]
   long long split_stride;        // floats between split partial buffers
   float* y;                      // [T][lin_rows] (mode 2)
   int T;
-  int lin_rows, lin_cols, lin_bits;
+  int lin_rows, lin_cols, lin_bits, lin_n_max;
   const uint16_t* lin_lut;
   const uint32_t* lin_planes;    // plane pages of the standalone block (mode 2)
   int* err;                      // device error word (may be null)

@@ -27,11 +27,13 @@
  *   covering columns 32w..32w+31 of a row, bit (i % 32) is column i; pad bits
  *   are zero.  A b-bit view reads planes 0..b-1 only:
  *   code_b = sum_{k<b} bit_k << (b-1-k) = code_{n_max} >> (n_max - b).
- *   Pages: each plane is one page; the library reads pages in its paged
- *   layout, plane-major, each plane pw_plane_bytes(rows, cols) bytes of 4 KB
- *   tiles (128 rows x 8 words, rows' 16-byte halves swapped on rows with bit
- *   2 set; see csrc/pages.h).  pw_repack_planes converts the row-major layout
- *   [plane][rows][words] into it.
+ *   Pages: each plane is one page.  The library reads a block's n_max planes
+ *   in its paged layout: tile groups of 128 rows x 8 words, each holding the
+ *   n_max planes' 4 KB tiles one after the other (so the b active planes of a
+ *   group are one contiguous b * 4 KB run); rows' 16-byte halves are swapped
+ *   on rows with bit 2 set (csrc/pages.h).  A block takes n_max *
+ *   pw_plane_bytes(rows, cols) bytes; pw_repack_planes converts the
+ *   row-major layout [plane][rows][words] into it.
  *   LUT of bitwidth b: fp16 [rows][2^b]; W[o][i] = LUT_b[o][code_b(o, i)].
  *   Router: logit[t][e] = x_t . Wr_e (+ bias_e) in fp32; experts ranked by
  *   logit, ties to the lower index; the first k are selected in that order;
@@ -102,7 +104,8 @@ typedef struct {
 /* One linear-block page (see "Definitions").  rows and cols follow from the
  * block id and the config. */
 typedef struct {
-  uint32_t* d_planes;   /* device, n_max plane pages; planes 0..bits-1 must
+  uint32_t* d_planes;   /* device, the block's n_max plane pages (paged
+                           layout, n_max * pw_plane_bytes); planes 0..bits-1 must
                            be resident at create; the library writes planes
                            bits..n_max-1 when a switch raises the bitwidth */
   uint16_t* d_lut[2];   /* device, two LUT slots of rows * 2^n_max fp16 each;
@@ -154,17 +157,19 @@ pw_status_t pw_moe_forward_host(pw_moe_t* h, const uint16_t* x_host, int32_t T,
 int64_t pw_plane_bytes(int32_t rows, int32_t cols);
 
 /* Convert n_planes row-major planes d_src [n_planes][rows][ceil(cols/32)]
- * into plane pages d_dst (n_planes * pw_plane_bytes bytes), on stream. */
+ * into the paged layout of an n_max = n_planes block, d_dst
+ * (n_planes * pw_plane_bytes bytes), on stream. */
 pw_status_t pw_repack_planes(const uint32_t* d_src, uint32_t* d_dst, int32_t rows, int32_t cols,
                              int32_t n_planes, pw_stream_t stream);
 
 /* One dequantised linear-block on its own: d_y[t][o] = sum_i W_b[o][i] x[t][i]
- * with fp32 output.  d_planes: >= bits plane pages, d_lut [rows][2^bits]
+ * with fp32 output.  d_planes: a block of n_max planes in the paged layout
+ * (bits <= n_max are read), d_lut [rows][2^bits]
  * fp16, d_x bf16 [T][cols], d_y fp32 [T][rows]; T >= 0, bits 1..8.  Uses the
  * same dequantisation and contraction as the MoE experts. */
 pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t rows,
-                      int32_t cols, int32_t bits, const uint16_t* d_x, int32_t T,
-                      float* d_y, pw_stream_t stream);
+                      int32_t cols, int32_t n_max, int32_t bits, const uint16_t* d_x,
+                      int32_t T, float* d_y, pw_stream_t stream);
 
 /* Bitwidth the next forward will use, and the pending one (0 if none). */
 pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_next,

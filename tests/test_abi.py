@@ -89,11 +89,12 @@ def test_null_handle_calls(pwlib):
 
 def test_linear_rejects_bad_args(pwlib):
     L = pwlib.lib()
-    assert L.pw_linear(4096, 4096, 0, 32, 4, 4096, 1, 4096, None) == 1      # rows
-    assert L.pw_linear(4096, 4096, 8, 32, 9, 4096, 1, 4096, None) == 1      # bits
-    assert L.pw_linear(None, 4096, 8, 32, 4, 4096, 1, 4096, None) == 1      # null planes
-    assert L.pw_linear(4100, 4096, 8, 32, 4, 4096, 1, 4096, None) == 1      # misaligned
-    assert L.pw_linear(4096, 4096, 8, 32, 4, None, 0, None, None) == 0      # T = 0: nothing to do
+    assert L.pw_linear(4096, 4096, 0, 32, 8, 4, 4096, 1, 4096, None) == 1      # rows
+    assert L.pw_linear(4096, 4096, 8, 32, 8, 9, 4096, 1, 4096, None) == 1      # bits > n_max
+    assert L.pw_linear(4096, 4096, 8, 32, 3, 4, 4096, 1, 4096, None) == 1      # bits > n_max
+    assert L.pw_linear(None, 4096, 8, 32, 8, 4, 4096, 1, 4096, None) == 1      # null planes
+    assert L.pw_linear(4100, 4096, 8, 32, 8, 4, 4096, 1, 4096, None) == 1      # misaligned
+    assert L.pw_linear(4096, 4096, 8, 32, 8, 4, None, 0, None, None) == 0      # T = 0: nothing to do
     assert L.pw_repack_planes(None, 4096, 8, 32, 1, None) == 1
     assert L.pw_repack_planes(4096, 4096, 8, 32, 9, None) == 1
 

@@ -53,23 +53,23 @@ def _identity_lut(rows, b):
 # ---------------------------------------------------------------- page layout
 
 def _paged_reference(planes, cols):
-    """The plane-page layout written out from its definition: plane k, tile
-    (rt, kt) of 128 rows x 8 words at ((k n_rt + rt) n_kt + kt) * 1024 words;
-    row r at 8r words, its two 4-word halves swapped when bit 2 of r is set."""
+    """The paged layout written out from its definition: tile groups of 128
+    rows x 8 words in (row tile, word tile) order, each holding the n planes'
+    tiles of 1024 words one after the other; row r at 8r words within a tile,
+    its two 4-word halves swapped when bit 2 of r is set."""
     n, rows, words = planes.shape
     n_rt, n_kt = -(-rows // 128), -(-words // 8)
-    out = np.zeros((n, n_rt, n_kt, 128, 8), np.uint32)
     padded = np.zeros((n, n_rt * 128, n_kt * 8), np.uint32)
     padded[:, :rows, :words] = planes
+    out = np.zeros((n_rt, n_kt, n, 128, 8), np.uint32)
     for rt in range(n_rt):
         for kt in range(n_kt):
-            tile = padded[:, rt * 128:(rt + 1) * 128, kt * 8:(kt + 1) * 8]
-            for r in range(128):
-                if (r >> 2) & 1:
-                    out[:, rt, kt, r, :] = np.concatenate([tile[:, r, 4:], tile[:, r, :4]], axis=1)
-                else:
-                    out[:, rt, kt, r, :] = tile[:, r, :]
-    return out.reshape(n, -1)
+            for k in range(n):
+                tile = padded[k, rt * 128:(rt + 1) * 128, kt * 8:(kt + 1) * 8]
+                for r in range(128):
+                    row = tile[r]
+                    out[rt, kt, k, r] = np.concatenate([row[4:], row[:4]]) if (r >> 2) & 1 else row
+    return out.reshape(-1)
 
 
 @pytest.mark.parametrize("rows,cols", [(128, 256), (200, 300), (5, 33), (300, 1408)])
@@ -77,7 +77,7 @@ def test_repack_matches_page_layout(pw, rows, cols):
     rng = np.random.default_rng(rows + cols)
     planes = synth.random_planes(rng, 3, rows, cols)
     got = _dev_planes(planes, cols, pw).cpu().numpy().view(np.uint32)
-    assert got.shape[1] * 4 == pw.plane_bytes(rows, cols)
+    assert got.size * 4 == 3 * pw.plane_bytes(rows, cols)
     np.testing.assert_array_equal(got, _paged_reference(planes, cols))
 
 
