@@ -22,8 +22,8 @@ STATUS = {0: "PW_OK", 1: "PW_ERR_INVALID_ARG", 2: "PW_ERR_CUDA", 3: "PW_ERR_OOM"
 EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy",
             "pw_moe_forward_host", "pw_linear", "pw_get_block_bits", "pw_get_routing",
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
-            "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_last_error",
-            "pw_abi_version"]
+            "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
+            "pw_last_error", "pw_abi_version"]
 
 
 class PwError(RuntimeError):
@@ -71,6 +71,7 @@ def lib():
         L.pw_plane_bytes.argtypes = [i32, i32]
         L.pw_plane_bytes.restype = C.c_int64
         L.pw_repack_planes.argtypes = [P, P, i32, i32, i32, P]
+        L.pw_route_static.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P]
         L.pw_last_error.restype = C.c_char_p
         L.pw_abi_version.restype = i32
         for name in EXPORTED:
@@ -125,6 +126,23 @@ def linear(planes, lut, bits: int, x, rows: int, y=None, stream=None):
     check(lib().pw_linear(_ptr(planes), _ptr(lut), rows, cols, n_max, bits, _ptr(x), T, _ptr(y),
                           _stream(stream)))
     return y
+
+
+def route_static(x, router_w, top_k: int, renorm_topk: int, router_bias=None, idx=None, w=None,
+                 stream=None):
+    """Routing alone through pw_route_static (no device allocation inside
+    the library): x bf16 [T][H], router_w fp32 [E][H] -> (idx int32 [T][k],
+    w fp32 [T][k]).  Pass idx / w to reuse output buffers."""
+    import torch
+    T, H = x.shape
+    E = router_w.shape[0]
+    if idx is None:
+        idx = torch.empty((T, top_k), dtype=torch.int32, device=x.device)
+    if w is None:
+        w = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
+    check(lib().pw_route_static(_ptr(x), _ptr(router_w), _ptr(router_bias), T, H, E, top_k,
+                                renorm_topk, _ptr(idx), _ptr(w), _stream(stream)))
+    return idx, w
 
 
 class MoELayer:

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpw_b200.so")
-SOURCES = ["pw_api.cu", "route.cu", "simple.cu", "tc.cu", "repack.cu"]
+SOURCES = ["pw_api.cu", "route.cu", "simple.cu", "tc.cu", "repack.cu", "route_static.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

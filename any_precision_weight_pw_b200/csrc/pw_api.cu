@@ -46,6 +46,13 @@ pw_status_t fail(pw_status_t st, const char* fmt, ...) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
+// Error text for calls implemented in other translation units.
+pw_status_t pw::record_error(pw_status_t st, const char* msg) { return fail(st, "%s", msg); }
+
+namespace {
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
 // library needs no link-time dependency on libcuda.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -86,6 +86,9 @@ struct SimpleParams {
   const uint16_t* lin_lut;
 };
 
+// Sets the calling thread's pw_last_error() text and returns st (pw_api.cu).
+pw_status_t record_error(pw_status_t st, const char* msg);
+
 // Launchers (defined in the .cu files).
 cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s);
 cudaError_t launch_repack(const uint32_t* src, uint32_t* dst, int rows, int cols, int n_planes,

@@ -195,6 +195,39 @@ pw_status_t pw_profile_read(pw_moe_t* h, float* ms, int32_t n, int32_t* n_forwar
 /* Number of kernel launches one forward of this handle issues for T tokens. */
 int32_t pw_forward_launches(const pw_moe_t* h, int32_t T);
 
+/* ---- routing without device allocation ------------------------------- */
+
+/* The router alone, allocating nothing: the same routing as pw_moe_forward
+ * (logits, top-k, softmax, per-expert bucketing in one launch), with its
+ * scratch in one fixed device array of PW_ROUTE_STATIC_SCRATCH_BYTES per
+ * device instead of a handle's workspace.  The PagedWeight pages have no
+ * counterpart of this call; it serves callers that cannot allocate device
+ * memory where they route (all of HBM already handed to weight pages and KV
+ * cache, or no room for cudaMalloc's implicit device synchronisation in the
+ * middle of an asynchronous page move).
+ *   d_x bf16 [T][hidden], d_router_w fp32 [n_experts][hidden],
+ *   d_router_bias fp32 [n_experts] or NULL (device, caller-owned);
+ *   d_idx int32 [T][top_k] and d_w fp32 [T][top_k] receive the selected
+ *   experts in selection order and their weights, exactly as pw_get_routing
+ *   reports them after a forward of the same x.
+ *   0 <= T <= PW_ROUTE_STATIC_MAX_TOKENS, 1 <= top_k <= min(n_experts, 8),
+ *   n_experts <= 128, renorm_topk 0 or 1; anything else is PW_ERR_INVALID_ARG
+ *   with nothing enqueued.  T = 0 returns PW_OK at once.
+ * The first call on a device looks up the array's address
+ * (cudaGetSymbolAddress; PW_ERR_CUDA if that fails) and caches it; make that
+ * first call before any stream capture on the device begins.
+ * Races: the array is shared by every call on the device in the process.  Two
+ * calls whose kernels can overlap (different streams without an event between
+ * them, or several host threads) corrupt each other's scratch and results;
+ * the caller serialises calls per device, e.g. by issuing them all on one
+ * stream. */
+#define PW_ROUTE_STATIC_MAX_TOKENS 256
+#define PW_ROUTE_STATIC_SCRATCH_BYTES 156672 /* logits 128 KB + lists and counter */
+pw_status_t pw_route_static(const uint16_t* d_x, const float* d_router_w,
+                            const float* d_router_bias, int32_t T, int32_t hidden,
+                            int32_t n_experts, int32_t top_k, int32_t renorm_topk,
+                            int32_t* d_idx, float* d_w, pw_stream_t stream);
+
 const char* pw_last_error(void);
 int32_t pw_abi_version(void);
 

@@ -97,6 +97,15 @@ def test_linear_rejects_bad_args(pwlib):
     assert L.pw_linear(4096, 4096, 8, 32, 8, 4, None, 0, None, None) == 0      # T = 0: nothing to do
     assert L.pw_repack_planes(None, 4096, 8, 32, 1, None) == 1
     assert L.pw_repack_planes(4096, 4096, 8, 32, 9, None) == 1
+    # pw_route_static: limits are checked before anything touches a device
+    assert L.pw_route_static(4096, 4096, None, 257, 64, 8, 2, 1, 4096, 4096, None) == 1  # T > 256
+    assert L.pw_route_static(4096, 4096, None, -1, 64, 8, 2, 1, 4096, 4096, None) == 1   # T < 0
+    assert L.pw_route_static(4096, 4096, None, 4, 64, 129, 2, 1, 4096, 4096, None) == 1  # E > 128
+    assert L.pw_route_static(4096, 4096, None, 4, 64, 4, 5, 1, 4096, 4096, None) == 1    # k > E
+    assert L.pw_route_static(4096, 4096, None, 4, 64, 60, 9, 0, 4096, 4096, None) == 1   # k > 8
+    assert L.pw_route_static(4096, 4096, None, 4, 64, 8, 2, 2, 4096, 4096, None) == 1    # renorm
+    assert L.pw_route_static(4096, 4096, None, 4, 0, 8, 2, 1, 4096, 4096, None) == 1     # hidden
+    assert L.pw_route_static(None, None, None, 0, 64, 8, 2, 1, None, None, None) == 0    # T = 0
 
 
 def test_plane_bytes(pwlib):
