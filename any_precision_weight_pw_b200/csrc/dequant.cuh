@@ -10,19 +10,21 @@
 // half and (8j + m + 4) in its high half.  The token tile is permuted the same
 // way, so the contraction is unchanged.
 //
-// Lookups, chosen per bitwidth:
-//   b <= 3   the row's 8-entry LUT sits in four registers as separate low-
-//            and high-byte tables; one byte permute (PRMT) looks up four
-//            weights' low bytes, one their high bytes, two more interleave
-//            them into fp16 pairs.  Selectors are 3-bit codes in nibbles.
-//   b == 4   4-bit codes in nibbles address a shared-memory table.
-//   b >= 5   an 8x8 bit-matrix transpose of the planes (zero planes for
-//            k >= b) gives one code per byte, which addresses the table.
-// The shared-memory table holds entry v of local row r in the low half of
-// word v * 128 + r, so the 32 threads of a warp (32 consecutive rows) read 32
-// different banks; the byte offset of an entry is (v << 9) | 4r, formed with
-// one shift and one LOP3 per weight.  Right shifts are written as high
-// multiplies so they issue on the FMA pipe, not the integer ALU pipe.
+// Codes come from an 8x8 bit-matrix transpose of plane words: input row p
+// becomes bit p of every byte, so byte n of output row q collects column
+// 8n + q.  The byte then IS an address byte: one byte permute (PRMT) puts it
+// next to the thread's row byte, and one shared-memory load fetches the
+// entry.  Two tables, both 128 local rows (threads) x at most 64 KB:
+//   b <= 3   pair table: the byte holds (v1 << (b + 1)) | (v2 << 1) | h for
+//            columns c (v1) and c + 4 (v2) and the row half h = r >= 64;
+//            the 32-bit entry at byte (byte << 8) | 4 (r mod 64) is the fp16
+//            pair (LUT[v1], LUT[v2]) -- one load gives one output register.
+//   b >= 4   single table: the byte holds v; the fp16 entry of row r is at
+//            byte (v << 8) | 4 (r mod 64) | 2h (rows r and r + 64 share a
+//            word).  Two loads and one multiply-add give one output register.
+// In both the 32 threads of a warp (32 consecutive rows) read 32 different
+// banks.  Shifts are written as multiplies (left) and high multiplies (right)
+// so they issue on the FMA pipe; the ALU pipe keeps the LOP3 and PRMT work.
 //
 // Everything here is __host__ __device__ so the bit manipulation can be
 // checked on the CPU (tests/dequant_selftest.cpp) against a plain unpack.
@@ -73,154 +75,106 @@ PW_HD uint32_t shr(uint32_t x) {
 // x << S for S >= 0, x >> -S for S < 0.
 template <int S>
 PW_HD uint32_t shl(uint32_t x) {
-  if (S >= 0) return x << (S >= 0 ? S : 0);
+  if (S >= 0) return x * (1u << (S >= 0 ? S : 0));
   return shr<(S < 0 ? -S : 0)>(x);
 }
 // (hi << 16) | lo for 16-bit lo and hi, as a multiply-add (FMA pipe).
 PW_HD uint32_t pack16(uint32_t lo, uint32_t hi) { return hi * 65536u + lo; }
 
-// ---- nibble codes ----------------------------------------------------------
-// Nibble n of the result = the NB-bit number whose bits come from planes
-// P[K0] (most significant) .. P[K0+NB-1] at column 4n + M.
-template <int M, int K0, int NB, int B>
-PW_HD uint32_t nibble_codes(const uint32_t (&P)[B]) {
-  uint32_t s = 0;
+// ---- 8x8 bit-matrix transpose --------------------------------------------------
+// One delta swap: the bits of a selected by ~m trade places with the bits of b
+// selected by m, S positions apart.
+template <int S>
+PW_HD void delta_swap(uint32_t& a, uint32_t& b, uint32_t m) {
+  const uint32_t a2 = (a & m) | (shl<S>(b) & ~m);
+  const uint32_t b2 = (b & ~m) | (shr<S>(a) & m);
+  a = a2;
+  b = b2;
+}
+
+// In place: afterwards X[q] byte n bit p = (input X[p] bit 8n + q).
+PW_HD void transpose8(uint32_t (&X)[8]) {
 #pragma unroll
-  for (int i = 0; i < NB; ++i) {
-    const int j = NB - 1 - i;  // nibble bit this plane supplies
-    // bit 4n + j  <-  plane bit 4n + M
-    uint32_t t;
-    switch (j - M) {
-      case -3: t = shl<-3>(P[K0 + i]); break;
-      case -2: t = shl<-2>(P[K0 + i]); break;
-      case -1: t = shl<-1>(P[K0 + i]); break;
-      case 0: t = P[K0 + i]; break;
-      case 1: t = shl<1>(P[K0 + i]); break;
-      case 2: t = shl<2>(P[K0 + i]); break;
-      default: t = shl<3>(P[K0 + i]); break;
-    }
-    s |= t & (0x11111111u << j);
-  }
-  return s;
-}
-
-// ---- b <= 3: register tables -----------------------------------------------
-struct RegLut {
-  uint32_t lo0, lo1, hi0, hi1;  // low/high bytes of entries 0-3 and 4-7
-};
-
-// w[i] = fp16 entries 2i (low half) and 2i+1 (high half); entries >= 2^b are
-// never selected.
-template <int B>
-PW_HD RegLut make_reg_lut(const uint32_t* w) {
-  uint32_t e[4] = {0u, 0u, 0u, 0u};
+  for (int i = 0; i < 4; ++i) delta_swap<4>(X[i], X[i + 4], 0x0F0F0F0Fu);
 #pragma unroll
-  for (int i = 0; i < (1 << B) / 2; ++i) e[i] = w[i];
-  RegLut L;
-  L.lo0 = prmt(e[0], e[1], 0x6420);
-  L.hi0 = prmt(e[0], e[1], 0x7531);
-  L.lo1 = prmt(e[2], e[3], 0x6420);
-  L.hi1 = prmt(e[2], e[3], 0x7531);
-  return L;
-}
-
-template <int M, int B>
-PW_HD void reg_quarter(const uint32_t (&P)[B], const RegLut& L, uint32_t* out) {
-  const uint32_t s = nibble_codes<M, 0, B, B>(P);  // codes of columns 4n + M
+  for (int i = 0; i < 8; ++i)
+    if (!(i & 2)) delta_swap<2>(X[i], X[i + 2], 0x33333333u);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t sel = h ? shr<16>(s) : s;
-    const uint32_t lo = prmt(L.lo0, L.lo1, sel);
-    const uint32_t hi = prmt(L.hi0, L.hi1, sel);
-    out[4 * M + 2 * h + 0] = prmt(lo, hi, 0x5140);  // columns (8(2h) + M, +4)
-    out[4 * M + 2 * h + 1] = prmt(lo, hi, 0x7362);  // columns (8(2h+1) + M, +4)
-  }
+  for (int i = 0; i < 8; i += 2) delta_swap<1>(X[i], X[i + 1], 0x55555555u);
 }
 
-template <int B>
-PW_HD void dq_word_reg(const uint32_t (&P)[B], const RegLut& L, uint32_t* out) {
-  static_assert(B >= 1 && B <= 3, "register tables hold at most 8 entries");
-  reg_quarter<0, B>(P, L, out);
-  reg_quarter<1, B>(P, L, out);
-  reg_quarter<2, B>(P, L, out);
-  reg_quarter<3, B>(P, L, out);
+// The same for output rows 0..3 only (X[4..7] are left undefined).
+PW_HD void transpose8_lo(uint32_t (&X)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) X[i] = (X[i] & 0x0F0F0F0Fu) | (shl<4>(X[i + 4]) & 0xF0F0F0F0u);
+  delta_swap<2>(X[0], X[2], 0x33333333u);
+  delta_swap<2>(X[1], X[3], 0x33333333u);
+  delta_swap<1>(X[0], X[1], 0x55555555u);
+  delta_swap<1>(X[2], X[3], 0x55555555u);
 }
 
-// ---- shared-memory tables ----------------------------------------------------
-// Lds(x) returns the 16-bit entry at byte offset x of the table region.
-// r4 = 4 * (local row), in bits 2..8.
-
-// b == 4: entry offset of nibble n of s = ((s >> 4n) & 15) << 9 | r4.
+// Address of the entry for byte N of x: byte 0 from rowb (the row byte),
+// byte 1 = byte N of x, bytes 2-3 from byte 1 of rowb (zero).
 template <int N>
-PW_HD uint32_t nib_addr(uint32_t s, uint32_t r4) {
-  return (shl<9 - 4 * N>(s) & (0xFu << 9)) | r4;
+PW_HD uint32_t code_addr(uint32_t x, uint32_t rowb) {
+  return prmt(x, rowb, 0x5504u | (static_cast<uint32_t>(N) << 4));
 }
 
-template <int M, class Lds>
-PW_HD void smem4_quarter(const uint32_t (&P)[4], uint32_t r4, Lds lds, uint32_t* out) {
-  const uint32_t s = nibble_codes<M, 0, 4, 4>(P);  // 4-bit codes of columns 4n + M
-  out[4 * M + 0] = pack16(lds(nib_addr<0>(s, r4)), lds(nib_addr<1>(s, r4)));
-  out[4 * M + 1] = pack16(lds(nib_addr<2>(s, r4)), lds(nib_addr<3>(s, r4)));
-  out[4 * M + 2] = pack16(lds(nib_addr<4>(s, r4)), lds(nib_addr<5>(s, r4)));
-  out[4 * M + 3] = pack16(lds(nib_addr<6>(s, r4)), lds(nib_addr<7>(s, r4)));
-}
+// Row bytes: pair table 4 (r mod 64), single table 4 (r mod 64) + 2h.
+PW_HD uint32_t pair_row_byte(uint32_t r) { return 4u * (r & 63u); }
+PW_HD uint32_t single_row_byte(uint32_t r) { return 4u * (r & 63u) + 2u * (r >> 6); }
 
-// b >= 5: X[q] byte n = 8-bit code (zero-padded below for b < 8) of column
-// 8n + q, after transposing the 8x8 bit blocks of the planes.
-template <int B>
-PW_HD void transpose_codes(const uint32_t (&P)[B], uint32_t (&X)[8]) {
-  // X[p] = plane 7 - p (code bit p of an 8-bit code), zero for planes >= B
+// Byte offsets of table entries (for writing the tables).
+PW_HD uint32_t pair_offset(uint32_t v1, uint32_t v2, int b, uint32_t r) {
+  const uint32_t byte = (v1 << (b + 1)) | (v2 << 1) | (r >> 6);
+  return (byte << 8) | pair_row_byte(r);
+}
+PW_HD uint32_t single_offset(uint32_t v, uint32_t r) { return (v << 8) | single_row_byte(r); }
+
+// b <= 3.  Lds32(x) returns the 32-bit entry at byte offset x.
+template <int B, class Lds32>
+PW_HD void dq_word_pair(const uint32_t (&P)[B], uint32_t r, Lds32 lds32, uint32_t* out) {
+  static_assert(B >= 1 && B <= 3, "pair tables serve b = 1..3");
+  uint32_t X[8];
+  // byte bit 0 = row half; bits 1..B = code of column c + 4 (moved down 4
+  // columns); bits B+1..2B = code of column c; plane 0 is the code's MSB
+  X[0] = (r >> 6) ? 0xFFFFFFFFu : 0u;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) X[p] = (7 - p < B) ? P[(7 - p < B) ? 7 - p : 0] : 0u;
-  // 4x4 blocks: rows i, i+4
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t t = (shr<4>(X[i]) ^ X[i + 4]) & 0x0F0F0F0Fu;
-    X[i + 4] ^= t;
-    X[i] ^= t << 4;
+  for (int j = 0; j < B; ++j) {
+    X[1 + j] = shr<4>(P[B - 1 - j]);
+    X[1 + B + j] = P[B - 1 - j];
   }
-  // 2x2 blocks: rows i, i+2
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (i & 2) continue;
-    const uint32_t t = (shr<2>(X[i]) ^ X[i + 2]) & 0x33333333u;
-    X[i + 2] ^= t;
-    X[i] ^= t << 2;
-  }
-  // single bits: rows i, i+1
+  for (int p = 1 + 2 * B; p < 8; ++p) X[p] = 0u;
+  transpose8_lo(X);
+  const uint32_t rowb = pair_row_byte(r);
 #pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    const uint32_t t = (shr<1>(X[i]) ^ X[i + 1]) & 0x55555555u;
-    X[i + 1] ^= t;
-    X[i] ^= t << 1;
+  for (int m = 0; m < 4; ++m) {
+    // byte j of X[m]: columns 8j + m and 8j + m + 4
+    out[4 * m + 0] = lds32(code_addr<0>(X[m], rowb));
+    out[4 * m + 1] = lds32(code_addr<1>(X[m], rowb));
+    out[4 * m + 2] = lds32(code_addr<2>(X[m], rowb));
+    out[4 * m + 3] = lds32(code_addr<3>(X[m], rowb));
   }
 }
 
-// Offset of the entry for byte n of x (an 8-bit code v << (8 - B)).
-template <int N, int B>
-PW_HD uint32_t byte_addr(uint32_t x, uint32_t r4) {
-  return (shl<B + 1 - 8 * N>(x) & (((1u << B) - 1u) << 9)) | r4;
-}
-
-template <int B, class Lds>
-PW_HD void dq_word_smem(const uint32_t (&P)[B], uint32_t r4, Lds lds, uint32_t* out) {
-  if constexpr (B == 4) {
-    smem4_quarter<0>(P, r4, lds, out);
-    smem4_quarter<1>(P, r4, lds, out);
-    smem4_quarter<2>(P, r4, lds, out);
-    smem4_quarter<3>(P, r4, lds, out);
-  } else {
-    static_assert(B >= 5 && B <= 8, "transposed codes serve b = 5..8");
-    uint32_t X[8];
-    transpose_codes<B>(P, X);
+// b >= 4.  Lds16(x) returns the 16-bit entry at byte offset x.
+template <int B, class Lds16>
+PW_HD void dq_word_single(const uint32_t (&P)[B], uint32_t r, Lds16 lds16, uint32_t* out) {
+  static_assert(B >= 4 && B <= 8, "single tables serve b = 4..8");
+  uint32_t X[8];
+  // byte bit p = code bit p (right-aligned code); plane 0 is the MSB
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      // columns 8j + m (X[m] byte j) and 8j + m + 4 (X[m+4] byte j)
-      out[4 * m + 0] = pack16(lds(byte_addr<0, B>(X[m], r4)), lds(byte_addr<0, B>(X[m + 4], r4)));
-      out[4 * m + 1] = pack16(lds(byte_addr<1, B>(X[m], r4)), lds(byte_addr<1, B>(X[m + 4], r4)));
-      out[4 * m + 2] = pack16(lds(byte_addr<2, B>(X[m], r4)), lds(byte_addr<2, B>(X[m + 4], r4)));
-      out[4 * m + 3] = pack16(lds(byte_addr<3, B>(X[m], r4)), lds(byte_addr<3, B>(X[m + 4], r4)));
-    }
+  for (int p = 0; p < 8; ++p) X[p] = (p < B) ? P[(p < B) ? B - 1 - p : 0] : 0u;
+  transpose8(X);
+  const uint32_t rowb = single_row_byte(r);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    // columns 8j + m (X[m] byte j) and 8j + m + 4 (X[m + 4] byte j)
+    out[4 * m + 0] = pack16(lds16(code_addr<0>(X[m], rowb)), lds16(code_addr<0>(X[m + 4], rowb)));
+    out[4 * m + 1] = pack16(lds16(code_addr<1>(X[m], rowb)), lds16(code_addr<1>(X[m + 4], rowb)));
+    out[4 * m + 2] = pack16(lds16(code_addr<2>(X[m], rowb)), lds16(code_addr<2>(X[m + 4], rowb)));
+    out[4 * m + 3] = pack16(lds16(code_addr<3>(X[m], rowb)), lds16(code_addr<3>(X[m + 4], rowb)));
   }
 }
 

@@ -75,14 +75,15 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
 // Shared memory (offsets from a 1024-byte aligned base; compile-time so the
 // table lookups fold the base into the load's immediate offset).
-constexpr uint32_t kOffLut = 0;                // 128 rows x 128 words x 4 B
-constexpr uint32_t kLutBytes = 128u * 128u * 4u;
+constexpr uint32_t kOffLut = 0;                // 256 code lines x 64 row words x 4 B
+constexpr uint32_t kLutBytes = 256u * 64u * 4u;
 constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
 constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
 constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
 constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 4 + 2;
 constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-constexpr uint32_t kSmemTotal = kOffMisc + 16 + 4 * (kMaxGroups + 2);
+constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 4 * (kMaxGroups + 2);
+constexpr uint32_t kSmemTotal = kOffSlotUser + 4 * kNSlot;
 static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
 
 // Plane stages take `bits` consecutive slots of the ring; a stage that would
@@ -108,6 +109,12 @@ __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(b)) : "memory");
+}
+// One arrival for the whole warp, after every lane's earlier accesses (the
+// warp barrier orders them before lane 0's release).
+__device__ __forceinline__ void mbar_arrive_warp(uint64_t* b) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(b);
 }
 __device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(b)),
@@ -189,6 +196,15 @@ __device__ __forceinline__ void tc_commit(uint64_t* b) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_addr(b))
                : "memory");
+}
+// One lane of the (converged) warp, the same lane every time.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n.reg .pred P1;\n.reg .b32 r;\nelect.sync r|P1, %1;\nselp.u32 %0, 1, 0, P1;\n}\n"
+      : "=r"(pred)
+      : "r"(0xffffffffu));
+  return pred != 0;
 }
 __device__ __forceinline__ void tc_mma(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc,
                                        uint32_t acc) {
@@ -274,10 +290,13 @@ struct Item {
   int g, row0, tok0, ntok, pos0, split, rows, cols, npass, s_begin, s_end;
 };
 
+// Items are visited in increasing order by every role, so the group search
+// resumes from the previous item's group (gh).
 __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix, int G,
-                                            int i, Item& it) {
-  int g = 0;
+                                            int i, Item& it, int& gh) {
+  int g = gh;
   while (g + 1 < G && s_prefix[g + 1] <= i) ++g;
+  gh = g;
   const int local = i - s_prefix[g];
   int n, pos0;
   if (p.mode == kTcLinear) {
@@ -330,7 +349,7 @@ __device__ __forceinline__ uint4 read_plane_chunk(uint32_t slot_off, int r, int 
 // All dequantiser threads meet (a bounded wait, unlike a hardware barrier,
 // so a warp that gave up cannot leave the others blocked).
 __device__ __forceinline__ bool dq_sync(uint64_t* bar, uint32_t& phase, const Ctl& ctl) {
-  mbar_arrive(bar);
+  mbar_arrive_warp(bar);
   const bool ok = mbar_wait_warp(bar, phase, ctl);
   phase ^= 1u;
   return ok;
@@ -342,39 +361,19 @@ struct DequantState {
   uint32_t a_ctr;      // stages processed by this K half
 };
 
-// b = 8 tables are packed two entries per word: word (v >> 1) * 128 + r.
-// The offset of the entry for byte n of x (an 8-bit code) is
-// ((v >> 1) << 9) | ((v & 1) << 1) | 4r.
-template <int N>
-__device__ __forceinline__ uint32_t byte_addr8(uint32_t x, uint32_t r4) {
-  const uint32_t a = (dq::shl<8 - 8 * N>(x) & 0xFE00u) | r4;
-  return (dq::shl<1 - 8 * N>(x) & 2u) | a;
-}
-__device__ __forceinline__ void dq_word8(const uint32_t (&P)[8], uint32_t r4, uint32_t* out) {
-  uint32_t X[8];
-  dq::transpose_codes<8>(P, X);
-  auto lds = [](uint32_t x) -> uint32_t {
-    return *reinterpret_cast<const uint16_t*>(pw_tc_smem + kOffLut + x);
-  };
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    out[4 * m + 0] = dq::pack16(lds(byte_addr8<0>(X[m], r4)), lds(byte_addr8<0>(X[m + 4], r4)));
-    out[4 * m + 1] = dq::pack16(lds(byte_addr8<1>(X[m], r4)), lds(byte_addr8<1>(X[m + 4], r4)));
-    out[4 * m + 2] = dq::pack16(lds(byte_addr8<2>(X[m], r4)), lds(byte_addr8<2>(X[m + 4], r4)));
-    out[4 * m + 3] = dq::pack16(lds(byte_addr8<3>(X[m], r4)), lds(byte_addr8<3>(X[m + 4], r4)));
-  }
-}
-
 template <int B>
-__device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegLut& L,
+__device__ bool dequant_stages(const Item& it, int grp, int quad,
                                uint64_t* sf, uint64_t* se, uint64_t* af, uint64_t* ae,
                                uint32_t tmem_base, DequantState& st, const Ctl& ctl) {
   const int lane = threadIdx.x & 31;
   const int r = 32 * quad + lane;
-  const uint32_t r4 = 4u * static_cast<uint32_t>(r);
+  const uint32_t ru = static_cast<uint32_t>(r);
   const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * quad) << 16);
-  auto lds = [](uint32_t x) -> uint32_t {
+  auto lds16 = [](uint32_t x) -> uint32_t {
     return *reinterpret_cast<const uint16_t*>(pw_tc_smem + kOffLut + x);
+  };
+  auto lds32 = [](uint32_t x) -> uint32_t {
+    return *reinterpret_cast<const uint32_t*>(pw_tc_smem + kOffLut + x);
   };
   for (int s = it.s_begin; s < it.s_end; ++s) {
     uint32_t P[4][B];
@@ -389,7 +388,7 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegL
       P[2][k] = q4.z;
       P[3][k] = q4.w;
     }
-    mbar_arrive(&se[e]);
+    mbar_arrive_warp(&se[e]);
     st.stage_ctr++;
     const uint32_t a_idx = 2u * st.a_ctr + static_cast<uint32_t>(grp);
     const uint32_t qa = a_idx % kNA;
@@ -399,20 +398,17 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad, const dq::RegL
     for (int h = 0; h < 2; ++h) {
       uint32_t out[32];
       if constexpr (B <= 3) {
-        dq::dq_word_reg<B>(P[2 * h], L, out);
-        dq::dq_word_reg<B>(P[2 * h + 1], L, out + 16);
-      } else if constexpr (B <= 7) {
-        dq::dq_word_smem<B>(P[2 * h], r4, lds, out);
-        dq::dq_word_smem<B>(P[2 * h + 1], r4, lds, out + 16);
+        dq::dq_word_pair<B>(P[2 * h], ru, lds32, out);
+        dq::dq_word_pair<B>(P[2 * h + 1], ru, lds32, out + 16);
       } else {
-        dq_word8(P[2 * h], r4, out);
-        dq_word8(P[2 * h + 1], r4, out + 16);
+        dq::dq_word_single<B>(P[2 * h], ru, lds16, out);
+        dq::dq_word_single<B>(P[2 * h + 1], ru, lds16, out + 16);
       }
       tmem_st32(tcol + 32 * h, out);
     }
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(&af[qa]);
+    mbar_arrive_warp(&af[qa]);
     st.a_ctr++;
   }
   return true;
@@ -441,7 +437,9 @@ __device__ __forceinline__ void lut_prefetch(const Item& it, const Pass& ps, int
   if (b <= 3) {
     const uint32_t* src = reinterpret_cast<const uint32_t*>(row);
     uint32_t w[4] = {0u, 0u, 0u, 0u};
-    for (int i = 0; i < (1 << b) / 2; ++i) w[i] = src[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < (1 << b) / 2) w[i] = src[i];
     f.v[0] = make_uint4(w[0], w[1], w[2], w[3]);
     return;
   }
@@ -452,15 +450,35 @@ __device__ __forceinline__ void lut_prefetch(const Item& it, const Pass& ps, int
 }
 
 __device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int grp, int r,
-                                            const LutPrefetch& f, dq::RegLut& L) {
+                                            const LutPrefetch& f) {
   if (!f.live) return;
   const int b = ps.bits;
-  uint32_t* dst = reinterpret_cast<uint32_t*>(pw_tc_smem + kOffLut + 4u * r);
+  const uint32_t ru = static_cast<uint32_t>(r);
   if (b <= 3) {
-    const uint32_t w[4] = {f.v[0].x, f.v[0].y, f.v[0].z, f.v[0].w};
-    L = dq::make_reg_lut<3>(w);
+    // pair table: entry (v1, v2) = (LUT[v1], LUT[v2]); this thread writes the
+    // entries with v1 in its half of the codes
+    const uint64_t w01 = f.v[0].x | (static_cast<uint64_t>(f.v[0].y) << 32);
+    const uint64_t w23 = f.v[0].z | (static_cast<uint64_t>(f.v[0].w) << 32);
+    auto entry = [&](int v) -> uint32_t {
+      return static_cast<uint32_t>(((v < 4) ? w01 : w23) >> (16 * (v & 3))) & 0xFFFFu;
+    };
+    const int n = 1 << b, half = n >> 1;
+    for (int v1 = grp * half; v1 < grp * half + half; ++v1) {
+      const uint32_t lo = entry(v1);
+      for (int v2 = 0; v2 < n; ++v2) {
+        const uint32_t hi = entry(v2);
+        *reinterpret_cast<uint32_t*>(pw_tc_smem + kOffLut + dq::pair_offset(v1, v2, b, ru)) =
+            lo | (hi << 16);
+      }
+    }
     return;
   }
+  // single table: entry v of row r at dq::single_offset(v, r); this thread
+  // writes entries grp * half .. grp * half + half - 1
+  auto put = [&](int v, uint32_t e) {
+    *reinterpret_cast<uint16_t*>(pw_tc_smem + kOffLut + dq::single_offset(v, ru)) =
+        static_cast<uint16_t>(e);
+  };
   const int half = 1 << (b - 1);
   if (b <= 6) {
 #pragma unroll
@@ -468,36 +486,17 @@ __device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int 
       if (i >= (1 << (b - 4))) break;
       const uint32_t e4[4] = {f.v[i].x, f.v[i].y, f.v[i].z, f.v[i].w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t ent = (e & 1) ? (e4[e >> 1] >> 16) : (e4[e >> 1] & 0xFFFFu);
-        dst[(grp * half + 8 * i + e) * 128] = ent;
-      }
+      for (int e = 0; e < 8; ++e) put(grp * half + 8 * i + e, (e & 1) ? (e4[e >> 1] >> 16) : e4[e >> 1]);
     }
     return;
   }
   const uint16_t* row = ps.lut + (static_cast<size_t>(it.row0 + r) << b);
-  if (b == 8) {
-    // packed: word j (entries 2j, 2j+1) at (j << 9) | 4r; this thread's 64 words
-    const uint4* src = reinterpret_cast<const uint4*>(row) + grp * 16;
-    for (int i = 0; i < 16; ++i) {
-      const uint4 v = src[i];
-      const uint32_t j = static_cast<uint32_t>(grp * 64 + 4 * i);
-      dst[(j + 0) * 128] = v.x;
-      dst[(j + 1) * 128] = v.y;
-      dst[(j + 2) * 128] = v.z;
-      dst[(j + 3) * 128] = v.w;
-    }
-    return;
-  }
   const uint4* src = reinterpret_cast<const uint4*>(row + grp * half);
   for (int i = 0; i < half / 8; ++i) {
     const uint4 v = src[i];
     const uint32_t e4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t ent = (e & 1) ? (e4[e >> 1] >> 16) : (e4[e >> 1] & 0xFFFFu);
-      dst[(grp * half + 8 * i + e) * 128] = ent;
-    }
+    for (int e = 0; e < 8; ++e) put(grp * half + 8 * i + e, (e & 1) ? (e4[e >> 1] >> 16) : e4[e >> 1]);
   }
 }
 
@@ -558,6 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   int* s_prefix = reinterpret_cast<int*>(smem + kOffMisc + 16);
+  uint32_t* slot_user = reinterpret_cast<uint32_t*>(smem + kOffSlotUser);  // producer only
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {
       mbar_init(&sf[i], 1);
-      mbar_init(&se[i], kDqThreads);
+      mbar_init(&se[i], kDqThreads / 32);
     }
     for (int i = 0; i < kNB; ++i) {
       mbar_init(&bfull[i], p.mode == kTcLinear ? 32 : 1);
@@ -574,14 +574,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&df[i], 1);
-      mbar_init(&de[i], 128);
+      mbar_init(&de[i], 4);
     }
     for (int i = 0; i < kNA; ++i) {
-      mbar_init(&af[i], 128);
+      mbar_init(&af[i], 4);
       mbar_init(&ae[i], 1);
     }
     mbar_init(drain, 1);
-    mbar_init(dqbar, kDqThreads);
+    mbar_init(dqbar, kDqThreads / 32);
+    for (int k = 0; k < kNSlot; ++k) slot_user[k] = 0u;
     // the table offsets assume a 1024-byte aligned dynamic shared memory base
     *s_abort = (smem_addr(smem) & 1023u) ? 1 : 0;
     if (*s_abort && p.err) atomicExch(p.err, PW_ERR_UNSUPPORTED);
@@ -620,6 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   if (warp < 8) {
     // ------------------------------------------------ dequantisers
     DequantState st{0u, 0u, 0u};
+    int gh = 0;
     const int grp = warp >> 2, quad = warp & 3;
     const int r = 32 * quad + lane;
     uint32_t sync_phase = 0;
@@ -630,33 +632,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     Item it;
     LutPrefetch pre;
     if (i < total) {
-      decode_item(p, s_prefix, G, i, it);
+      decode_item(p, s_prefix, G, i, it, gh);
       lut_prefetch(it, get_pass(p, it, 0), grp, r, pre);
     }
     while (i < total && ok) {
       const Pass ps = get_pass(p, it, q);
       // every thread is done with the previous pass's table before it changes
       if (!dq_sync(dqbar, sync_phase, ctl)) break;
-      dq::RegLut L{0u, 0u, 0u, 0u};
-      lut_install(it, ps, grp, r, pre, L);
+      lut_install(it, ps, grp, r, pre);
       if (!dq_sync(dqbar, sync_phase, ctl)) break;
       const Item cur = it;
       int ni = i, nq = q + 1;
       if (nq >= it.npass) {
         ni = i + gridDim.x;
         nq = 0;
-        if (ni < total) decode_item(p, s_prefix, G, ni, it);
+        if (ni < total) decode_item(p, s_prefix, G, ni, it, gh);
       }
       if (ni < total) lut_prefetch(it, get_pass(p, it, nq), grp, r, pre);
       switch (ps.bits) {
-        case 1: ok = dequant_stages<1>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 2: ok = dequant_stages<2>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 3: ok = dequant_stages<3>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 4: ok = dequant_stages<4>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 5: ok = dequant_stages<5>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 6: ok = dequant_stages<6>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 7: ok = dequant_stages<7>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
-        default: ok = dequant_stages<8>(cur, grp, quad, L, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 1: ok = dequant_stages<1>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 2: ok = dequant_stages<2>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 3: ok = dequant_stages<3>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 4: ok = dequant_stages<4>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 5: ok = dequant_stages<5>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 6: ok = dequant_stages<6>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 7: ok = dequant_stages<7>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        default: ok = dequant_stages<8>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
       }
       i = ni;
       q = nq;
@@ -665,12 +666,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     // ------------------------------------------------ producer (planes)
     if (lane == 0) {
       uint32_t t = 0, ring_end = 0;
-      uint32_t rs[kNS], re[kNS];  // slot range of each stage in flight
+      int gh = 0;
       bool ok = true;
       const int n_max = (p.mode == kTcLinear) ? p.lin_n_max : p.n_max;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
-        decode_item(p, s_prefix, G, i, it);
+        decode_item(p, s_prefix, G, i, it, gh);
         const int n_kt = pages::k_tiles(it.cols);
         const int rt = it.row0 / kTileRows;
         for (int q = 0; q < it.npass && ok; ++q) {
@@ -683,18 +684,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
               ok = false;
               break;
             }
-            // ... and so are the slots: wait for the latest earlier stage
-            // still holding any of them (stages are released in order)
-            for (uint32_t j = 1; j < kNS && j <= t; ++j) {
-              const uint32_t u = t - j;
-              if (rs[u % kNS] < start + ps.bits && start < re[u % kNS]) {
-                if (!mbar_wait(&se[u % kNS], (u / kNS) & 1u, ctl)) ok = false;
+            // ... and so are the slots: wait for the latest earlier stage that
+            // used any of them (slot_user holds stage index + 1).  Stages are
+            // released in order, so users older than t - kNS are already free.
+            uint32_t u1 = 0;
+#pragma unroll
+            for (int k = 0; k < PW_MAX_BITS; ++k)
+              if (k < ps.bits) u1 = max(u1, slot_user[start + k]);
+            if (u1 > 0 && u1 - 1 + kNS > t) {
+              const uint32_t u = u1 - 1;
+              if (!mbar_wait(&se[u % kNS], (u / kNS) & 1u, ctl)) {
+                ok = false;
                 break;
               }
             }
-            if (!ok) break;
-            rs[e] = start;
-            re[e] = start + ps.bits;
+#pragma unroll
+            for (int k = 0; k < PW_MAX_BITS; ++k)
+              if (k < ps.bits) slot_user[start + k] = t + 1;
             const int64_t grp_idx = static_cast<int64_t>(rt) * n_kt + s;
             const uint32_t bytes = static_cast<uint32_t>(ps.bits) * kSlotBytes;
             mbar_arrive_tx(&sf[e], bytes);
@@ -712,10 +718,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   } else if (warp == kWarpLoader) {
     // ------------------------------------------------ token-tile loader
     uint32_t b_ctr = 0;
+    int gh = 0;
     bool ok = true;
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
       Item it;
-      decode_item(p, s_prefix, G, i, it);
+      decode_item(p, s_prefix, G, i, it, gh);
       const int rows_b = tile_rows(it.ntok);  // token rows loaded per stage
       for (int q = 0; q < it.npass && ok; ++q) {
         for (int s = it.s_begin; s < it.s_end; ++s) {
@@ -745,68 +752,82 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t a_ctr = 0, b_ctr = 0, d_ctr = 0;
-      bool ok = true;
-      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-        Item it;
-        decode_item(p, s_prefix, G, i, it);
-        const int n = it.ntok <= 16 ? 16 : 32;
-        const uint32_t idesc = mma_idesc(n);
-        const uint32_t atom_bytes = static_cast<uint32_t>(tile_rows(it.ntok)) * 128u;
-        const uint32_t jd = d_ctr & 1u;
-        if (!mbar_wait(&de[jd], ((d_ctr >> 1) & 1u) ^ 1u, ctl)) break;
-        tc_fence_after();
-        for (int q = 0; q < it.npass && ok; ++q) {
-          const uint32_t dt = tmem_base + jd * kDColsPerBuf + 32 * q;
-          uint32_t accum = 0;
-          for (int s = it.s_begin; s < it.s_end && ok; ++s) {
-            const uint32_t jb = b_ctr % kNB;
-            if (!mbar_wait(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+    // The whole warp walks the items and waits (so every operand address is
+    // warp-uniform); one elected lane issues the MMAs and their commits.
+    const bool leader = elect_one();
+    int gh = 0;
+    uint32_t a_ctr = 0, b_ctr = 0, d_ctr = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+      Item it;
+      decode_item(p, s_prefix, G, i, it, gh);
+      const int n = it.ntok <= 16 ? 16 : 32;
+      const uint32_t idesc = mma_idesc(n);
+      // descriptor step of one 64-column atom of the token tile (16-byte units)
+      const uint32_t atom_step = static_cast<uint32_t>(tile_rows(it.ntok)) * 8u;
+      const uint32_t jd = d_ctr & 1u;
+      if (!mbar_wait_warp(&de[jd], ((d_ctr >> 1) & 1u) ^ 1u, ctl)) break;
+      tc_fence_after();
+      for (int q = 0; q < it.npass && ok; ++q) {
+        const uint32_t dt = tmem_base + jd * kDColsPerBuf + 32 * q;
+        uint32_t accum = 0;
+        for (int s = it.s_begin; s < it.s_end && ok; ++s) {
+          const uint32_t jb = b_ctr % kNB;
+          if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + kOffB + jb * kBStageBytes));
+          for (int sub = 0; sub < 2; ++sub) {
+            const uint32_t qa = a_ctr % kNA;
+            if (!mbar_wait_warp(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t bbase = smem_addr(smem + kOffB + jb * kBStageBytes);
-            for (int sub = 0; sub < 2; ++sub) {
-              const uint32_t qa = a_ctr % kNA;
-              if (!mbar_wait(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t at = tmem_base + kAColBase + qa * kAColsPerSlot;
+            const uint32_t at = tmem_base + kAColBase + qa * kAColsPerSlot;
+            if (leader) {
+              // K step kk of this 128-column half: atom 2 sub + kk / 4, 32 bytes
+              // per 16 columns inside the atom
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
-                const int kp = sub * 128 + kk * 16;
-                const uint32_t baddr = bbase + (kp >> 6) * atom_bytes + (kp & 63) * 2;
-                tc_mma(dt, at + kk * 8, smem_desc_sw128(baddr), idesc, accum);
-                accum = 1;
+                const uint64_t bd =
+                    bdesc + (2u * sub + (kk >> 2)) * atom_step + 2u * (kk & 3);
+                tc_mma(dt, at + kk * 8, bd, idesc, accum | kk);
               }
               tc_commit(&ae[qa]);
-              a_ctr++;
             }
-            if (!ok) break;
-            tc_commit(&bempty[jb]);
-            b_ctr++;
+            __syncwarp();
+            accum = 1;
+            a_ctr++;
           }
+          if (!ok) break;
+          if (leader) tc_commit(&bempty[jb]);
+          __syncwarp();
+          b_ctr++;
         }
-        if (!ok) break;
-        tc_commit(&df[jd]);
-        d_ctr++;
       }
-      // all issued MMAs complete before TMEM is released
+      if (!ok) break;
+      if (leader) tc_commit(&df[jd]);
+      __syncwarp();
+      d_ctr++;
+    }
+    // all issued MMAs complete before TMEM is released
+    if (leader) {
       tc_commit(drain);
       mbar_drain(drain, 0);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------ epilogue
     const int qd = warp & 3;
     const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
     uint32_t d_ctr = 0;
+    int gh = 0;
     for (int i = blockIdx.x; i < total; i += gridDim.x) {
       Item it;
-      decode_item(p, s_prefix, G, i, it);
+      decode_item(p, s_prefix, G, i, it, gh);
       const uint32_t jd = d_ctr & 1u;
       if (!mbar_wait_warp(&df[jd], (d_ctr >> 1) & 1u, ctl)) break;
       tc_fence_after();
@@ -815,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       if (it.npass == 2) tmem_ld32(tmem_lane + jd * kDColsPerBuf + 32, u);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&de[jd]);
+      mbar_arrive_warp(&de[jd]);
       d_ctr++;
       const int o = it.row0 + 32 * qd + lane;
       if (o < it.rows) {

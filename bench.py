@@ -21,6 +21,7 @@ import argparse
 import json
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -77,7 +78,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "bench_clocks_%d.csv" % os.getpid())
+        # raw samples go to PW_BENCH_CLOCKS_DIR (default: the temp directory)
+        self.path = os.path.join(os.environ.get("PW_BENCH_CLOCKS_DIR", tempfile.gettempdir()),
+                                 "bench_clocks_%d.csv" % os.getpid())
 
     def __enter__(self):
         try:

@@ -17,8 +17,8 @@
 //     linear-block, and fuses routing, expert activation and output
 //     accumulation.
 // The pages fix neither the bit layout nor the routing formula nor the
-// activation; the readings taken here are listed in the design doc and repeated
-// at each function below.
+// activation; the reading taken for each is stated at the function that
+// uses it below.
 //
 // Arithmetic: router logits and the top-k decision in fp32 with one fixed
 // summation order (the decision is integer-valued, so both sides take it in

@@ -4,6 +4,7 @@
 // LUT[code] of the column the K order assigns to it.  Exit status 0 = pass.
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <random>
 #include <vector>
@@ -21,29 +22,39 @@ static int code_of(const uint32_t* P, int B, int c) {
 template <int B>
 static int check(std::mt19937& rng) {
   int bad = 0;
-  std::vector<uint8_t> region(1u << 17, 0);  // emulated shared-memory table
+  std::vector<uint8_t> region(1u << 16, 0);  // emulated 64 KB shared-memory table
   for (int trial = 0; trial < 2000; ++trial) {
-    const int r = rng() % 128;
+    const uint32_t r = rng() % 128;
     uint32_t P[B];
     for (int k = 0; k < B; ++k) P[k] = rng();
     if (trial == 0) for (int k = 0; k < B; ++k) P[k] = 0xFFFFFFFFu;
     if (trial == 1) for (int k = 0; k < B; ++k) P[k] = 0u;
     uint16_t lut[256];
     for (int v = 0; v < (1 << B); ++v) lut[v] = static_cast<uint16_t>(rng());
+    std::fill(region.begin(), region.end(), 0xEE);  // unwritten bytes never match
+    auto put16 = [&](uint32_t off, uint16_t v) -> bool {
+      if (off + 1 >= region.size()) return false;
+      region[off] = v & 0xFF;
+      region[off + 1] = v >> 8;
+      return true;
+    };
+    auto get16 = [&](uint32_t x) -> uint32_t {
+      if (x + 1 >= region.size()) { std::printf("read out of range\n"); std::exit(1); }
+      return region[x] | (region[x + 1] << 8);
+    };
     uint32_t out[16];
     if constexpr (B <= 3) {
-      uint32_t w[4] = {0, 0, 0, 0};
-      for (int v = 0; v < (1 << B); ++v) w[v / 2] |= static_cast<uint32_t>(lut[v]) << (16 * (v & 1));
-      RegLut L = make_reg_lut<B>(w);
-      dq_word_reg<B>(P, L, out);
+      for (int v1 = 0; v1 < (1 << B); ++v1)
+        for (int v2 = 0; v2 < (1 << B); ++v2) {
+          const uint32_t off = pair_offset(v1, v2, B, r);
+          if (!put16(off, lut[v1]) || !put16(off + 2, lut[v2])) { std::printf("offset out of range\n"); return 1; }
+        }
+      auto lds32 = [&](uint32_t x) -> uint32_t { return get16(x) | (get16(x + 2) << 16); };
+      dq_word_pair<B>(P, r, lds32, out);
     } else {
-      for (int v = 0; v < (1 << B); ++v) {
-        const uint32_t off = (static_cast<uint32_t>(v) << 9) | (4u * r);
-        region[off] = lut[v] & 0xFF;
-        region[off + 1] = lut[v] >> 8;
-      }
-      auto lds = [&](uint32_t x) -> uint32_t { return region[x] | (region[x + 1] << 8); };
-      dq_word_smem<B>(P, 4u * r, lds, out);
+      for (int v = 0; v < (1 << B); ++v)
+        if (!put16(single_offset(v, r), lut[v])) { std::printf("offset out of range\n"); return 1; }
+      dq_word_single<B>(P, r, get16, out);
     }
     for (int pr = 0; pr < 16; ++pr) {
       const int m = pr >> 2, j = pr & 3;
@@ -58,10 +69,41 @@ static int check(std::mt19937& rng) {
   return bad;
 }
 
+// The tables of all rows of a warp-quarter: distinct rows never share a
+// 2-byte entry, and the 32 rows of a warp address 32 different banks.
+static int check_layout() {
+  int bad = 0;
+  for (int b = 4; b <= 8; ++b)
+    for (uint32_t v = 0; v < (1u << b); ++v)
+      for (uint32_t r = 0; r < 128; ++r)
+        for (uint32_t r2 = r + 1; r2 < 128; ++r2)
+          if (single_offset(v, r) == single_offset(v, r2)) ++bad;
+  for (uint32_t q = 0; q < 4; ++q) {
+    bool bank[32] = {};
+    for (uint32_t l = 0; l < 32; ++l) {
+      const uint32_t r = 32 * q + l;
+      const uint32_t bk = (single_offset(l % 7, r) / 4) % 32;  // any codes
+      if (bank[bk]) ++bad;
+      bank[bk] = true;
+    }
+  }
+  for (uint32_t q = 0; q < 4; ++q) {
+    bool bank[32] = {};
+    for (uint32_t l = 0; l < 32; ++l) {
+      const uint32_t r = 32 * q + l;
+      const uint32_t bk = (pair_offset(l % 5, l % 3, 3, r) / 4) % 32;
+      if (bank[bk]) ++bad;
+      bank[bk] = true;
+    }
+  }
+  if (bad) std::printf("layout: %d problems\n", bad);
+  return bad;
+}
+
 int main() {
   std::mt19937 rng(12345);
   int bad = check<1>(rng) + check<2>(rng) + check<3>(rng) + check<4>(rng) + check<5>(rng) +
-            check<6>(rng) + check<7>(rng) + check<8>(rng);
+            check<6>(rng) + check<7>(rng) + check<8>(rng) + check_layout();
   std::printf(bad ? "FAIL %d\n" : "ok\n", bad);
   return bad ? 1 : 0;
 }
