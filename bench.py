@@ -69,6 +69,14 @@ def algorithmic_bytes(layer, idx):
     return {"gu": gu + T * wl.hidden * 2, "down": down, "total": gu + down + router + act}
 
 
+def kernel_source_hash():
+    """sha256 of the tensor-core kernel's sources (tc.cu, dequant.cuh, pages.h, tc.h)."""
+    import hashlib
+    src = b"".join(open(os.path.join(ROOT, "any_precision_weight_pw_b200", "csrc", f), "rb").read()
+                   for f in ("tc.cu", "dequant.cuh", "pages.h", "tc.h"))
+    return hashlib.sha256(src).hexdigest()
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -210,7 +218,8 @@ def run_ours(args, rank, world, local_rank):
     prof_path = os.path.join(ROOT, "profiles", "traffic_per_forward.json")
     if os.path.exists(prof_path):
         tr = json.load(open(prof_path))
-        if tr.get("workload") == "%s T=%d" % HEADLINE:
+        # counters count only while the kernel source is the one they were taken on
+        if tr.get("workload") == "%s T=%d" % HEADLINE and tr.get("source_sha256") == kernel_source_hash():
             traffic = tr.get("dram_bytes_per_forward")
 
     # end to end: host activations in, host output out, through the C ABI
