@@ -17,6 +17,7 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kRouteThreads = 256;
+constexpr int kStageFloats = 4096;  // logits staged in shared memory (16 KB)
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -43,8 +44,21 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
     const int e = pair - t * E;
     const uint16_t* xr = p.x + static_cast<size_t>(t) * H;
     const float* wr = p.wr + static_cast<size_t>(e) * H;
+    // loads in batches of 32 per lane (independent of the sum, so their
+    // latencies overlap); the fused multiply-adds stay in ascending i
     float s = 0.0f;
-    for (int i = lane; i < H; i += 32) s = __fmaf_rn(bf16_bits_to_f32(xr[i]), wr[i], s);
+    int i0 = lane;
+    for (; i0 + 32 * 31 < H; i0 += 32 * 32) {
+      float xv[32], wv[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        xv[u] = bf16_bits_to_f32(xr[i0 + 32 * u]);
+        wv[u] = wr[i0 + 32 * u];
+      }
+#pragma unroll
+      for (int u = 0; u < 32; ++u) s = __fmaf_rn(xv[u], wv[u], s);
+    }
+    for (int i = i0; i < H; i += 32) s = __fmaf_rn(bf16_bits_to_f32(xr[i]), wr[i], s);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) s = s + __shfl_xor_sync(kFull, s, m);
     if (lane == 0) ws.logits[pair] = p.bias ? s + p.bias[e] : s;
@@ -59,41 +73,59 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   __threadfence();
 
   // ---- phase 2 (one block): top-k + softmax ------------------------------
+  // Small problems stage the logits in shared memory with one coalesced pass
+  // (each thread's top-k then reads shared memory instead of waiting on L2).
+  __shared__ float s_logits[kStageFloats];
+  const bool staged = T * E <= kStageFloats;
+  if (staged)
+    for (int j = threadIdx.x; j < T * E; j += kRouteThreads) s_logits[j] = __ldcg(ws.logits + j);
+  __syncthreads();
+  __shared__ int s_idx[kStageFloats];  // top-k of every token when staged
   for (int t = threadIdx.x; t < T; t += kRouteThreads) {
-    const float* l = ws.logits + static_cast<size_t>(t) * E;
+    const float* l = staged ? s_logits + t * E : ws.logits + static_cast<size_t>(t) * E;
     int sel[PW_MAX_TOPK];
     float lsel[PW_MAX_TOPK];
-    for (int j = 0; j < k; ++j) {
+    uint64_t taken_lo = 0ull, taken_hi = 0ull;  // experts already selected (E <= 128)
+#pragma unroll
+    for (int j = 0; j < PW_MAX_TOPK; ++j) {
+      if (j >= k) break;
       int bi = -1;
       float best = 0.0f;
       for (int e = 0; e < E; ++e) {
-        bool taken = false;
-        for (int q = 0; q < j; ++q) taken |= (sel[q] == e);
-        if (taken) continue;
-        const float v = __ldcg(l + e);
+        if ((((e < 64) ? taken_lo : taken_hi) >> (e & 63)) & 1ull) continue;
+        const float v = staged ? l[e] : __ldcg(l + e);
         if (bi < 0 || v > best) {  // strict: equal logits keep the lower index
           best = v;
           bi = e;
         }
       }
+      if (bi < 64) taken_lo |= 1ull << bi; else taken_hi |= 1ull << (bi & 63);
       sel[j] = bi;
       lsel[j] = best;
     }
     const float mx = lsel[0];
     float z = 0.0f;
-    for (int e = 0; e < E; ++e) z += expf(__ldcg(l + e) - mx);
+    for (int e = 0; e < E; ++e) z += expf((staged ? l[e] : __ldcg(l + e)) - mx);
     float psel[PW_MAX_TOPK];
     float ssum = 0.0f;
-    for (int j = 0; j < k; ++j) {
+#pragma unroll
+    for (int j = 0; j < PW_MAX_TOPK; ++j) {
+      if (j >= k) break;
       psel[j] = expf(lsel[j] - mx) / z;
       ssum += psel[j];
     }
-    for (int j = 0; j < k; ++j) {
+#pragma unroll
+    for (int j = 0; j < PW_MAX_TOPK; ++j) {
+      if (j >= k) break;
       ws.topk_idx[t * k + j] = sel[j];
       ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
+      if (staged) s_idx[t * k + j] = sel[j];
     }
   }
   __syncthreads();
+  auto sel_of = [&](int t, int j) -> int {
+    return staged ? s_idx[t * k + j] : __ldcg(ws.topk_idx + t * k + j);
+  };
 
   // ---- bucketing: counts per expert with warp ballots ---------------------
   __shared__ int s_cnt[kMaxGroups + 1];
@@ -104,7 +136,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       const int t = base + lane;
       bool hit = false;
       if (t < T)
-        for (int j = 0; j < k; ++j) hit |= (__ldcg(ws.topk_idx + t * k + j) == e);
+        for (int j = 0; j < k; ++j) hit |= (sel_of(t, j) == e);
       cnt += __popc(__ballot_sync(kFull, hit));
     }
     if (lane == 0) s_cnt[e] = cnt;
@@ -136,7 +168,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       int slot = -1;
       if (t < T)
         for (int j = 0; j < k; ++j)
-          if (__ldcg(ws.topk_idx + t * k + j) == e) slot = j;
+          if (sel_of(t, j) == e) slot = j;
       const unsigned m = __ballot_sync(kFull, slot >= 0);
       if (slot >= 0) {
         const int pos = run + __popc(m & lt_mask);
