@@ -35,6 +35,7 @@ HEADLINE = ("mixtral_8x7b", 16)
 SWEEP = [("mixtral_8x7b", 1), ("mixtral_8x7b", 64), ("qwen15_moe_a27b", 1),
          ("qwen15_moe_a27b", 8), ("qwen15_moe_a27b", 32)]
 N_BATCHES = 8  # distinct token batches cycled through the timed steps
+FALLBACK_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -139,6 +140,109 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
+def page_move_stress(dev, n_forwards=1000, warmup=20):
+    """Bitwidth-switch stress on the Qwen-shaped layer at 32 decode tokens:
+    before every 10th forward a quarter of the linear-blocks change bitwidth
+    (up or down within 3..8); each change is a page move on a side stream
+    (plane pages of an upgrade and the new LUT, from pinned host copies).
+    Reports steady-state tokens/s and the per-forward latency distribution
+    from CUDA events on the forward stream, next to the same layer without
+    switches.  No L2 flush: steady serving."""
+    import torch
+    from any_precision_weight_pw_b200 import binding, synth
+    wl = synth.WORKLOADS["qwen15_moe_a27b_switch"]
+    T = wl.tokens[0]
+    layer = synth.Layer(wl, seed=0)
+    d = binding.upload_synth_layer(layer, max_tokens=T, host_copies=True)
+    wr = torch.from_numpy(layer.router_w).to(dev)
+    xs = [torch.from_numpy(synth.tokens(wl, T, seed=0, batch=b).view(np.int16)).to(dev)
+          for b in range(N_BATCHES)]
+    ys = [torch.empty_like(x) for x in xs]
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    total = warmup + n_forwards
+    sched = synth.switch_schedule(wl, layer.bits, total, every=10)
+    pb = [binding.plane_bytes(*layer.shape(blk)) for blk in range(wl.n_blocks)]
+
+    def run(with_switches):
+        bits = list(layer.bits) if with_switches else None
+        moved = 0
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(total)]
+        for f in range(total):
+            if with_switches and f in sched:
+                for blk, nb in sched[f]:
+                    d.set_block_bits(blk, nb, side)
+                    rows = layer.shape(blk)[0]
+                    if f >= warmup:
+                        moved += max(nb - bits[blk], 0) * pb[blk] + rows * (1 << nb) * 2
+                    bits[blk] = nb
+            evs[f][0].record(stream)
+            d.forward(xs[f % N_BATCHES], wr, None, ys[f % N_BATCHES])
+            evs[f][1].record(stream)
+        torch.cuda.synchronize()
+        d.check_device_error()
+        lat = np.array([a.elapsed_time(b) for a, b in evs[warmup:]])
+        span = evs[warmup][0].elapsed_time(evs[-1][1])
+        return lat, span, moved
+
+    base_lat, base_span, _ = run(False)
+    lat, span, moved = run(True)
+    n_switch = sum(1 for f in sched if f >= warmup)
+    out = {"workload": "qwen15_moe_a27b decode T=%d, 25%% of blocks switch every 10 forwards" % T,
+           "forwards": n_forwards, "tokens_per_s": round(n_forwards * T / (span / 1e3), 1),
+           "ms_per_forward_mean": round(float(lat.mean()), 4),
+           "ms_per_forward_p50": round(float(np.percentile(lat, 50)), 4),
+           "ms_per_forward_p99": round(float(np.percentile(lat, 99)), 4),
+           "ms_per_forward_max": round(float(lat.max()), 4),
+           "page_bytes_per_switch": int(moved / max(n_switch, 1)),
+           "blocks_per_switch": len(next(iter(sched.values()))),
+           "no_switch": {"tokens_per_s": round(n_forwards * T / (base_span / 1e3), 1),
+                         "ms_per_forward_p99": round(float(np.percentile(base_lat, 99)), 4)}}
+    d.close()
+    return out
+
+
+def prefill_measure(dev, steps=5, warmup=2):
+    """The Mixtral-shaped layer at prefill scale (4096 tokens, Zipf-skewed
+    routing): forward time with CUDA events, tokens/s and achieved TFLOP/s of
+    the expert contractions (2 x 3 x H x F per routed slot) against the
+    measured dense bf16 peak (fp16 runs at the same tensor rate)."""
+    import torch
+    from any_precision_weight_pw_b200 import binding, synth
+    wl = synth.WORKLOADS["mixtral_8x7b_prefill"]
+    T = wl.tokens[0]
+    layer = synth.Layer(wl, seed=0)
+    d = binding.upload_synth_layer(layer, max_tokens=T)
+    wr = torch.from_numpy(layer.router_w).to(dev)
+    bias = torch.from_numpy(layer.router_bias).to(dev)
+    x = torch.from_numpy(synth.tokens(wl, T, seed=0).view(np.int16)).to(dev)
+    y = torch.empty_like(x)
+    for _ in range(warmup):
+        d.forward(x, wr, bias, y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        d.forward(x, wr, bias, y)
+    e1.record()
+    torch.cuda.synchronize()
+    d.check_device_error()
+    ms = e0.elapsed_time(e1) / steps
+    idx, _ = d.routing(T)
+    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=wl.n_experts)
+    flops = 2.0 * 3 * wl.hidden * wl.ffn * T * wl.top_k
+    pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    peak = float(pk.get("bf16_tflops", FALLBACK_TFLOPS))
+    d.close()
+    return {"workload": "mixtral_8x7b prefill T=%d (Zipf 1.2 usage, experts 0-1 at 8 bits, rest 4)" % T,
+            "ms_per_forward": round(ms, 3), "tokens_per_s": round(T / (ms / 1e3), 1),
+            "tflops": round(flops / (ms / 1e3) / 1e12, 2), "peak_tflops": peak,
+            "frac_of_peak": round(flops / (ms / 1e3) / 1e12 / peak, 4),
+            "tokens_per_expert": counts.tolist()}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from any_precision_weight_pw_b200 import binding, build, synth
@@ -243,6 +347,8 @@ def run_ours(args, rank, world, local_rank):
     # decode sweep (other batch sizes and the Qwen-shaped layer); L2 flushed
     # between timed forwards so small layers are not served from cache
     sweep = []
+    page_move = None
+    prefill = None
     if rank == 0 and not args.no_sweep:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         cur = (name, layer, d, wr, bias)
@@ -273,6 +379,8 @@ def run_ours(args, rank, world, local_rank):
             del xs2, ys2
         cur[2].close()
         del flush
+        page_move = page_move_stress(dev)
+        prefill = prefill_measure(dev)
     else:
         d.close()
 
@@ -316,6 +424,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(t_begin, t_end),
         "gpu_launches": launches,
         "sweep": sweep,
+        "page_move": page_move,
+        "prefill": prefill,
     }
     return out
 

@@ -296,3 +296,27 @@ def test_forward_host_matches_device(pw):
     yh = dev.forward_host(xh, wr)
     assert torch.equal(yd, yh)
     dev.close()
+
+
+def test_prefill_scale_layer_sampled(pw, oracle):
+    """Mixtral-shaped layer at prefill scale (4096 tokens, Zipf-skewed expert
+    usage, experts 0 and 1 at 8 bits, the rest at 4): every token's routing
+    is compared with the oracle's, and the outputs of a sample of tokens
+    (the oracle computes each token on its own)."""
+    wl = synth.WORKLOADS["mixtral_8x7b_prefill"]
+    layer = synth.Layer(wl, seed=0)
+    T = 4096
+    y, idx, w, x = _run_layer(pw, layer, T)
+    logits = oracle.router_logits(x, layer.router_w, layer.router_bias)
+    ridx, rw = oracle.topk_softmax(logits, wl.top_k, bool(wl.renorm_topk))
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=1e-5, atol=1e-7)
+    counts = np.bincount(idx.reshape(-1), minlength=wl.n_experts)
+    assert counts[0] == counts.max() and counts[0] > 2 * np.sort(counts)[-3]  # skewed usage
+    rng = np.random.default_rng(7)
+    heavy = np.flatnonzero(idx[:, 0] == 0)[:4]          # tokens on the 8-bit expert 0
+    sample = np.unique(np.concatenate([heavy, rng.choice(T, 12, replace=False), [0, T - 1]]))
+    L = oracle_layer(oracle, layer)
+    ref, sidx, _ = L.forward(x[sample], layer.router_w, layer.router_bias, threads=32)
+    np.testing.assert_array_equal(sidx, idx[sample])
+    assert_output_close(y[sample], ref)
