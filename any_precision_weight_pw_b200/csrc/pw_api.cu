@@ -100,6 +100,22 @@ pw_status_t make_row_maps(CUtensorMap* m, const uint16_t* base, int ld, int rows
   return PW_OK;
 }
 
+// Map for the prefill passes: box {64 columns, 256 rows, 1 atom}.
+pw_status_t make_chunk_map(CUtensorMap* m, const uint16_t* base, int ld, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(ld / 64)};
+  cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(rows) * 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(pw::kTcPfTokens), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled (token chunks) failed (%d)", (int)r);
+  return PW_OK;
+}
+
 int env_int(const char* name, int dflt) {
   const char* v = getenv(name);
   return v ? atoi(v) : dflt;
@@ -132,6 +148,10 @@ struct pw_moe {
   uint16_t* h_perm = nullptr;   // tensor-core path: fp16 silu(g) * u, K-permuted
   int x_ld = 0, h_perm_ld = 0;
   CUtensorMap x_maps[4], h_maps[4];  // token-tile maps over x_sorted and h_perm
+  CUtensorMap x_pf_map, h_pf_map;    // 256-row chunk maps (prefill passes)
+  float* gbuf = nullptr;             // prefill: gate outputs [P_max][Fmax] fp32
+  int gbuf_ld = 0;
+  bool pf = false;                   // the prefill passes are available
   float* ysorted = nullptr;
   int* err = nullptr;
   uint16_t* stage_x = nullptr;
@@ -184,6 +204,15 @@ int down_splits(const pw_moe* h, int T) {
   if (ns > h->max_split) ns = h->max_split;
   if (ns < 1) ns = 1;
   return ns;
+}
+
+// Prefill passes (256-token chunks) when the routed slots average at least
+// 64 tokens per expert; PW_PREFILL=0/1 forces the choice.
+bool use_prefill(const pw_moe* h, int T) {
+  if (!h->pf) return false;
+  const int forced = env_int("PW_PREFILL", -1);
+  if (forced >= 0) return forced != 0;
+  return static_cast<long long>(T) * h->cfg.top_k >= 64ll * h->cfg.n_experts;
 }
 
 }  // namespace
@@ -282,6 +311,9 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->x_ld);
   const size_t o_hp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->h_perm_ld);
   const size_t o_ys = off; off += al(sizeof(float) * size_t(h->max_split) * h->P_max * c.hidden);
+  h->pf = h->tc && h->P_max >= pw::kTcPfTokens;
+  h->gbuf_ld = h->pf ? Fmax : 0;
+  const size_t o_gb = off; off += al(sizeof(float) * size_t(h->P_max) * h->gbuf_ld);
   const size_t o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
   const size_t o_sy = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
   if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
@@ -302,6 +334,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->x_sorted = reinterpret_cast<uint16_t*>(w + o_xp);
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
   h->ysorted = reinterpret_cast<float*>(w + o_ys);
+  h->gbuf = reinterpret_cast<float*>(w + o_gb);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
   h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
   if (cudaMemset(w + o_tk, 0, al(sizeof(uint32_t) * 4) + al(sizeof(int) * 4)) != cudaSuccess ||
@@ -313,6 +346,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   if (h->tc) {
     pw_status_t st = make_row_maps(h->x_maps, h->x_sorted, h->x_ld, h->P_max);
     if (st == PW_OK) st = make_row_maps(h->h_maps, h->h_perm, h->h_perm_ld, h->P_max);
+    if (st == PW_OK && h->pf) st = make_chunk_map(&h->x_pf_map, h->x_sorted, h->x_ld, h->P_max);
+    if (st == PW_OK && h->pf) st = make_chunk_map(&h->h_pf_map, h->h_perm, h->h_perm_ld, h->P_max);
     if (st != PW_OK) {
       free_all(h);
       return st;
@@ -395,6 +430,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     pt.bits[i] = static_cast<uint8_t>(h->blk[i].bits);
   }
   const int has_shared = c.shared_ffn > 0 ? 1 : 0;
+  const bool prefill = h->tc && use_prefill(h, T);
   std::vector<cudaEvent_t> evs;
   if (h->profiling) {
     for (int i = 0; i < 5; ++i) {
@@ -442,7 +478,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
-    tp.mode = pw::kTcGateUp;
+    tp.mode = prefill ? pw::kTcPfGate : pw::kTcGateUp;
     tp.H = c.hidden;
     tp.F = c.ffn;
     tp.S = c.shared_ffn;
@@ -458,6 +494,14 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_perm_ld = h->h_perm_ld;
     tp.h_rows = h->P_max;
     tp.err = h->err;
+    if (prefill) {
+      // gate -> g (fp32), then up -> h = silu(g) * u
+      tp.pf_map = h->x_pf_map;
+      tp.gbuf = h->gbuf;
+      tp.gbuf_ld = h->gbuf_ld;
+      PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
+      tp.mode = pw::kTcPfUp;
+    }
     PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
   } else {
     pw::SimpleParams sp;
@@ -483,11 +527,12 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   // down pass
   int n_split = 1;
   if (h->tc) {
-    n_split = down_splits(h, T);
+    n_split = prefill ? 1 : down_splits(h, T);
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
-    tp.mode = pw::kTcDown;
+    tp.mode = prefill ? pw::kTcPfDown : pw::kTcDown;
+    tp.pf_map = h->h_pf_map;
     tp.H = c.hidden;
     tp.F = c.ffn;
     tp.S = c.shared_ffn;
@@ -686,7 +731,9 @@ pw_status_t pw_profile_read(pw_moe_t* h, float* ms, int32_t n, int32_t* n_forwar
 
 int32_t pw_forward_launches(const pw_moe_t* h, int32_t T) {
   if (!h) return 0;
-  return T > 0 ? (h->tc ? 5 : 4) : 0;
+  if (T <= 0) return 0;
+  if (!h->tc) return 4;
+  return use_prefill(h, T) ? 6 : 5;
 }
 
 pw_status_t pw_destroy(pw_moe_t* h) {

@@ -58,39 +58,57 @@ namespace {
 constexpr int kTileRows = 128;
 constexpr int kStageWords = 8;                 // 256 columns per stage
 constexpr int kSlotBytes = kTileRows * kStageWords * 4;  // 4 KB: one plane of a stage
-constexpr int kNSlot = 20;                     // plane slots (80 KB)
 constexpr int kNS = 8;                         // plane stages in flight (barrier pairs)
-constexpr int kNT = kTcTokens;                 // token tile (MMA N <= 32)
-constexpr int kBStageBytes = kNT * 256 * 2;    // 32 rows x 256 K fp16 = 16 KB
-constexpr int kNB = 4;                         // token-tile ring depth
-constexpr int kNA = 6;                         // TMEM A ring slots (128 K each)
-constexpr int kAColsPerSlot = 64;
-constexpr int kAColBase = 128;
-constexpr int kDColsPerBuf = 64;               // gate at +0, up at +32
+constexpr int kAColsPerSlot = 64;              // TMEM columns of one 128-K A slot
 constexpr int kTmemCols = 512;
 constexpr int kDqThreads = 256;                // 8 dequantiser warps
 constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpLoader = 10;
 constexpr int kThreads = 15 * 32;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
-
-// Shared memory (offsets from a 1024-byte aligned base; compile-time so the
-// table lookups fold the base into the load's immediate offset).
 constexpr uint32_t kOffLut = 0;                // 256 code lines x 64 row words x 4 B
 constexpr uint32_t kLutBytes = 256u * 64u * 4u;
-constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
-constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
-constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
-constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 4 + 2;
-constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 4 * (kMaxGroups + 2);
-constexpr uint32_t kSmemTotal = kOffSlotUser + 4 * kNSlot;
-static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
+
+// Two configurations of the kernel.
+//   decode  token tiles of up to 32 rows (MMA N = 16 or 32); one TMA box per
+//           256-column B stage; two accumulator buffers (gate and up side by
+//           side) so an item's epilogue overlaps the next item's MMAs.
+//   prefill 256-token chunks (MMA N = 256), so each dequantised weight tile
+//           serves 256 tokens; B stages of 64 columns (32 KB); one 256-column
+//           accumulator, so gate and up run as separate launches.
+// Shared memory offsets are compile-time (from a 1024-byte aligned base) so
+// table lookups fold the base into the loads' immediate offsets.
+template <bool PF>
+struct Cfg {
+  static constexpr bool kPrefill = PF;
+  static constexpr int kNSlot = PF ? 16 : 20;  // plane slots
+  static constexpr int kNT = PF ? kTcPfTokens : kTcTokens;
+  static constexpr int kBStageK = PF ? 64 : 256;
+  static constexpr int kBStageBytes = kNT * kBStageK * 2;
+  static constexpr int kBPerStage = 256 / kBStageK;
+  static constexpr int kNB = PF ? 3 : 4;        // token-tile ring depth
+  static constexpr int kNA = PF ? 4 : 6;        // TMEM A ring slots (128 K each)
+  static constexpr int kNDBuf = PF ? 1 : 2;     // accumulator buffers
+  static constexpr int kDColsPerBuf = PF ? 256 : 64;
+  static constexpr int kAColBase = kNDBuf * kDColsPerBuf;
+  static constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
+  static constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
+  static constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
+  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 2 * kNDBuf + 2;
+  static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
+  static constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 4 * (kMaxGroups + 2);
+  static constexpr uint32_t kSmemTotal = kOffSlotUser + 4 * kNSlot;
+  static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
+  static_assert(kAColBase + kNA * kAColsPerSlot <= kTmemCols, "tensor memory budget");
+};
+using Dec = Cfg<false>;
+using Pre = Cfg<true>;
 
 // Plane stages take `bits` consecutive slots of the ring; a stage that would
 // run past the end starts again at slot 0.  Producer and dequantisers walk
 // the same sequence of stages, so both derive the same placement.
+template <class C>
 __device__ __forceinline__ uint32_t place_stage(uint32_t& ring_end, int bits) {
-  const uint32_t start = (ring_end + bits <= static_cast<uint32_t>(kNSlot)) ? ring_end : 0u;
+  const uint32_t start = (ring_end + bits <= static_cast<uint32_t>(C::kNSlot)) ? ring_end : 0u;
   ring_end = start + bits;
   return start;
 }
@@ -292,6 +310,11 @@ struct Item {
 
 // Items are visited in increasing order by every role, so the group search
 // resumes from the previous item's group (gh).
+__device__ __forceinline__ bool gate_or_up(int mode) {
+  return mode == kTcGateUp || mode == kTcPfGate || mode == kTcPfUp;
+}
+
+template <class C>
 __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix, int G,
                                             int i, Item& it, int& gh) {
   int g = gh;
@@ -306,24 +329,40 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
     pos0 = 0;
   } else {
     const int Fg = (g == p.E) ? p.S : p.F;
-    it.rows = (p.mode == kTcGateUp) ? Fg : p.H;
-    it.cols = (p.mode == kTcGateUp) ? p.H : Fg;
+    it.rows = gate_or_up(p.mode) ? Fg : p.H;
+    it.cols = gate_or_up(p.mode) ? p.H : Fg;
     pos0 = p.offsets[g];
     n = p.offsets[g + 1] - pos0;
   }
   const int rt = (it.rows + kTileRows - 1) / kTileRows;
+  const int stages = (((it.cols + 31) >> 5) + kStageWords - 1) / kStageWords;
+  it.g = g;
+  if constexpr (C::kPrefill) {
+    // token chunks vary fastest, so the CTAs working at the same time share
+    // a row tile's plane pages in L2
+    const int chunks = (n + C::kNT - 1) / C::kNT;
+    const int row_tile = local / chunks;
+    const int chunk = local - row_tile * chunks;
+    it.split = 0;
+    it.row0 = row_tile * kTileRows;
+    it.tok0 = chunk * C::kNT;
+    it.ntok = min(C::kNT, n - it.tok0);
+    it.pos0 = pos0 + it.tok0;
+    it.s_begin = 0;
+    it.s_end = stages;
+    it.npass = 1;
+    return;
+  }
   const int ns = p.n_split;
   const int per_tt = rt * ns;
   const int tt = local / per_tt;
   const int r = local - tt * per_tt;
   const int row_tile = r / ns;
   it.split = r - row_tile * ns;
-  it.g = g;
   it.row0 = row_tile * kTileRows;
-  it.tok0 = tt * kNT;
-  it.ntok = min(kNT, n - it.tok0);
+  it.tok0 = tt * C::kNT;
+  it.ntok = min(C::kNT, n - it.tok0);
   it.pos0 = pos0 + it.tok0;
-  const int stages = (((it.cols + 31) >> 5) + kStageWords - 1) / kStageWords;
   it.s_begin = static_cast<int>((static_cast<long long>(stages) * it.split) / ns);
   it.s_end = static_cast<int>((static_cast<long long>(stages) * (it.split + 1)) / ns);
   it.npass = (p.mode == kTcGateUp) ? 2 : 1;
@@ -332,7 +371,10 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
 // Block, bitwidth, LUT and plane tensor map of pass q of an item.
 __device__ __forceinline__ Pass get_pass(const TcParams& p, const Item& it, int q) {
   if (p.mode == kTcLinear) return Pass{-1, p.lin_bits, p.lin_lut, p.lin_planes};
-  const int blk = 3 * it.g + ((p.mode == kTcGateUp) ? q : 2);
+  const int proj = (p.mode == kTcGateUp) ? q
+                   : (p.mode == kTcPfGate) ? 0
+                   : (p.mode == kTcPfUp) ? 1 : 2;
+  const int blk = 3 * it.g + proj;
   return Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.pt.blk[blk].planes};
 }
 
@@ -361,7 +403,7 @@ struct DequantState {
   uint32_t a_ctr;      // stages processed by this K half
 };
 
-template <int B>
+template <class C, int B>
 __device__ bool dequant_stages(const Item& it, int grp, int quad,
                                uint64_t* sf, uint64_t* se, uint64_t* af, uint64_t* ae,
                                uint32_t tmem_base, DequantState& st, const Ctl& ctl) {
@@ -378,11 +420,11 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad,
   for (int s = it.s_begin; s < it.s_end; ++s) {
     uint32_t P[4][B];
     const uint32_t e = st.stage_ctr % kNS;
-    const uint32_t slot0 = place_stage(st.ring_end, B);
+    const uint32_t slot0 = place_stage<C>(st.ring_end, B);
     if (!mbar_wait_warp(&sf[e], (st.stage_ctr / kNS) & 1u, ctl)) return false;
 #pragma unroll
     for (int k = 0; k < B; ++k) {
-      const uint4 q4 = read_plane_chunk(kOffSlots + (slot0 + k) * kSlotBytes, r, grp);
+      const uint4 q4 = read_plane_chunk(C::kOffSlots + (slot0 + k) * kSlotBytes, r, grp);
       P[0][k] = q4.x;
       P[1][k] = q4.y;
       P[2][k] = q4.z;
@@ -391,9 +433,9 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad,
     mbar_arrive_warp(&se[e]);
     st.stage_ctr++;
     const uint32_t a_idx = 2u * st.a_ctr + static_cast<uint32_t>(grp);
-    const uint32_t qa = a_idx % kNA;
-    if (!mbar_wait_warp(&ae[qa], ((a_idx / kNA) & 1u) ^ 1u, ctl)) return false;
-    const uint32_t tcol = tmem_lane + kAColBase + qa * kAColsPerSlot;
+    const uint32_t qa = a_idx % C::kNA;
+    if (!mbar_wait_warp(&ae[qa], ((a_idx / C::kNA) & 1u) ^ 1u, ctl)) return false;
+    const uint32_t tcol = tmem_lane + C::kAColBase + qa * kAColsPerSlot;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t out[32];
@@ -541,9 +583,11 @@ __device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t
 }
 
 // ---------------------------------------------------------------- kernel
+template <class C>
 __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr int kNB = C::kNB, kNA = C::kNA, kNDBuf = C::kNDBuf;
   uint8_t* smem = pw_tc_smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* sf = bars;      // plane stage full (bulk copy landed)
   uint64_t* se = sf + kNS;  // plane stage empty (all dequantisers read it)
   uint64_t* bfull = se + kNS;
@@ -551,13 +595,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   uint64_t* af = bempty + kNB;
   uint64_t* ae = af + kNA;
   uint64_t* df = ae + kNA;
-  uint64_t* de = df + 2;
-  uint64_t* drain = de + 2;
+  uint64_t* de = df + kNDBuf;
+  uint64_t* drain = de + kNDBuf;
   uint64_t* dqbar = drain + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  int* s_prefix = reinterpret_cast<int*>(smem + kOffMisc + 16);
-  uint32_t* slot_user = reinterpret_cast<uint32_t*>(smem + kOffSlotUser);  // producer only
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  int* s_prefix = reinterpret_cast<int*>(smem + C::kOffMisc + 16);
+  uint32_t* slot_user = reinterpret_cast<uint32_t*>(smem + C::kOffSlotUser);  // producer only
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -572,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       mbar_init(&bfull[i], p.mode == kTcLinear ? 32 : 1);
       mbar_init(&bempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNDBuf; ++i) {
       mbar_init(&df[i], 1);
       mbar_init(&de[i], 4);
     }
@@ -582,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     }
     mbar_init(drain, 1);
     mbar_init(dqbar, kDqThreads / 32);
-    for (int k = 0; k < kNSlot; ++k) slot_user[k] = 0u;
+    for (int k = 0; k < C::kNSlot; ++k) slot_user[k] = 0u;
     // the table offsets assume a 1024-byte aligned dynamic shared memory base
     *s_abort = (smem_addr(smem) & 1023u) ? 1 : 0;
     if (*s_abort && p.err) atomicExch(p.err, PW_ERR_UNSUPPORTED);
@@ -596,10 +640,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         n = p.T;
       } else {
         const int Fg = (g == p.E) ? p.S : p.F;
-        rows = (p.mode == kTcGateUp) ? Fg : p.H;
+        rows = gate_or_up(p.mode) ? Fg : p.H;
         n = p.offsets[g + 1] - p.offsets[g];
       }
-      const int tt = (n + kNT - 1) / kNT;
+      const int tt = (n + C::kNT - 1) / C::kNT;
       acc += ((rows + kTileRows - 1) / kTileRows) * tt * p.n_split;
     }
     s_prefix[G] = acc;
@@ -632,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     Item it;
     LutPrefetch pre;
     if (i < total) {
-      decode_item(p, s_prefix, G, i, it, gh);
+      decode_item<C>(p, s_prefix, G, i, it, gh);
       lut_prefetch(it, get_pass(p, it, 0), grp, r, pre);
     }
     while (i < total && ok) {
@@ -646,18 +690,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       if (nq >= it.npass) {
         ni = i + gridDim.x;
         nq = 0;
-        if (ni < total) decode_item(p, s_prefix, G, ni, it, gh);
+        if (ni < total) decode_item<C>(p, s_prefix, G, ni, it, gh);
       }
       if (ni < total) lut_prefetch(it, get_pass(p, it, nq), grp, r, pre);
       switch (ps.bits) {
-        case 1: ok = dequant_stages<1>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 2: ok = dequant_stages<2>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 3: ok = dequant_stages<3>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 4: ok = dequant_stages<4>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 5: ok = dequant_stages<5>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 6: ok = dequant_stages<6>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        case 7: ok = dequant_stages<7>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
-        default: ok = dequant_stages<8>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 1: ok = dequant_stages<C, 1>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 2: ok = dequant_stages<C, 2>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 3: ok = dequant_stages<C, 3>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 4: ok = dequant_stages<C, 4>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 5: ok = dequant_stages<C, 5>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 6: ok = dequant_stages<C, 6>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        case 7: ok = dequant_stages<C, 7>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
+        default: ok = dequant_stages<C, 8>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
       }
       i = ni;
       q = nq;
@@ -671,14 +715,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       const int n_max = (p.mode == kTcLinear) ? p.lin_n_max : p.n_max;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
-        decode_item(p, s_prefix, G, i, it, gh);
+        decode_item<C>(p, s_prefix, G, i, it, gh);
         const int n_kt = pages::k_tiles(it.cols);
         const int rt = it.row0 / kTileRows;
         for (int q = 0; q < it.npass && ok; ++q) {
           const Pass ps = get_pass(p, it, q);
           for (int s = it.s_begin; s < it.s_end; ++s, ++t) {
             const uint32_t e = t % kNS;
-            const uint32_t start = place_stage(ring_end, ps.bits);
+            const uint32_t start = place_stage<C>(ring_end, ps.bits);
             // the barrier pair of stage t - kNS is free ...
             if (!mbar_wait(&se[e], ((t / kNS) & 1u) ^ 1u, ctl)) {
               ok = false;
@@ -704,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             const int64_t grp_idx = static_cast<int64_t>(rt) * n_kt + s;
             const uint32_t bytes = static_cast<uint32_t>(ps.bits) * kSlotBytes;
             mbar_arrive_tx(&sf[e], bytes);
-            bulk_load(smem_addr(smem + kOffSlots + start * kSlotBytes),
+            bulk_load(smem_addr(smem + C::kOffSlots + start * kSlotBytes),
                       ps.planes + grp_idx * n_max * (kSlotBytes / 4), bytes, &sf[e]);
           }
         }
@@ -722,26 +766,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     bool ok = true;
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
       Item it;
-      decode_item(p, s_prefix, G, i, it, gh);
-      const int rows_b = tile_rows(it.ntok);  // token rows loaded per stage
+      decode_item<C>(p, s_prefix, G, i, it, gh);
+      const int rows_b = tile_rows(it.ntok);  // token rows loaded per stage (decode)
       for (int q = 0; q < it.npass && ok; ++q) {
-        for (int s = it.s_begin; s < it.s_end; ++s) {
-          const uint32_t jb = b_ctr % kNB;
-          if (!mbar_wait_warp(&bempty[jb], ((b_ctr / kNB) & 1u) ^ 1u, ctl)) {
-            ok = false;
-            break;
+        for (int s = it.s_begin; s < it.s_end && ok; ++s) {
+          for (int j = 0; j < C::kBPerStage; ++j) {
+            const uint32_t jb = b_ctr % kNB;
+            if (!mbar_wait_warp(&bempty[jb], ((b_ctr / kNB) & 1u) ^ 1u, ctl)) {
+              ok = false;
+              break;
+            }
+            const uint32_t buf = smem_addr(smem + C::kOffB + jb * C::kBStageBytes);
+            if constexpr (C::kPrefill) {
+              if (lane == 0) {
+                // {64 columns, 256 rows, 1 atom}: atom 4 s + j of the chunk's rows
+                mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(C::kNT) * 128u);
+                tma_load_3d(buf, &p.pf_map, 0, it.pos0, 4 * s + j, &bfull[jb]);
+              }
+            } else if (p.mode == kTcLinear) {
+              fill_b_linear(p, it, s, buf, lane);
+              fence_proxy_async();
+              mbar_arrive(&bfull[jb]);
+            } else if (lane == 0) {
+              // {64 columns, rows_b rows, 4 atoms} starting at column 256 s
+              mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(rows_b) * 4u * 128u);
+              tma_load_3d(buf, &p.b_maps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s, &bfull[jb]);
+            }
+            b_ctr++;
           }
-          const uint32_t buf = smem_addr(smem + kOffB + jb * kBStageBytes);
-          if (p.mode == kTcLinear) {
-            fill_b_linear(p, it, s, buf, lane);
-            fence_proxy_async();
-            mbar_arrive(&bfull[jb]);
-          } else if (lane == 0) {
-            // {64 columns, rows_b rows, 4 atoms} starting at column 256 s
-            mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(rows_b) * 4u * 128u);
-            tma_load_3d(buf, &p.b_maps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s, &bfull[jb]);
-          }
-          b_ctr++;
         }
       }
     }
@@ -758,60 +810,113 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     int gh = 0;
     uint32_t a_ctr = 0, b_ctr = 0, d_ctr = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
-      Item it;
-      decode_item(p, s_prefix, G, i, it, gh);
-      const int n = it.ntok <= 16 ? 16 : 32;
-      const uint32_t idesc = mma_idesc(n);
-      // descriptor step of one 64-column atom of the token tile (16-byte units)
-      const uint32_t atom_step = static_cast<uint32_t>(tile_rows(it.ntok)) * 8u;
-      const uint32_t jd = d_ctr & 1u;
-      if (!mbar_wait_warp(&de[jd], ((d_ctr >> 1) & 1u) ^ 1u, ctl)) break;
-      tc_fence_after();
-      for (int q = 0; q < it.npass && ok; ++q) {
-        const uint32_t dt = tmem_base + jd * kDColsPerBuf + 32 * q;
+    if constexpr (C::kPrefill) {
+      const uint32_t idesc = mma_idesc(C::kNT);
+      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        Item it;
+        decode_item<C>(p, s_prefix, G, i, it, gh);
+        const uint32_t jd = d_ctr % kNDBuf;
+        if (!mbar_wait_warp(&de[jd], ((d_ctr / kNDBuf) & 1u) ^ 1u, ctl)) break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + jd * C::kDColsPerBuf;
         uint32_t accum = 0;
         for (int s = it.s_begin; s < it.s_end && ok; ++s) {
-          const uint32_t jb = b_ctr % kNB;
-          if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + kOffB + jb * kBStageBytes));
-          for (int sub = 0; sub < 2; ++sub) {
+          for (int sub = 0; sub < 2 && ok; ++sub) {
             const uint32_t qa = a_ctr % kNA;
             if (!mbar_wait_warp(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t at = tmem_base + kAColBase + qa * kAColsPerSlot;
-            if (leader) {
-              // K step kk of this 128-column half: atom 2 sub + kk / 4, 32 bytes
-              // per 16 columns inside the atom
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t bd =
-                    bdesc + (2u * sub + (kk >> 2)) * atom_step + 2u * (kk & 3);
-                tc_mma(dt, at + kk * 8, bd, idesc, accum | kk);
+            const uint32_t at = tmem_base + C::kAColBase + qa * kAColsPerSlot;
+            // two 64-column B stages per 128-column A slot
+            for (int j = 0; j < 2; ++j) {
+              const uint32_t jb = b_ctr % kNB;
+              if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+                ok = false;
+                break;
               }
-              tc_commit(&ae[qa]);
+              tc_fence_after();
+              const uint64_t bdesc =
+                  smem_desc_sw128(smem_addr(smem + C::kOffB + jb * C::kBStageBytes));
+              if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  tc_mma(dt, at + (4 * j + kk) * 8, bdesc + 2u * kk, idesc,
+                         accum | static_cast<uint32_t>(j | kk));
+                tc_commit(&bempty[jb]);
+              }
+              __syncwarp();
+              accum = 1;
+              b_ctr++;
             }
+            if (!ok) break;
+            if (leader) tc_commit(&ae[qa]);
             __syncwarp();
-            accum = 1;
             a_ctr++;
           }
-          if (!ok) break;
-          if (leader) tc_commit(&bempty[jb]);
-          __syncwarp();
-          b_ctr++;
         }
+        if (!ok) break;
+        if (leader) tc_commit(&df[jd]);
+        __syncwarp();
+        d_ctr++;
       }
-      if (!ok) break;
-      if (leader) tc_commit(&df[jd]);
-      __syncwarp();
-      d_ctr++;
+    } else {
+      for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
+        Item it;
+        decode_item<C>(p, s_prefix, G, i, it, gh);
+        const int n = it.ntok <= 16 ? 16 : 32;
+        const uint32_t idesc = mma_idesc(n);
+        // descriptor step of one 64-column atom of the token tile (16-byte units)
+        const uint32_t atom_step = static_cast<uint32_t>(tile_rows(it.ntok)) * 8u;
+        const uint32_t jd = d_ctr & 1u;
+        if (!mbar_wait_warp(&de[jd], ((d_ctr >> 1) & 1u) ^ 1u, ctl)) break;
+        tc_fence_after();
+        for (int q = 0; q < it.npass && ok; ++q) {
+          const uint32_t dt = tmem_base + jd * C::kDColsPerBuf + 32 * q;
+          uint32_t accum = 0;
+          for (int s = it.s_begin; s < it.s_end && ok; ++s) {
+            const uint32_t jb = b_ctr % kNB;
+            if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + C::kOffB + jb * C::kBStageBytes));
+            for (int sub = 0; sub < 2; ++sub) {
+              const uint32_t qa = a_ctr % kNA;
+              if (!mbar_wait_warp(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t at = tmem_base + C::kAColBase + qa * kAColsPerSlot;
+              if (leader) {
+                // K step kk of this 128-column half: atom 2 sub + kk / 4, 32 bytes
+                // per 16 columns inside the atom
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint64_t bd =
+                      bdesc + (2u * sub + (kk >> 2)) * atom_step + 2u * (kk & 3);
+                  tc_mma(dt, at + kk * 8, bd, idesc, accum | kk);
+                }
+                tc_commit(&ae[qa]);
+              }
+              __syncwarp();
+              accum = 1;
+              a_ctr++;
+            }
+            if (!ok) break;
+            if (leader) tc_commit(&bempty[jb]);
+            __syncwarp();
+            b_ctr++;
+          }
+        }
+        if (!ok) break;
+        if (leader) tc_commit(&df[jd]);
+        __syncwarp();
+        d_ctr++;
+      }
     }
     // all issued MMAs complete before TMEM is released
     if (leader) {
@@ -821,53 +926,107 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     __syncwarp();
   } else {
     // ------------------------------------------------ epilogue
-    const int qd = warp & 3;
-    const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
-    uint32_t d_ctr = 0;
-    int gh = 0;
-    for (int i = blockIdx.x; i < total; i += gridDim.x) {
-      Item it;
-      decode_item(p, s_prefix, G, i, it, gh);
-      const uint32_t jd = d_ctr & 1u;
-      if (!mbar_wait_warp(&df[jd], (d_ctr >> 1) & 1u, ctl)) break;
-      tc_fence_after();
-      uint32_t v[32], u[32];
-      tmem_ld32(tmem_lane + jd * kDColsPerBuf, v);
-      if (it.npass == 2) tmem_ld32(tmem_lane + jd * kDColsPerBuf + 32, u);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive_warp(&de[jd]);
-      d_ctr++;
-      const int o = it.row0 + 32 * qd + lane;
-      if (o < it.rows) {
-        if (p.mode == kTcGateUp) {
-          // h = silu(g) * u, fp16, at o's position in the down pass's K order
-          // atom-major [ld/64][rows][64]: column col of row pos at
-          // ((col / 64) * rows + pos) * 64 + col % 64
-          const int col = (o & ~31) + dq::kpos_of_col(o & 31);
-          uint16_t* hp = p.h_perm + static_cast<size_t>(col >> 6) * p.h_rows * 64 + (col & 63);
+    if constexpr (C::kPrefill) {
+      const int qd = warp & 3;
+      const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
+      uint32_t d_ctr = 0;
+      int gh = 0;
+      for (int i = blockIdx.x; i < total; i += gridDim.x) {
+        Item it;
+        decode_item<C>(p, s_prefix, G, i, it, gh);
+        const uint32_t jd = d_ctr % kNDBuf;
+        if (!mbar_wait_warp(&df[jd], (d_ctr / kNDBuf) & 1u, ctl)) break;
+        tc_fence_after();
+        const int o = it.row0 + 32 * qd + lane;
+        const bool live = o < it.rows;
+        // h = silu(g) * u goes to o's position in the down pass's K order
+        const int col = (o & ~31) + dq::kpos_of_col(o & 31);
+        uint16_t* hp = p.h_perm + static_cast<size_t>(col >> 6) * p.h_rows * 64 + (col & 63);
+        for (int c = 0; c < C::kNT / 32; ++c) {
+          if (32 * c >= it.ntok) break;
+          uint32_t v[32];
+          tmem_ld32(tmem_lane + jd * C::kDColsPerBuf + 32 * c, v);
+          tmem_wait_ld();
+          if (!live) continue;
+          const int nv = min(32, it.ntok - 32 * c);
+          const int pos = it.pos0 + 32 * c;
+          if (p.mode == kTcPfGate) {
 #pragma unroll
-          for (int n = 0; n < kNT; ++n) {
-            if (n >= it.ntok) break;
-            const float g = __uint_as_float(v[n]);
-            const float h = g / (1.0f + expf(-g)) * __uint_as_float(u[n]);
-            hp[static_cast<size_t>(it.pos0 + n) * 64] = __half_as_ushort(__float2half_rn(h));
+            for (int n = 0; n < 32; ++n) {
+              if (n >= nv) break;
+              p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] = __uint_as_float(v[n]);
+            }
+          } else if (p.mode == kTcPfUp) {
+#pragma unroll
+            for (int n = 0; n < 32; ++n) {
+              if (n >= nv) break;
+              const float g = p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o];
+              const float h = g / (1.0f + expf(-g)) * __uint_as_float(v[n]);
+              hp[static_cast<size_t>(pos + n) * 64] = __half_as_ushort(__float2half_rn(h));
+            }
+          } else {
+#pragma unroll
+            for (int n = 0; n < 32; ++n) {
+              if (n >= nv) break;
+              p.ysorted[static_cast<size_t>(pos + n) * p.H + o] =
+                  p.slot_w[pos + n] * __uint_as_float(v[n]);
+            }
           }
-        } else if (p.mode == kTcDown) {
-#pragma unroll
-          for (int n = 0; n < kNT; ++n) {
-            if (n >= it.ntok) break;
-            p.ysorted[it.split * p.split_stride + static_cast<size_t>(it.pos0 + n) * p.H + o] =
-                p.slot_w[it.pos0 + n] * __uint_as_float(v[n]);
-          }
-        } else {
-#pragma unroll
-          for (int n = 0; n < kNT; ++n) {
-            if (n >= it.ntok) break;
-            p.y[static_cast<size_t>(it.tok0 + n) * it.rows + o] = __uint_as_float(v[n]);
+        }
+        tc_fence_before();
+        mbar_arrive_warp(&de[jd]);
+        d_ctr++;
+      }
+    } else {
+      const int qd = warp & 3;
+      const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
+      uint32_t d_ctr = 0;
+      int gh = 0;
+      for (int i = blockIdx.x; i < total; i += gridDim.x) {
+        Item it;
+        decode_item<C>(p, s_prefix, G, i, it, gh);
+        const uint32_t jd = d_ctr & 1u;
+        if (!mbar_wait_warp(&df[jd], (d_ctr >> 1) & 1u, ctl)) break;
+        tc_fence_after();
+        uint32_t v[32], u[32];
+        tmem_ld32(tmem_lane + jd * C::kDColsPerBuf, v);
+        if (it.npass == 2) tmem_ld32(tmem_lane + jd * C::kDColsPerBuf + 32, u);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive_warp(&de[jd]);
+        d_ctr++;
+        const int o = it.row0 + 32 * qd + lane;
+        if (o < it.rows) {
+          if (p.mode == kTcGateUp) {
+            // h = silu(g) * u, fp16, at o's position in the down pass's K order
+            // atom-major [ld/64][rows][64]: column col of row pos at
+            // ((col / 64) * rows + pos) * 64 + col % 64
+            const int col = (o & ~31) + dq::kpos_of_col(o & 31);
+            uint16_t* hp = p.h_perm + static_cast<size_t>(col >> 6) * p.h_rows * 64 + (col & 63);
+  #pragma unroll
+            for (int n = 0; n < C::kNT; ++n) {
+              if (n >= it.ntok) break;
+              const float g = __uint_as_float(v[n]);
+              const float h = g / (1.0f + expf(-g)) * __uint_as_float(u[n]);
+              hp[static_cast<size_t>(it.pos0 + n) * 64] = __half_as_ushort(__float2half_rn(h));
+            }
+          } else if (p.mode == kTcDown) {
+  #pragma unroll
+            for (int n = 0; n < C::kNT; ++n) {
+              if (n >= it.ntok) break;
+              p.ysorted[it.split * p.split_stride + static_cast<size_t>(it.pos0 + n) * p.H + o] =
+                  p.slot_w[it.pos0 + n] * __uint_as_float(v[n]);
+            }
+          } else {
+  #pragma unroll
+            for (int n = 0; n < C::kNT; ++n) {
+              if (n >= it.ntok) break;
+              p.y[static_cast<size_t>(it.tok0 + n) * it.rows + o] = __uint_as_float(v[n]);
+            }
           }
         }
       }
+  
     }
   }
 
@@ -882,18 +1041,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
 
 }  // namespace
 
-size_t tc_smem_bytes() { return kSmemTotal; }
-
-cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s) {
+template <class C>
+cudaError_t launch_cfg(const TcParams& p, int n_sm, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemTotal));
+    cudaError_t e = cudaFuncSetAttribute(tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::kSmemTotal));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  tc_kernel<<<n_sm, kThreads, kSmemTotal, s>>>(p);
+  tc_kernel<C><<<n_sm, kThreads, C::kSmemTotal, s>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s) {
+  if (p.mode == kTcPfGate || p.mode == kTcPfUp || p.mode == kTcPfDown)
+    return launch_cfg<Pre>(p, n_sm, s);
+  return launch_cfg<Dec>(p, n_sm, s);
 }
 
 }  // namespace pw

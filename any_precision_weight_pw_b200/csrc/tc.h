@@ -7,15 +7,22 @@
 
 namespace pw {
 
-constexpr int kTcTokens = 32;  // token tile of one work item (MMA N <= 32)
-constexpr int kTcGateUp = 0;   // gate and up blocks of every group -> h = silu(g) * u
-constexpr int kTcDown = 1;     // down blocks, B = h -> routing-weighted partials
-constexpr int kTcLinear = 2;   // one standalone block -> y
+constexpr int kTcTokens = 32;   // decode token tile of one work item (MMA N <= 32)
+constexpr int kTcPfTokens = 256;  // prefill token chunk of one work item (MMA N = 256)
+// decode modes (token tiles of up to 32 rows)
+constexpr int kTcGateUp = 0;    // gate and up blocks of every group -> h = silu(g) * u
+constexpr int kTcDown = 1;      // down blocks, B = h -> routing-weighted partials
+constexpr int kTcLinear = 2;    // one standalone block -> y
+// prefill modes (256-token chunks; gate and up in separate launches)
+constexpr int kTcPfGate = 3;    // gate blocks -> g (fp32, gbuf)
+constexpr int kTcPfUp = 4;      // up blocks -> h = silu(g) * u (h_perm)
+constexpr int kTcPfDown = 5;    // down blocks -> routing-weighted outputs (ysorted)
 
 struct TcParams {
   CUtensorMap b_maps[4];         // token-tile source (modes 0, 1): x_sorted or h_perm
                                  // as {64 columns, rows, atoms}; box i holds 8(i+1)
                                  // rows x 4 atoms, 128-byte swizzle
+  CUtensorMap pf_map;            // prefill modes: the same source, box 256 rows x 1 atom
   PageTable pt;                  // planes, bits, active LUT slot per block (modes 0, 1)
   int mode;
   int H, F, S, E, n_groups, n_max;
@@ -34,10 +41,11 @@ struct TcParams {
   int lin_rows, lin_cols, lin_bits, lin_n_max;
   const uint16_t* lin_lut;
   const uint32_t* lin_planes;    // plane pages of the standalone block (mode 2)
+  float* gbuf;                   // prefill: gate outputs [rows][gbuf_ld] fp32
+  int gbuf_ld;
   int* err;                      // device error word (may be null)
 };
 
-size_t tc_smem_bytes();
 cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s);
 
 }  // namespace pw

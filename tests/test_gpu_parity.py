@@ -320,3 +320,51 @@ def test_prefill_scale_layer_sampled(pw, oracle):
     ref, sidx, _ = L.forward(x[sample], layer.router_w, layer.router_bias, threads=32)
     np.testing.assert_array_equal(sidx, idx[sample])
     assert_output_close(y[sample], ref)
+
+
+def _run_layer_env(pw, layer, T, env, batch=0):
+    old = {k: os.environ.get(k) for k in env}
+    os.environ.update(env)
+    try:
+        return _run_layer(pw, layer, T, batch=batch)
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+@pytest.mark.parametrize("T,bias_expert", [(200, None), (300, 5)])
+def test_prefill_passes_tiny_layer(pw, oracle, T, bias_expert):
+    """The prefill passes (256-token chunks; gate, up and down launches) on
+    the tiny layer, every output compared; with a router bias one expert gets
+    every token (two chunks, the second partial)."""
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=4)
+    if bias_expert is not None:
+        layer.router_bias = np.zeros(8, np.float32)
+        layer.router_bias[bias_expert] = 50.0
+    y, idx, w, x = _run_layer_env(pw, layer, T, {"PW_PREFILL": "1"})
+    ref, ridx, rw = _oracle_forward(oracle, layer, x, threads=32)
+    np.testing.assert_array_equal(idx, ridx)
+    assert_output_close(y, ref)
+    # the decode passes give the same routing and outputs within the same bound
+    y2, idx2, _, _ = _run_layer_env(pw, layer, T, {"PW_PREFILL": "0"})
+    np.testing.assert_array_equal(idx2, ridx)
+    assert_output_close(y2, ref)
+
+
+def test_prefill_passes_qwen_shaped_sampled(pw, oracle):
+    """Qwen-shaped layer (shared expert of 5632) through the prefill passes at
+    320 tokens: all routing, and the outputs of a token sample."""
+    layer = synth.Layer(synth.WORKLOADS["qwen15_moe_a27b"], seed=5)
+    T = 320
+    y, idx, w, x = _run_layer_env(pw, layer, T, {"PW_PREFILL": "1"})
+    wl = layer.wl
+    ridx, _ = oracle.topk_softmax(oracle.router_logits(x, layer.router_w, None), wl.top_k,
+                                  bool(wl.renorm_topk))
+    np.testing.assert_array_equal(idx, ridx)
+    sample = np.array([0, 1, 77, 150, 255, 256, 300, T - 1])
+    L = oracle_layer(oracle, layer)
+    ref, _, _ = L.forward(x[sample], layer.router_w, None, threads=32)
+    assert_output_close(y[sample], ref)
