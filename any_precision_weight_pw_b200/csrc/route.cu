@@ -18,6 +18,7 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kRouteThreads = 256;
 constexpr int kStageFloats = 4096;  // logits staged in shared memory (16 KB)
+constexpr int kStageSel = 16384;    // selections kept in shared memory (one byte each)
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -73,58 +74,66 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   __threadfence();
 
   // ---- phase 2 (one block): top-k + softmax ------------------------------
-  // Small problems stage the logits in shared memory with one coalesced pass
-  // (each thread's top-k then reads shared memory instead of waiting on L2).
+  // The logits are staged in shared memory a chunk of tokens at a time with
+  // coalesced loads, so each thread's top-k reads shared memory instead of
+  // waiting on L2; the selections stay in shared memory (one byte each) for
+  // the bucketing below when they fit.
   __shared__ float s_logits[kStageFloats];
-  const bool staged = T * E <= kStageFloats;
-  if (staged)
-    for (int j = threadIdx.x; j < T * E; j += kRouteThreads) s_logits[j] = __ldcg(ws.logits + j);
-  __syncthreads();
-  __shared__ int s_idx[kStageFloats];  // top-k of every token when staged
-  for (int t = threadIdx.x; t < T; t += kRouteThreads) {
-    const float* l = staged ? s_logits + t * E : ws.logits + static_cast<size_t>(t) * E;
-    int sel[PW_MAX_TOPK];
-    float lsel[PW_MAX_TOPK];
-    uint64_t taken_lo = 0ull, taken_hi = 0ull;  // experts already selected (E <= 128)
+  __shared__ uint8_t s_idx[kStageSel];
+  const bool sel_staged = T * k <= kStageSel;
+  const int chunk = kStageFloats / E;  // tokens per staged chunk (>= 32)
+  for (int t0 = 0; t0 < T; t0 += chunk) {
+    const int nt = min(chunk, T - t0);
+    __syncthreads();
+    for (int j = threadIdx.x; j < nt * E; j += kRouteThreads)
+      s_logits[j] = __ldcg(ws.logits + static_cast<size_t>(t0) * E + j);
+    __syncthreads();
+    for (int tl = threadIdx.x; tl < nt; tl += kRouteThreads) {
+      const int t = t0 + tl;
+      const float* l = s_logits + tl * E;
+      int sel[PW_MAX_TOPK];
+      float lsel[PW_MAX_TOPK];
+      uint64_t taken_lo = 0ull, taken_hi = 0ull;  // experts already selected (E <= 128)
 #pragma unroll
-    for (int j = 0; j < PW_MAX_TOPK; ++j) {
-      if (j >= k) break;
-      int bi = -1;
-      float best = 0.0f;
-      for (int e = 0; e < E; ++e) {
-        if ((((e < 64) ? taken_lo : taken_hi) >> (e & 63)) & 1ull) continue;
-        const float v = staged ? l[e] : __ldcg(l + e);
-        if (bi < 0 || v > best) {  // strict: equal logits keep the lower index
-          best = v;
-          bi = e;
+      for (int j = 0; j < PW_MAX_TOPK; ++j) {
+        if (j >= k) break;
+        int bi = -1;
+        float best = 0.0f;
+        for (int e = 0; e < E; ++e) {
+          if ((((e < 64) ? taken_lo : taken_hi) >> (e & 63)) & 1ull) continue;
+          const float v = l[e];
+          if (bi < 0 || v > best) {  // strict: equal logits keep the lower index
+            best = v;
+            bi = e;
+          }
         }
+        if (bi < 64) taken_lo |= 1ull << bi; else taken_hi |= 1ull << (bi & 63);
+        sel[j] = bi;
+        lsel[j] = best;
       }
-      if (bi < 64) taken_lo |= 1ull << bi; else taken_hi |= 1ull << (bi & 63);
-      sel[j] = bi;
-      lsel[j] = best;
-    }
-    const float mx = lsel[0];
-    float z = 0.0f;
-    for (int e = 0; e < E; ++e) z += expf((staged ? l[e] : __ldcg(l + e)) - mx);
-    float psel[PW_MAX_TOPK];
-    float ssum = 0.0f;
+      const float mx = lsel[0];
+      float z = 0.0f;
+      for (int e = 0; e < E; ++e) z += expf(l[e] - mx);
+      float psel[PW_MAX_TOPK];
+      float ssum = 0.0f;
 #pragma unroll
-    for (int j = 0; j < PW_MAX_TOPK; ++j) {
-      if (j >= k) break;
-      psel[j] = expf(lsel[j] - mx) / z;
-      ssum += psel[j];
-    }
+      for (int j = 0; j < PW_MAX_TOPK; ++j) {
+        if (j >= k) break;
+        psel[j] = expf(lsel[j] - mx) / z;
+        ssum += psel[j];
+      }
 #pragma unroll
-    for (int j = 0; j < PW_MAX_TOPK; ++j) {
-      if (j >= k) break;
-      ws.topk_idx[t * k + j] = sel[j];
-      ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
-      if (staged) s_idx[t * k + j] = sel[j];
+      for (int j = 0; j < PW_MAX_TOPK; ++j) {
+        if (j >= k) break;
+        ws.topk_idx[t * k + j] = sel[j];
+        ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
+        if (sel_staged) s_idx[t * k + j] = static_cast<uint8_t>(sel[j]);
+      }
     }
   }
   __syncthreads();
   auto sel_of = [&](int t, int j) -> int {
-    return staged ? s_idx[t * k + j] : __ldcg(ws.topk_idx + t * k + j);
+    return sel_staged ? static_cast<int>(s_idx[t * k + j]) : __ldcg(ws.topk_idx + t * k + j);
   };
 
   // ---- bucketing: counts per expert with warp ballots ---------------------
@@ -173,7 +182,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       if (slot >= 0) {
         const int pos = run + __popc(m & lt_mask);
         ws.slot_token[pos] = t;
-        ws.slot_w[pos] = __ldcg(ws.topk_w + t * k + slot);
         ws.token_pos[t * k + slot] = pos;
       }
       run += __popc(m);
@@ -187,6 +195,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       ws.token_pos[T * k + t] = pos;
     }
   }
+  // routing weight of every routed position (independent loads, all threads)
+  __syncthreads();
+  for (int j = threadIdx.x; j < T * k; j += kRouteThreads)
+    ws.slot_w[__ldcg(ws.token_pos + j)] = __ldcg(ws.topk_w + j);
 }
 
 // x_sorted row pos = the activations of token slot_token[pos] as fp16, each

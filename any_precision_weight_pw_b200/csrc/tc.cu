@@ -957,11 +957,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
               p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] = __uint_as_float(v[n]);
             }
           } else if (p.mode == kTcPfUp) {
+            // all 32 gate values first, so their loads overlap
+            float g[32];
+#pragma unroll
+            for (int n = 0; n < 32; ++n)
+              g[n] = (n < nv) ? p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] : 0.0f;
 #pragma unroll
             for (int n = 0; n < 32; ++n) {
               if (n >= nv) break;
-              const float g = p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o];
-              const float h = g / (1.0f + expf(-g)) * __uint_as_float(v[n]);
+              const float h = g[n] / (1.0f + expf(-g[n])) * __uint_as_float(v[n]);
               hp[static_cast<size_t>(pos + n) * 64] = __half_as_ushort(__float2half_rn(h));
             }
           } else {
