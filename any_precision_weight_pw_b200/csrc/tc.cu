@@ -257,6 +257,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v) {
       : "r"(taddr)
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -934,43 +944,60 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       for (int i = blockIdx.x; i < total; i += gridDim.x) {
         Item it;
         decode_item<C>(p, s_prefix, G, i, it, gh);
+        const int o = it.row0 + 32 * qd + lane;
+        const bool live = o < it.rows;
+        const bool up = p.mode == kTcPfUp;
+        // gate values of the next 16-token chunk are loaded one chunk ahead
+        // (the first chunk's before the accumulator is ready), so their
+        // latency hides behind the MMAs and the previous chunk's work
+        constexpr int kCh = 16;
+        float gn[kCh];
+        auto load_g = [&](int c) {
+          const int nv = min(kCh, it.ntok - kCh * c);
+          const int pos = it.pos0 + kCh * c;
+#pragma unroll
+          for (int n = 0; n < kCh; ++n)
+            gn[n] = (live && n < nv) ? p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] : 0.0f;
+        };
+        if (up) load_g(0);
         const uint32_t jd = d_ctr % kNDBuf;
         if (!mbar_wait_warp(&df[jd], (d_ctr / kNDBuf) & 1u, ctl)) break;
         tc_fence_after();
-        const int o = it.row0 + 32 * qd + lane;
-        const bool live = o < it.rows;
         // h = silu(g) * u goes to o's position in the down pass's K order
         const int col = (o & ~31) + dq::kpos_of_col(o & 31);
         uint16_t* hp = p.h_perm + static_cast<size_t>(col >> 6) * p.h_rows * 64 + (col & 63);
-        for (int c = 0; c < C::kNT / 32; ++c) {
-          if (32 * c >= it.ntok) break;
-          uint32_t v[32];
-          tmem_ld32(tmem_lane + jd * C::kDColsPerBuf + 32 * c, v);
+        for (int c = 0; c < C::kNT / kCh; ++c) {
+          if (kCh * c >= it.ntok) break;
+          uint32_t v[kCh];
+          tmem_ld16(tmem_lane + jd * C::kDColsPerBuf + kCh * c, v);
+          float g[kCh];
+          if (up) {
+#pragma unroll
+            for (int n = 0; n < kCh; ++n) g[n] = gn[n];
+            if (kCh * (c + 1) < it.ntok) load_g(c + 1);
+          }
           tmem_wait_ld();
           if (!live) continue;
-          const int nv = min(32, it.ntok - 32 * c);
-          const int pos = it.pos0 + 32 * c;
+          const int nv = min(kCh, it.ntok - kCh * c);
+          const int pos = it.pos0 + kCh * c;
           if (p.mode == kTcPfGate) {
 #pragma unroll
-            for (int n = 0; n < 32; ++n) {
+            for (int n = 0; n < kCh; ++n) {
               if (n >= nv) break;
               p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] = __uint_as_float(v[n]);
             }
-          } else if (p.mode == kTcPfUp) {
-            // all 32 gate values first, so their loads overlap
-            float g[32];
+          } else if (up) {
 #pragma unroll
-            for (int n = 0; n < 32; ++n)
-              g[n] = (n < nv) ? p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] : 0.0f;
-#pragma unroll
-            for (int n = 0; n < 32; ++n) {
+            for (int n = 0; n < kCh; ++n) {
               if (n >= nv) break;
-              const float h = g[n] / (1.0f + expf(-g[n])) * __uint_as_float(v[n]);
+              // the accumulator waits for this epilogue (one buffer), so the
+              // activation uses the fast exponential and division
+              const float h = __fdividef(g[n], 1.0f + __expf(-g[n])) * __uint_as_float(v[n]);
               hp[static_cast<size_t>(pos + n) * 64] = __half_as_ushort(__float2half_rn(h));
             }
           } else {
 #pragma unroll
-            for (int n = 0; n < 32; ++n) {
+            for (int n = 0; n < kCh; ++n) {
               if (n >= nv) break;
               p.ysorted[static_cast<size_t>(pos + n) * p.H + o] =
                   p.slot_w[pos + n] * __uint_as_float(v[n]);

@@ -61,7 +61,12 @@
  *   tensor-core kernel (TMA + tcgen05; activations are fed to it as fp16, so
  *   |x| and |silu(g) u| must stay below 65504); other shapes run on the
  *   CUDA-core kernel in fp32.  pw_linear takes the tensor-core kernel when
- *   cols is a multiple of 128.
+ *   cols is a multiple of 128.  At prefill-sized batches (routed slots
+ *   averaging at least 64 tokens per expert, and max_tokens giving at least
+ *   256 sorted positions: max_tokens * (top_k + (shared_ffn > 0)) >= 256)
+ *   the tensor-core passes work on 256-token chunks, gate and up as separate
+ *   launches with the gate output kept in a workspace buffer; the result is
+ *   the same computation (PW_PREFILL=0/1 in the environment forces either).
  */
 #ifndef PW_H_
 #define PW_H_
