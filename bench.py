@@ -526,10 +526,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--prefill", action="store_true",
+                    help="only the prefill-scale measurement (one JSON object; for profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.prefill:
+        import torch
+        print(json.dumps(prefill_measure(torch.device("cuda", local_rank), steps=max(args.steps, 1),
+                                         warmup=max(args.warmup, 1))), flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
