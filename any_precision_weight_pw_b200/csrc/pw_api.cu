@@ -150,6 +150,7 @@ struct pw_moe {
   CUtensorMap x_maps[4], h_maps[4];  // token-tile maps over x_sorted and h_perm
   CUtensorMap x_pf_map, h_pf_map;    // 256-row chunk maps (prefill passes)
   float* gbuf = nullptr;             // prefill: gate outputs [P_max][Fmax] fp32
+  int* gu_done = nullptr;            // fused decode launch: per-group gate/up counts
   int gbuf_ld = 0;
   bool pf = false;                   // the prefill passes are available
   float* ysorted = nullptr;
@@ -307,6 +308,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const size_t o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
   const size_t o_tk = off; off += al(sizeof(uint32_t) * 4);
   const size_t o_err = off; off += al(sizeof(int) * 4);
+  const size_t o_gd = off; off += al(sizeof(int) * (h->G + 1));
   const size_t o_gu = off; off += al(sizeof(float) * size_t(h->P_max) * h->gu_stride);
   const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->x_ld);
   const size_t o_hp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->h_perm_ld);
@@ -330,6 +332,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->ws.token_pos = reinterpret_cast<int32_t*>(w + o_tp);
   h->ws.ticket = reinterpret_cast<uint32_t*>(w + o_tk);
   h->err = reinterpret_cast<int*>(w + o_err);
+  h->gu_done = reinterpret_cast<int*>(w + o_gd);
   h->gu = reinterpret_cast<float*>(w + o_gu);
   h->x_sorted = reinterpret_cast<uint16_t*>(w + o_xp);
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
@@ -337,7 +340,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->gbuf = reinterpret_cast<float*>(w + o_gb);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
   h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
-  if (cudaMemset(w + o_tk, 0, al(sizeof(uint32_t) * 4) + al(sizeof(int) * 4)) != cudaSuccess ||
+  if (cudaMemset(w + o_tk, 0, o_gd + al(sizeof(int) * (h->G + 1)) - o_tk) != cudaSuccess ||
       cudaMemset(w + o_xp, 0, o_sx - o_xp) != cudaSuccess) {
     free_all(h);
     return fail(PW_ERR_CUDA, "cudaMemset failed");
@@ -431,6 +434,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   }
   const int has_shared = c.shared_ffn > 0 ? 1 : 0;
   const bool prefill = h->tc && use_prefill(h, T);
+  // decode: gate/up and down in one launch (PW_FUSED=0 splits them)
+  const bool fused = h->tc && !prefill && env_int("PW_FUSED", 1) != 0;
   std::vector<cudaEvent_t> evs;
   if (h->profiling) {
     for (int i = 0; i < 5; ++i) {
@@ -460,6 +465,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   rp.renorm = c.renorm_topk;
   rp.has_shared = has_shared;
   rp.ws = h->ws;
+  rp.zero_words = fused ? h->gu_done : nullptr;
+  rp.n_zero = fused ? h->G : 0;
   PW_CUDA(pw::launch_route(rp, h->n_sm, s));
   PW_CUDA(mark(1));
 
@@ -478,7 +485,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
-    tp.mode = prefill ? pw::kTcPfGate : pw::kTcGateUp;
+    tp.mode = prefill ? pw::kTcPfGate : (fused ? pw::kTcFused : pw::kTcGateUp);
     tp.H = c.hidden;
     tp.F = c.ffn;
     tp.S = c.shared_ffn;
@@ -494,6 +501,13 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_perm_ld = h->h_perm_ld;
     tp.h_rows = h->P_max;
     tp.err = h->err;
+    if (fused) {
+      tp.n_split = down_splits(h, T);
+      for (int i = 0; i < 4; ++i) tp.h_maps[i] = h->h_maps[i];
+      tp.gu_done = h->gu_done;
+      tp.ysorted = h->ysorted;
+      tp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
+    }
     if (prefill) {
       // gate -> g (fp32), then up -> h = silu(g) * u
       tp.pf_map = h->x_pf_map;
@@ -526,7 +540,9 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   PW_CUDA(mark(2));
   // down pass
   int n_split = 1;
-  if (h->tc) {
+  if (fused) {
+    n_split = down_splits(h, T);  // the down items ran in the launch above
+  } else if (h->tc) {
     n_split = prefill ? 1 : down_splits(h, T);
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
@@ -733,7 +749,8 @@ int32_t pw_forward_launches(const pw_moe_t* h, int32_t T) {
   if (!h) return 0;
   if (T <= 0) return 0;
   if (!h->tc) return 4;
-  return use_prefill(h, T) ? 6 : 5;
+  if (use_prefill(h, T)) return 6;
+  return env_int("PW_FUSED", 1) != 0 ? 4 : 5;
 }
 
 pw_status_t pw_destroy(pw_moe_t* h) {

@@ -47,6 +47,8 @@ struct RouteParams {
   const float* bias;       // [E] or null
   int T, H, E, k, renorm, has_shared;
   RouteWorkspace ws;
+  int* zero_words;         // counters of the launches that follow, set to zero
+  int n_zero;              // (may be null / 0)
 };
 
 struct GatherParams {

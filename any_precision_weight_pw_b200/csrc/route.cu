@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       s_off[E + 1] = run + T;
     }
     for (int g = 0; g <= G; ++g) ws.offsets[g] = s_off[g];
+    for (int j = 0; j < p.n_zero; ++j) p.zero_words[j] = 0;
     *ws.ticket = 0u;  // ready for the next forward (kernels on a stream do not overlap)
   }
   __syncthreads();

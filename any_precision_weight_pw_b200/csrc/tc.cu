@@ -95,7 +95,7 @@ struct Cfg {
   static constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
   static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 2 * kNDBuf + 2;
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-  static constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 4 * (kMaxGroups + 2);
+  static constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 8 * (kMaxGroups + 2);
   static constexpr uint32_t kSmemTotal = kOffSlotUser + 4 * kNSlot;
   static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
   static_assert(kAColBase + kNA * kAColsPerSlot <= kTmemCols, "tensor memory budget");
@@ -200,6 +200,28 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
       : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// A fused launch's down item of group g reads h rows that other CTAs' gate/up
+// epilogues write: wait (bounded) until all of g's gate/up items are counted,
+// then order the TMA reads that follow after those writes.
+__device__ __noinline__ bool wait_gate_up(const TcParams& p, int g, int need, const Ctl& c) {
+  const unsigned long long t0 = global_ns();
+  while (ld_acquire_gpu(p.gu_done + g) < need) {
+    if (*c.abort) return false;
+    if (global_ns() - t0 > kWaitNs) {
+      *c.abort = 1;
+      if (c.err) atomicExch(c.err, PW_ERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(200);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -316,6 +338,7 @@ struct Pass {
 };
 struct Item {
   int g, row0, tok0, ntok, pos0, split, rows, cols, npass, s_begin, s_end;
+  int kind;  // the item's pass: the launch mode, or gate/up or down in a fused launch
 };
 
 // Items are visited in increasing order by every role, so the group search
@@ -324,13 +347,30 @@ __device__ __forceinline__ bool gate_or_up(int mode) {
   return mode == kTcGateUp || mode == kTcPfGate || mode == kTcPfUp;
 }
 
+// Items of a fused launch: [0, s_prefix[G]) gate/up, then the down items
+// listed by s_prefix2; gh holds one search hint per list.
 template <class C>
-__device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix, int G,
-                                            int i, Item& it, int& gh) {
-  int g = gh;
-  while (g + 1 < G && s_prefix[g + 1] <= i) ++g;
-  gh = g;
-  const int local = i - s_prefix[g];
+__device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix,
+                                            const int* s_prefix2, int G, int i, Item& it,
+                                            int (&gh)[2]) {
+  int kind = p.mode;
+  const int* pre = s_prefix;
+  int li = i, hl = 0;
+  if (p.mode == kTcFused) {
+    if (i < s_prefix[G]) {
+      kind = kTcGateUp;
+    } else {
+      kind = kTcDown;
+      pre = s_prefix2;
+      li = i - s_prefix[G];
+      hl = 1;
+    }
+  }
+  int g = gh[hl];
+  while (g + 1 < G && pre[g + 1] <= li) ++g;
+  gh[hl] = g;
+  it.kind = kind;
+  const int local = li - pre[g];
   int n, pos0;
   if (p.mode == kTcLinear) {
     it.rows = p.lin_rows;
@@ -339,8 +379,8 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
     pos0 = 0;
   } else {
     const int Fg = (g == p.E) ? p.S : p.F;
-    it.rows = gate_or_up(p.mode) ? Fg : p.H;
-    it.cols = gate_or_up(p.mode) ? p.H : Fg;
+    it.rows = gate_or_up(kind) ? Fg : p.H;
+    it.cols = gate_or_up(kind) ? p.H : Fg;
     pos0 = p.offsets[g];
     n = p.offsets[g + 1] - pos0;
   }
@@ -363,7 +403,7 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
     it.npass = 1;
     return;
   }
-  const int ns = p.n_split;
+  const int ns = (kind == kTcDown) ? p.n_split : 1;
   const int per_tt = rt * ns;
   const int tt = local / per_tt;
   const int r = local - tt * per_tt;
@@ -375,15 +415,15 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
   it.pos0 = pos0 + it.tok0;
   it.s_begin = static_cast<int>((static_cast<long long>(stages) * it.split) / ns);
   it.s_end = static_cast<int>((static_cast<long long>(stages) * (it.split + 1)) / ns);
-  it.npass = (p.mode == kTcGateUp) ? 2 : 1;
+  it.npass = (kind == kTcGateUp) ? 2 : 1;
 }
 
 // Block, bitwidth, LUT and plane tensor map of pass q of an item.
 __device__ __forceinline__ Pass get_pass(const TcParams& p, const Item& it, int q) {
   if (p.mode == kTcLinear) return Pass{-1, p.lin_bits, p.lin_lut, p.lin_planes};
-  const int proj = (p.mode == kTcGateUp) ? q
-                   : (p.mode == kTcPfGate) ? 0
-                   : (p.mode == kTcPfUp) ? 1 : 2;
+  const int proj = (it.kind == kTcGateUp) ? q
+                   : (it.kind == kTcPfGate) ? 0
+                   : (it.kind == kTcPfUp) ? 1 : 2;
   const int blk = 3 * it.g + proj;
   return Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.pt.blk[blk].planes};
 }
@@ -611,6 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_prefix = reinterpret_cast<int*>(smem + C::kOffMisc + 16);
+  int* s_prefix2 = s_prefix + (kMaxGroups + 2);  // fused launch: the down items
   uint32_t* slot_user = reinterpret_cast<uint32_t*>(smem + C::kOffSlotUser);  // producer only
 
   const int warp = threadIdx.x >> 5;
@@ -640,23 +681,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     // the table offsets assume a 1024-byte aligned dynamic shared memory base
     *s_abort = (smem_addr(smem) & 1023u) ? 1 : 0;
     if (*s_abort && p.err) atomicExch(p.err, PW_ERR_UNSUPPORTED);
-    // items per group: row tiles x token tiles x K splits
-    int acc = 0;
-    for (int g = 0; g < G; ++g) {
-      s_prefix[g] = acc;
-      int rows, n;
-      if (p.mode == kTcLinear) {
-        rows = p.lin_rows;
-        n = p.T;
-      } else {
-        const int Fg = (g == p.E) ? p.S : p.F;
-        rows = gate_or_up(p.mode) ? Fg : p.H;
-        n = p.offsets[g + 1] - p.offsets[g];
+    // items per group: row tiles x token tiles x K splits (gate/up items of a
+    // fused launch take no split; its down items are listed in s_prefix2)
+    for (int list = 0; list < (p.mode == kTcFused ? 2 : 1); ++list) {
+      const int kind = (p.mode == kTcFused) ? (list == 0 ? kTcGateUp : kTcDown) : p.mode;
+      int* pre = list == 0 ? s_prefix : s_prefix2;
+      int acc = 0;
+      for (int g = 0; g < G; ++g) {
+        pre[g] = acc;
+        int rows, n;
+        if (p.mode == kTcLinear) {
+          rows = p.lin_rows;
+          n = p.T;
+        } else {
+          const int Fg = (g == p.E) ? p.S : p.F;
+          rows = gate_or_up(kind) ? Fg : p.H;
+          n = p.offsets[g + 1] - p.offsets[g];
+        }
+        const int tt = (n + C::kNT - 1) / C::kNT;
+        acc += ((rows + kTileRows - 1) / kTileRows) * tt * (kind == kTcDown ? p.n_split : 1);
       }
-      const int tt = (n + C::kNT - 1) / C::kNT;
-      acc += ((rows + kTileRows - 1) / kTileRows) * tt * p.n_split;
+      pre[G] = acc;
     }
-    s_prefix[G] = acc;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -669,13 +715,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int total = *s_abort ? 0 : s_prefix[G];
+  const int total =
+      *s_abort ? 0 : s_prefix[G] + (p.mode == kTcFused ? s_prefix2[G] : 0);
   const Ctl ctl{s_abort, p.err};
 
   if (warp < 8) {
     // ------------------------------------------------ dequantisers
     DequantState st{0u, 0u, 0u};
-    int gh = 0;
+    int gh[2] = {0, 0};
     const int grp = warp >> 2, quad = warp & 3;
     const int r = 32 * quad + lane;
     uint32_t sync_phase = 0;
@@ -686,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     Item it;
     LutPrefetch pre;
     if (i < total) {
-      decode_item<C>(p, s_prefix, G, i, it, gh);
+      decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
       lut_prefetch(it, get_pass(p, it, 0), grp, r, pre);
     }
     while (i < total && ok) {
@@ -700,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       if (nq >= it.npass) {
         ni = i + gridDim.x;
         nq = 0;
-        if (ni < total) decode_item<C>(p, s_prefix, G, ni, it, gh);
+        if (ni < total) decode_item<C>(p, s_prefix, s_prefix2, G, ni, it, gh);
       }
       if (ni < total) lut_prefetch(it, get_pass(p, it, nq), grp, r, pre);
       switch (ps.bits) {
@@ -720,12 +767,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     // ------------------------------------------------ producer (planes)
     if (lane == 0) {
       uint32_t t = 0, ring_end = 0;
-      int gh = 0;
+      int gh[2] = {0, 0};
       bool ok = true;
       const int n_max = (p.mode == kTcLinear) ? p.lin_n_max : p.n_max;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
-        decode_item<C>(p, s_prefix, G, i, it, gh);
+        decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
         const int n_kt = pages::k_tiles(it.cols);
         const int rt = it.row0 / kTileRows;
         for (int q = 0; q < it.npass && ok; ++q) {
@@ -772,12 +819,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   } else if (warp == kWarpLoader) {
     // ------------------------------------------------ token-tile loader
     uint32_t b_ctr = 0;
-    int gh = 0;
+    int gh[2] = {0, 0};
     bool ok = true;
     for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
       Item it;
-      decode_item<C>(p, s_prefix, G, i, it, gh);
+      decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
       const int rows_b = tile_rows(it.ntok);  // token rows loaded per stage (decode)
+      const bool fused_down = p.mode == kTcFused && it.kind == kTcDown;
+      if (fused_down && lane == 0)
+        ok = wait_gate_up(p, it.g, 4 * (s_prefix[it.g + 1] - s_prefix[it.g]), ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      const CUtensorMap* bmaps = fused_down ? p.h_maps : p.b_maps;
       for (int q = 0; q < it.npass && ok; ++q) {
         for (int s = it.s_begin; s < it.s_end && ok; ++s) {
           for (int j = 0; j < C::kBPerStage; ++j) {
@@ -800,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             } else if (lane == 0) {
               // {64 columns, rows_b rows, 4 atoms} starting at column 256 s
               mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(rows_b) * 4u * 128u);
-              tma_load_3d(buf, &p.b_maps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s, &bfull[jb]);
+              tma_load_3d(buf, &bmaps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s, &bfull[jb]);
             }
             b_ctr++;
           }
@@ -817,14 +869,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     // The whole warp walks the items and waits (so every operand address is
     // warp-uniform); one elected lane issues the MMAs and their commits.
     const bool leader = elect_one();
-    int gh = 0;
+    int gh[2] = {0, 0};
     uint32_t a_ctr = 0, b_ctr = 0, d_ctr = 0;
     bool ok = true;
     if constexpr (C::kPrefill) {
       const uint32_t idesc = mma_idesc(C::kNT);
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
-        decode_item<C>(p, s_prefix, G, i, it, gh);
+        decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
         const uint32_t jd = d_ctr % kNDBuf;
         if (!mbar_wait_warp(&de[jd], ((d_ctr / kNDBuf) & 1u) ^ 1u, ctl)) break;
         tc_fence_after();
@@ -874,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     } else {
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
-        decode_item<C>(p, s_prefix, G, i, it, gh);
+        decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
         const int n = it.ntok <= 16 ? 16 : 32;
         const uint32_t idesc = mma_idesc(n);
         // descriptor step of one 64-column atom of the token tile (16-byte units)
@@ -940,10 +992,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       const int qd = warp & 3;
       const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
       uint32_t d_ctr = 0;
-      int gh = 0;
+      int gh[2] = {0, 0};
       for (int i = blockIdx.x; i < total; i += gridDim.x) {
         Item it;
-        decode_item<C>(p, s_prefix, G, i, it, gh);
+        decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
         const int o = it.row0 + 32 * qd + lane;
         const bool live = o < it.rows;
         const bool up = p.mode == kTcPfUp;
@@ -1012,10 +1064,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       const int qd = warp & 3;
       const uint32_t tmem_lane = tmem_base + (static_cast<uint32_t>(32 * qd) << 16);
       uint32_t d_ctr = 0;
-      int gh = 0;
+      int gh[2] = {0, 0};
       for (int i = blockIdx.x; i < total; i += gridDim.x) {
         Item it;
-        decode_item<C>(p, s_prefix, G, i, it, gh);
+        decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
         const uint32_t jd = d_ctr & 1u;
         if (!mbar_wait_warp(&df[jd], (d_ctr >> 1) & 1u, ctl)) break;
         tc_fence_after();
@@ -1028,32 +1080,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         d_ctr++;
         const int o = it.row0 + 32 * qd + lane;
         if (o < it.rows) {
-          if (p.mode == kTcGateUp) {
+          if (it.kind == kTcGateUp) {
             // h = silu(g) * u, fp16, at o's position in the down pass's K order
             // atom-major [ld/64][rows][64]: column col of row pos at
             // ((col / 64) * rows + pos) * 64 + col % 64
             const int col = (o & ~31) + dq::kpos_of_col(o & 31);
             uint16_t* hp = p.h_perm + static_cast<size_t>(col >> 6) * p.h_rows * 64 + (col & 63);
-  #pragma unroll
+#pragma unroll
             for (int n = 0; n < C::kNT; ++n) {
               if (n >= it.ntok) break;
               const float g = __uint_as_float(v[n]);
               const float h = g / (1.0f + expf(-g)) * __uint_as_float(u[n]);
               hp[static_cast<size_t>(it.pos0 + n) * 64] = __half_as_ushort(__float2half_rn(h));
             }
-          } else if (p.mode == kTcDown) {
-  #pragma unroll
+          } else if (it.kind == kTcDown) {
+#pragma unroll
             for (int n = 0; n < C::kNT; ++n) {
               if (n >= it.ntok) break;
               p.ysorted[it.split * p.split_stride + static_cast<size_t>(it.pos0 + n) * p.H + o] =
                   p.slot_w[it.pos0 + n] * __uint_as_float(v[n]);
             }
           } else {
-  #pragma unroll
+#pragma unroll
             for (int n = 0; n < C::kNT; ++n) {
               if (n >= it.ntok) break;
               p.y[static_cast<size_t>(it.tok0 + n) * it.rows + o] = __uint_as_float(v[n]);
             }
+          }
+        }
+        if (p.mode == kTcFused && it.kind == kTcGateUp) {
+          // this warp's h rows of the item are written: count them for the
+          // group's down items (the fence makes every lane's stores visible
+          // at GPU scope before the count)
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            atomicAdd(p.gu_done + it.g, 1);
           }
         }
       }

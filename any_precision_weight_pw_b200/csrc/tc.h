@@ -17,12 +17,16 @@ constexpr int kTcLinear = 2;    // one standalone block -> y
 constexpr int kTcPfGate = 3;    // gate blocks -> g (fp32, gbuf)
 constexpr int kTcPfUp = 4;      // up blocks -> h = silu(g) * u (h_perm)
 constexpr int kTcPfDown = 5;    // down blocks -> routing-weighted outputs (ysorted)
+// decode, both passes in one launch: gate/up items, then down items; a down
+// item of group g starts loading h once g's gate/up items are all written
+constexpr int kTcFused = 6;
 
 struct TcParams {
   CUtensorMap b_maps[4];         // token-tile source (modes 0, 1): x_sorted or h_perm
                                  // as {64 columns, rows, atoms}; box i holds 8(i+1)
                                  // rows x 4 atoms, 128-byte swizzle
   CUtensorMap pf_map;            // prefill modes: the same source, box 256 rows x 1 atom
+  CUtensorMap h_maps[4];         // fused mode: the down items' source (h_perm)
   PageTable pt;                  // planes, bits, active LUT slot per block (modes 0, 1)
   int mode;
   int H, F, S, E, n_groups, n_max;
@@ -41,6 +45,8 @@ struct TcParams {
   int lin_rows, lin_cols, lin_bits, lin_n_max;
   const uint16_t* lin_lut;
   const uint32_t* lin_planes;    // plane pages of the standalone block (mode 2)
+  int* gu_done;                   // fused mode: per group, 4 x gate/up items written
+                                 // (zero at launch)
   float* gbuf;                   // prefill: gate outputs [rows][gbuf_ld] fp32
   int gbuf_ld;
   int* err;                      // device error word (may be null)
