@@ -191,7 +191,9 @@ void free_all(pw_moe* h) {
   delete h;
 }
 
-int down_splits(const pw_moe* h, int T) {
+// K splits of the down items: enough items for `per_sm` rounds of the grid
+// (more in the fused launch, where down items also fill the gate/up tail).
+int down_splits(const pw_moe* h, int T, int per_sm) {
   const pw_moe_config_t& c = h->cfg;
   const int forced = env_int("PW_DOWN_SPLIT", 0);
   if (forced > 0) return forced < h->max_split ? forced : h->max_split;
@@ -199,7 +201,7 @@ int down_splits(const pw_moe* h, int T) {
   int groups = T * c.top_k < c.n_experts ? T * c.top_k : c.n_experts;
   if (c.shared_ffn > 0) groups += 1;
   const int items = row_tiles * groups;
-  int ns = (4 * h->n_sm + items - 1) / items;
+  int ns = (per_sm * h->n_sm + items - 1) / items;
   const int stages = ((c.ffn + 31) / 32 + 7) / 8;
   if (ns > stages) ns = stages;
   if (ns > h->max_split) ns = h->max_split;
@@ -502,7 +504,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_rows = h->P_max;
     tp.err = h->err;
     if (fused) {
-      tp.n_split = down_splits(h, T);
+      tp.n_split = down_splits(h, T, 6);
       for (int i = 0; i < 4; ++i) tp.h_maps[i] = h->h_maps[i];
       tp.gu_done = h->gu_done;
       tp.ysorted = h->ysorted;
@@ -541,9 +543,9 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   // down pass
   int n_split = 1;
   if (fused) {
-    n_split = down_splits(h, T);  // the down items ran in the launch above
+    n_split = down_splits(h, T, 6);  // the down items ran in the launch above
   } else if (h->tc) {
-    n_split = prefill ? 1 : down_splits(h, T);
+    n_split = prefill ? 1 : down_splits(h, T, 4);
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.pt = pt;
