@@ -47,6 +47,24 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x, world, device=None):
+    """The largest of every rank's value (all ranks get it; timings are taken
+    as the slowest rank's).  world == 1 returns x unchanged."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, steps, T, ms):
+    """Tokens per second of the whole job: every rank runs `steps` forwards of
+    T tokens (its own replica) in the slowest rank's `ms`."""
+    return world * steps * T / (ms / 1e3)
+
+
 # ---------------------------------------------------------------- bytes
 def block_bytes(layer, blk):
     rows, cols = layer.shape(blk)
@@ -304,16 +322,12 @@ def run_ours(args, rank, world, local_rank):
     d.profile(False)
     launches_per_forward = d.launches(T)
     d.check_device_error()
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     steps = args.steps
     bytes_total = sum(bts[i % N_BATCHES]["total"] for i in range(steps))
     bytes_gu = sum(bts[i % N_BATCHES]["gu"] for i in range(steps))
     bytes_down = sum(bts[i % N_BATCHES]["down"] for i in range(steps))
-    tok_s = world * steps * T / (ms_max / 1e3)
+    tok_s = whole_job_rate(world, steps, T, ms_max)
     fwd_gbs = bytes_total / (ms / 1e3) / 1e9
     # dominant kernel: the tensor-core dequant-GEMM (its gate/up and down launches)
     tc_ms = per_launch[1] + per_launch[2]
@@ -342,7 +356,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e2.elapsed_time(e3)
     e2e_wall = time.perf_counter() - t0
-    e2e_tok_s = world * args.steps * T / (max(e2e_ms, e2e_wall * 1e3) / 1e3)
+    e2e_tok_s = whole_job_rate(world, args.steps, T,
+                               max_over_ranks(max(e2e_ms, e2e_wall * 1e3), world, dev))
 
     # decode sweep (other batch sizes and the Qwen-shaped layer); L2 flushed
     # between timed forwards so small layers are not served from cache
