@@ -427,7 +427,7 @@ def run_ours(args, rank, world, local_rank):
         "hbm_gbs": round(fwd_gbs, 1),
         "hbm_frac": round(fwd_gbs / hbm_peak, 4),
         "hbm_peak": {"gbs": hbm_peak, "kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": "tc_kernel (gate/up + down launches)",
+        "roofline": {"bound": "hbm", "kernel": "tc_kernel (gate/up and down items; one fused launch at decode)",
                      "achieved": round(tc_gbs, 1) if tc_gbs else None, "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(tc_gbs / hbm_peak, 4) if tc_gbs else None,
                      "traffic": traffic,
