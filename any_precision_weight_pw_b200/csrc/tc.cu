@@ -6,11 +6,15 @@
 // resident pages directly, at a separate bitwidth for every linear-block, and
 // fuses the expert activation and the output accumulation.
 //
-// One persistent CTA per SM walks a list of work items.  An item is 128
-// output rows x up to 32 tokens of one expert, in one or two passes over K:
-// the gate/up item makes a gate pass and an up pass over the same rows (so
+// One persistent CTA per SM walks a list of work items.  A decode item is
+// 128 output rows x up to 32 tokens of one expert, in one or two passes over
+// K: the gate/up item makes a gate pass and an up pass over the same rows (so
 // its epilogue can apply SwiGLU); the down item makes one pass (over one K
-// range when the down pass is split); a standalone linear makes one pass.
+// range when the down pass is split); a standalone linear makes one pass.  At
+// decode both kinds run in one launch (mode kTcFused): gate/up items first,
+// then down items, a down item of group g loading h only after g's gate/up
+// epilogues have all counted themselves.  Prefill items (Cfg<true>) are 128
+// rows x 256 tokens, one pass each, gate, up and down as three launches.
 //   warp 8      producer: streams only the b active bit-planes of the block,
 //               128 rows x 256 columns (8 words) per stage: in the paged
 //               layout (pages.h) the b tiles are one contiguous b * 4 KB run,
@@ -21,24 +25,25 @@
 //   warp 10     token-tile loader: the item's token rows are contiguous in an
 //               fp16 buffer already in the A operand's K order (the gathered
 //               activations for gate/up, h = silu(g)*u for down), so one lane
-//               moves each stage's tile with ONE 3-D TMA box (4 atoms of 64
-//               columns x 8, 16, 24 or 32 rows, 128-byte swizzle = the MMA's
-//               K-major B layout) into a 4-deep ring.  A standalone linear
-//               converts its bf16 rows with all 32 lanes instead.
+//               moves each stage's tile with ONE 3-D TMA box (decode: 4 atoms
+//               of 64 columns x 8, 16, 24 or 32 rows; prefill: 1 atom x 256
+//               rows; 128-byte swizzle = the MMA's K-major B layout).  A
+//               standalone linear converts its bf16 rows with all 32 lanes.
 //   warps 0-7   dequantisers in two K halves: warps q and q+4 both own rows
 //               32q..32q+31 (thread <-> output row <-> TMEM lane); the first
 //               group takes columns 0-127 of every stage, the second
 //               columns 128-255.  Each thread unpacks its row's codes from the
-//               b plane words, looks them up in its row's LUT (registers for
-//               b <= 3, else a shared-memory table with one bank per thread;
-//               see dequant.cuh) and writes fp16 weights into a TMEM ring
-//               slot (the MMA's A operand).
-//   warp 9      MMA issuer: tcgen05.mma kind::f16, M=128, N=16/32, K=16,
-//               fp32 accumulators in TMEM (two buffers, alternating items;
-//               gate and up accumulate side by side).
+//               b plane words (a bit-matrix transpose), looks them up in the
+//               shared-memory table of the pass (pair table for b <= 3,
+//               single table above; see dequant.cuh) and writes fp16 weights
+//               into a TMEM ring slot (the MMA's A operand).
+//   warp 9      MMA issuer: tcgen05.mma kind::f16, M=128, N=16/32 (decode)
+//               or 256 (prefill), K=16, fp32 accumulators in TMEM (decode:
+//               two buffers, alternating items, gate and up side by side).
 //   warps 11-14 epilogue: tcgen05.ld the accumulators; write h = silu(g)*u
 //               as fp16 in the down pass's K order (gate/up), the routing-
-//               weighted fp32 partials (down), or the fp32 result (linear).
+//               weighted fp32 partials (down), g (prefill gate) or the fp32
+//               result (linear).
 // Every wait is an mbarrier try_wait (with a suspend hint, so waiting warps
 // do not spin) bounded by a global-timer deadline; a timeout raises the CTA's
 // abort flag and the device error word, and every role drains what it has in

@@ -67,6 +67,11 @@
  *   the tensor-core passes work on 256-token chunks, gate and up as separate
  *   launches with the gate output kept in a workspace buffer; the result is
  *   the same computation (PW_PREFILL=0/1 in the environment forces either).
+ *   At decode both tensor-core passes run in one launch (gate/up items, then
+ *   down items, each down item waiting on its expert's gate/up items).
+ *   Environment switches, for tests and measurements only: PW_FUSED=0 (two
+ *   decode launches), PW_PREFILL=0/1, PW_DOWN_SPLIT=n (K splits of the down
+ *   items), PW_FORCE_SIMPLE=1 (CUDA-core kernel; read at pw_moe_create).
  */
 #ifndef PW_H_
 #define PW_H_
