@@ -176,7 +176,9 @@ pw_status_t pw_repack_planes(const uint32_t* d_src, uint32_t* d_dst, int32_t row
  * with fp32 output.  d_planes: a block of n_max planes in the paged layout
  * (bits <= n_max are read), d_lut [rows][2^bits]
  * fp16, d_x bf16 [T][cols], d_y fp32 [T][rows]; T >= 0, bits 1..8.  Uses the
- * same dequantisation and contraction as the MoE experts. */
+ * same dequantisation and contraction as the MoE experts.  Its device waits
+ * are bounded like the forward's, but it has no handle and so no device
+ * error word: a wait that gives up leaves d_y unspecified without a report. */
 pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t rows,
                       int32_t cols, int32_t n_max, int32_t bits, const uint16_t* d_x,
                       int32_t T, float* d_y, pw_stream_t stream);
