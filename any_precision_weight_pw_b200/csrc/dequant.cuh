@@ -14,14 +14,18 @@
 // becomes bit p of every byte, so byte n of output row q collects column
 // 8n + q.  The byte then IS an address byte: one byte permute (PRMT) puts it
 // next to the thread's row byte, and one shared-memory load fetches the
-// entry.  Two tables, both 128 local rows (threads) x at most 64 KB:
-//   b <= 3   pair table: the byte holds (v1 << (b + 1)) | (v2 << 1) | h for
-//            columns c (v1) and c + 4 (v2) and the row half h = r >= 64;
-//            the 32-bit entry at byte (byte << 8) | 4 (r mod 64) is the fp16
-//            pair (LUT[v1], LUT[v2]) -- one load gives one output register.
-//   b >= 4   single table: the byte holds v; the fp16 entry of row r is at
+// entry.  Two tables, both for 128 local rows (threads):
+//   pair     b <= 4: the 32-bit entry for codes v1 (column c) and v2 (column
+//            c + 4) is the fp16 pair (LUT[v1], LUT[v2]) -- one load gives one
+//            output register.  For b <= 3 the byte holds
+//            (v1 << (b + 1)) | (v2 << 1) | h with the row half h = r >= 64,
+//            and the entry sits at byte (byte << 8) | 4 (r mod 64) (<= 64 KB);
+//            for b = 4 the byte is (v1 << 4) | v2 and h moves to the third
+//            address byte: (h << 16) | (byte << 8) | 4 (r mod 64) (128 KB).
+//   single   b >= 4: the byte holds v; the fp16 entry of row r is at
 //            byte (v << 8) | 4 (r mod 64) | 2h (rows r and r + 64 share a
-//            word).  Two loads and one multiply-add give one output register.
+//            word, 64 KB).  Two loads and one multiply-add give one output
+//            register.
 // In both the 32 threads of a warp (32 consecutive rows) read 32 different
 // banks.  Shifts are written as multiplies (left) and high multiplies (right)
 // so they issue on the FMA pipe; the ALU pipe keeps the LOP3 and PRMT work.
@@ -113,41 +117,50 @@ PW_HD void transpose8_lo(uint32_t (&X)[8]) {
   delta_swap<1>(X[2], X[3], 0x55555555u);
 }
 
-// Address of the entry for byte N of x: byte 0 from rowb (the row byte),
-// byte 1 = byte N of x, bytes 2-3 from byte 1 of rowb (zero).
+// Address of the entry for byte N of x: byte 0 = byte 0 of rowb (the row
+// byte), byte 1 = byte N of x, byte 2 = byte 1 of rowb (the row half for b = 4
+// pair tables, else zero), byte 3 = byte 2 of rowb (zero).
 template <int N>
 PW_HD uint32_t code_addr(uint32_t x, uint32_t rowb) {
-  return prmt(x, rowb, 0x5504u | (static_cast<uint32_t>(N) << 4));
+  return prmt(x, rowb, 0x6504u | (static_cast<uint32_t>(N) << 4));
 }
 
-// Row bytes: pair table 4 (r mod 64), single table 4 (r mod 64) + 2h.
-PW_HD uint32_t pair_row_byte(uint32_t r) { return 4u * (r & 63u); }
+// Row words: pair table 4 (r mod 64) (+ h << 8 for b = 4), single table
+// 4 (r mod 64) + 2h.
+PW_HD uint32_t pair_row_byte(uint32_t r, int b) {
+  return 4u * (r & 63u) | (b == 4 ? (r >> 6) << 8 : 0u);
+}
 PW_HD uint32_t single_row_byte(uint32_t r) { return 4u * (r & 63u) + 2u * (r >> 6); }
 
 // Byte offsets of table entries (for writing the tables).
 PW_HD uint32_t pair_offset(uint32_t v1, uint32_t v2, int b, uint32_t r) {
+  if (b == 4) return ((r >> 6) << 16) | (((v1 << 4) | v2) << 8) | 4u * (r & 63u);
   const uint32_t byte = (v1 << (b + 1)) | (v2 << 1) | (r >> 6);
-  return (byte << 8) | pair_row_byte(r);
+  return (byte << 8) | pair_row_byte(r, b);
 }
+// Bytes a pair table of bitwidth b spans.
+PW_HD constexpr uint32_t pair_table_bytes(int b) { return b == 4 ? (2u << 16) : (1u << 16); }
 PW_HD uint32_t single_offset(uint32_t v, uint32_t r) { return (v << 8) | single_row_byte(r); }
 
-// b <= 3.  Lds32(x) returns the 32-bit entry at byte offset x.
+// b <= 4.  Lds32(x) returns the 32-bit entry at byte offset x.
 template <int B, class Lds32>
 PW_HD void dq_word_pair(const uint32_t (&P)[B], uint32_t r, Lds32 lds32, uint32_t* out) {
-  static_assert(B >= 1 && B <= 3, "pair tables serve b = 1..3");
+  static_assert(B >= 1 && B <= 4, "pair tables serve b = 1..4");
   uint32_t X[8];
-  // byte bit 0 = row half; bits 1..B = code of column c + 4 (moved down 4
-  // columns); bits B+1..2B = code of column c; plane 0 is the code's MSB
-  X[0] = (r >> 6) ? 0xFFFFFFFFu : 0u;
+  // b <= 3: byte bit 0 = row half; bits 1..B = code of column c + 4 (moved
+  // down 4 columns); bits B+1..2B = code of column c.  b = 4: bits 0..3 and
+  // 4..7 the two codes.  Plane 0 is the code's MSB.
+  constexpr int kH = B <= 3 ? 1 : 0;
+  if (kH) X[0] = (r >> 6) ? 0xFFFFFFFFu : 0u;
 #pragma unroll
   for (int j = 0; j < B; ++j) {
-    X[1 + j] = shr<4>(P[B - 1 - j]);
-    X[1 + B + j] = P[B - 1 - j];
+    X[kH + j] = shr<4>(P[B - 1 - j]);
+    X[kH + B + j] = P[B - 1 - j];
   }
 #pragma unroll
-  for (int p = 1 + 2 * B; p < 8; ++p) X[p] = 0u;
+  for (int p = kH + 2 * B; p < 8; ++p) X[p] = 0u;
   transpose8_lo(X);
-  const uint32_t rowb = pair_row_byte(r);
+  const uint32_t rowb = pair_row_byte(r, B);
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     // byte j of X[m]: columns 8j + m and 8j + m + 4

@@ -81,15 +81,16 @@ EncodeTiledFn encode_fn() {
 bool tc_shape_ok(int cols) { return cols % 128 == 0; }
 
 // Maps over an atom-major fp16 buffer [ld / 64][rows][64] for the token
-// tiles, as {64 columns, rows, atoms}: box i loads 8(i+1) rows x 4 atoms with
-// the 128-byte swizzle of the MMA's K-major operand, one copy per stage.
+// tiles, as {64 columns, rows, atoms}: box i loads 8(i+1) rows x 2 atoms with
+// the 128-byte swizzle of the MMA's K-major operand, one copy per 128-column
+// B stage.
 pw_status_t make_row_maps(CUtensorMap* m, const uint16_t* base, int ld, int rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(PW_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   for (int i = 0; i < 4; ++i) {
     cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(ld / 64)};
     cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(rows) * 128};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(8 * (i + 1)), 4};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(8 * (i + 1)), 2};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(&m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<uint16_t*>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

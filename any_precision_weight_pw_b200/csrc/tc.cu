@@ -70,24 +70,28 @@ constexpr int kDqThreads = 256;                // 8 dequantiser warps
 constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpLoader = 10;
 constexpr int kThreads = 15 * 32;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
-constexpr uint32_t kOffLut = 0;                // 256 code lines x 64 row words x 4 B
-constexpr uint32_t kLutBytes = 256u * 64u * 4u;
+constexpr uint32_t kOffLut = 0;                // table region (dequant.cuh gives its layout)
 
 // Two configurations of the kernel.
 //   decode  token tiles of up to 32 rows (MMA N = 16 or 32); one TMA box per
-//           256-column B stage; two accumulator buffers (gate and up side by
-//           side) so an item's epilogue overlaps the next item's MMAs.
+//           128-column B stage (one per A slot); two accumulator buffers (gate
+//           and up side by side) so an item's epilogue overlaps the next
+//           item's MMAs; a 128 KB table region, so 4-bit blocks take pair
+//           tables too.
 //   prefill 256-token chunks (MMA N = 256), so each dequantised weight tile
 //           serves 256 tokens; B stages of 64 columns (32 KB); one 256-column
-//           accumulator, so gate and up run as separate launches.
+//           accumulator, so gate and up run as separate launches; a 64 KB
+//           table region (pair tables up to 3 bits).
 // Shared memory offsets are compile-time (from a 1024-byte aligned base) so
 // table lookups fold the base into the loads' immediate offsets.
 template <bool PF>
 struct Cfg {
   static constexpr bool kPrefill = PF;
-  static constexpr int kNSlot = PF ? 16 : 20;  // plane slots
+  static constexpr int kNSlot = 16;            // plane slots
   static constexpr int kNT = PF ? kTcPfTokens : kTcTokens;
-  static constexpr int kBStageK = PF ? 64 : 256;
+  static constexpr int kPairMax = PF ? 3 : 4;   // widest bitwidth with a pair table
+  static constexpr uint32_t kLutBytes = dq::pair_table_bytes(kPairMax);
+  static constexpr int kBStageK = PF ? 64 : 128;
   static constexpr int kBStageBytes = kNT * kBStageK * 2;
   static constexpr int kBPerStage = 256 / kBStageK;
   static constexpr int kNB = PF ? 3 : 4;        // token-tile ring depth
@@ -494,7 +498,7 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad,
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t out[32];
-      if constexpr (B <= 3) {
+      if constexpr (B <= C::kPairMax) {
         dq::dq_word_pair<B>(P[2 * h], ru, lds32, out);
         dq::dq_word_pair<B>(P[2 * h + 1], ru, lds32, out + 16);
       } else {
@@ -511,18 +515,21 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad,
   return true;
 }
 
-// This thread's share of a pass's LUT.  b <= 3 goes to registers (both
-// threads of a row load the whole row), wider tables to shared memory, each of
-// the two threads of a row writing half of the words.  For b <= 6 the global
-// loads are issued one pass ahead (prefetch) and installed when the pass
-// starts, so their latency hides behind the previous pass; b = 7, 8 tables
-// load when the pass starts.
+// This thread's share of a pass's LUT.  Pair-table bitwidths (b <= 3, and
+// b = 4 in the decode configuration) keep the whole row in registers (both
+// threads of a row load it) and each thread writes the entries whose first
+// code lies in its half; wider tables go to shared memory as single entries,
+// each of the two threads of a row writing half of them.  For b <= 6 the
+// global loads are issued one pass ahead (prefetch) and installed when the
+// pass starts, so their latency hides behind the previous pass; b = 7, 8
+// tables load when the pass starts.
 struct LutPrefetch {
   uint4 v[4];
   int bits;
   bool live;  // this thread's row exists
 };
 
+template <class C>
 __device__ __forceinline__ void lut_prefetch(const Item& it, const Pass& ps, int grp, int r,
                                              LutPrefetch& f) {
   const int o = it.row0 + r;
@@ -540,32 +547,53 @@ __device__ __forceinline__ void lut_prefetch(const Item& it, const Pass& ps, int
     f.v[0] = make_uint4(w[0], w[1], w[2], w[3]);
     return;
   }
+  if (b <= C::kPairMax) {
+    const uint4* src = reinterpret_cast<const uint4*>(row);
+    f.v[0] = src[0];
+    f.v[1] = src[1];
+    return;
+  }
   const uint4* src = reinterpret_cast<const uint4*>(row + grp * (1 << (b - 1)));
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (i < (1 << (b - 4))) f.v[i] = src[i];
 }
 
+template <class C>
 __device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int grp, int r,
                                             const LutPrefetch& f) {
   if (!f.live) return;
   const int b = ps.bits;
   const uint32_t ru = static_cast<uint32_t>(r);
-  if (b <= 3) {
+  if (b <= C::kPairMax) {
     // pair table: entry (v1, v2) = (LUT[v1], LUT[v2]); this thread writes the
     // entries with v1 in its half of the codes
-    const uint64_t w01 = f.v[0].x | (static_cast<uint64_t>(f.v[0].y) << 32);
-    const uint64_t w23 = f.v[0].z | (static_cast<uint64_t>(f.v[0].w) << 32);
-    auto entry = [&](int v) -> uint32_t {
-      return static_cast<uint32_t>(((v < 4) ? w01 : w23) >> (16 * (v & 3))) & 0xFFFFu;
+    // (entries stay in registers: the second code runs over a compile-time
+    // range, the first is picked by selects and shifts)
+    const bool wide = b > 3;
+    const uint32_t w[8] = {f.v[0].x, f.v[0].y, f.v[0].z, f.v[0].w,
+                           wide ? f.v[1].x : 0u, wide ? f.v[1].y : 0u,
+                           wide ? f.v[1].z : 0u, wide ? f.v[1].w : 0u};
+    auto pick = [&](int v) -> uint32_t {
+      const uint4 q = (v & 8) ? f.v[1] : f.v[0];
+      const uint64_t x = (v & 4) ? (q.z | (static_cast<uint64_t>(q.w) << 32))
+                                 : (q.x | (static_cast<uint64_t>(q.y) << 32));
+      return static_cast<uint32_t>(x >> (16 * (v & 3))) & 0xFFFFu;
     };
     const int n = 1 << b, half = n >> 1;
-    for (int v1 = grp * half; v1 < grp * half + half; ++v1) {
-      const uint32_t lo = entry(v1);
-      for (int v2 = 0; v2 < n; ++v2) {
-        const uint32_t hi = entry(v2);
-        *reinterpret_cast<uint32_t*>(pw_tc_smem + kOffLut + dq::pair_offset(v1, v2, b, ru)) =
-            lo | (hi << 16);
+    // offsets are linear in v2: base + v2 * step
+    const uint32_t step = dq::pair_offset(0, 1, b, ru) - dq::pair_offset(0, 0, b, ru);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= half) break;
+      const int v1 = grp * half + i;
+      const uint32_t lo = pick(v1);
+      uint8_t* base = pw_tc_smem + kOffLut + dq::pair_offset(v1, 0, b, ru);
+#pragma unroll
+      for (int v2 = 0; v2 < 16; ++v2) {
+        if (v2 >= n) break;
+        const uint32_t hi = (w[v2 >> 1] >> (16 * (v2 & 1))) & 0xFFFFu;
+        *reinterpret_cast<uint32_t*>(base + v2 * step) = lo | (hi << 16);
       }
     }
     return;
@@ -601,10 +629,12 @@ __device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int 
 // Linear mode: the activations are bf16 in natural column order; convert,
 // permute into the A slots' K order and store (generic stores; the caller
 // fences).  Stage s, token rows 0..ntok-1, this lane's share.
-__device__ void fill_b_linear(const TcParams& p, const Item& it, int s, uint32_t buf, int lane) {
-  for (int idx = lane; idx < it.ntok * kStageWords; idx += 32) {
-    const int n = idx >> 3, w = idx & 7;
-    const int col0 = s * 256 + 32 * w;
+__device__ void fill_b_linear(const TcParams& p, const Item& it, int s, int j, uint32_t buf,
+                              int lane) {
+  // words 4j .. 4j + 3 of stage s (columns 256 s + 128 j ..)
+  for (int idx = lane; idx < it.ntok * 4; idx += 32) {
+    const int n = idx >> 2, w = idx & 3;
+    const int col0 = s * 256 + 128 * j + 32 * w;
     float v[32];
     if (col0 < it.cols) {  // cols is a multiple of 128: whole 32-column groups
       const uint4* src = reinterpret_cast<const uint4*>(
@@ -739,13 +769,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     LutPrefetch pre;
     if (i < total) {
       decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
-      lut_prefetch(it, get_pass(p, it, 0), grp, r, pre);
+      lut_prefetch<C>(it, get_pass(p, it, 0), grp, r, pre);
     }
     while (i < total && ok) {
       const Pass ps = get_pass(p, it, q);
       // every thread is done with the previous pass's table before it changes
       if (!dq_sync(dqbar, sync_phase, ctl)) break;
-      lut_install(it, ps, grp, r, pre);
+      lut_install<C>(it, ps, grp, r, pre);
       if (!dq_sync(dqbar, sync_phase, ctl)) break;
       const Item cur = it;
       int ni = i, nq = q + 1;
@@ -754,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         nq = 0;
         if (ni < total) decode_item<C>(p, s_prefix, s_prefix2, G, ni, it, gh);
       }
-      if (ni < total) lut_prefetch(it, get_pass(p, it, nq), grp, r, pre);
+      if (ni < total) lut_prefetch<C>(it, get_pass(p, it, nq), grp, r, pre);
       switch (ps.bits) {
         case 1: ok = dequant_stages<C, 1>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
         case 2: ok = dequant_stages<C, 2>(cur, grp, quad, sf, se, af, ae, tmem_base, st, ctl); break;
@@ -851,13 +881,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
                 tma_load_3d(buf, &p.pf_map, 0, it.pos0, 4 * s + j, &bfull[jb]);
               }
             } else if (p.mode == kTcLinear) {
-              fill_b_linear(p, it, s, buf, lane);
+              fill_b_linear(p, it, s, j, buf, lane);
               fence_proxy_async();
               mbar_arrive(&bfull[jb]);
             } else if (lane == 0) {
-              // {64 columns, rows_b rows, 4 atoms} starting at column 256 s
-              mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(rows_b) * 4u * 128u);
-              tma_load_3d(buf, &bmaps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s, &bfull[jb]);
+              // {64 columns, rows_b rows, 2 atoms} starting at column 256 s + 128 j
+              mbar_arrive_tx(&bfull[jb], static_cast<uint32_t>(rows_b) * 2u * 128u);
+              tma_load_3d(buf, &bmaps[(rows_b >> 3) - 1], 0, it.pos0, 4 * s + 2 * j, &bfull[jb]);
             }
             b_ctr++;
           }
@@ -943,40 +973,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
           const uint32_t dt = tmem_base + jd * C::kDColsPerBuf + 32 * q;
           uint32_t accum = 0;
           for (int s = it.s_begin; s < it.s_end && ok; ++s) {
-            const uint32_t jb = b_ctr % kNB;
-            if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + C::kOffB + jb * C::kBStageBytes));
+            // each 128-column half of the stage: one B stage, one A slot
             for (int sub = 0; sub < 2; ++sub) {
+              const uint32_t jb = b_ctr % kNB;
+              if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+                ok = false;
+                break;
+              }
               const uint32_t qa = a_ctr % kNA;
               if (!mbar_wait_warp(&af[qa], (a_ctr / kNA) & 1u, ctl)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
+              const uint64_t bdesc =
+                  smem_desc_sw128(smem_addr(smem + C::kOffB + jb * C::kBStageBytes));
               const uint32_t at = tmem_base + C::kAColBase + qa * kAColsPerSlot;
               if (leader) {
-                // K step kk of this 128-column half: atom 2 sub + kk / 4, 32 bytes
-                // per 16 columns inside the atom
+                // K step kk: atom kk / 4 of the B stage, 32 bytes per 16
+                // columns inside the atom
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                  const uint64_t bd =
-                      bdesc + (2u * sub + (kk >> 2)) * atom_step + 2u * (kk & 3);
+                  const uint64_t bd = bdesc + (kk >> 2) * atom_step + 2u * (kk & 3);
                   tc_mma(dt, at + kk * 8, bd, idesc, accum | kk);
                 }
                 tc_commit(&ae[qa]);
+                tc_commit(&bempty[jb]);
               }
               __syncwarp();
               accum = 1;
               a_ctr++;
+              b_ctr++;
             }
-            if (!ok) break;
-            if (leader) tc_commit(&bempty[jb]);
-            __syncwarp();
-            b_ctr++;
           }
         }
         if (!ok) break;

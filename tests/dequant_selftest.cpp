@@ -19,10 +19,12 @@ static int code_of(const uint32_t* P, int B, int c) {
   return v;
 }
 
-template <int B>
+// PAIR: take the pair table (b <= 4) rather than the single one (b >= 4).
+template <int B, bool PAIR>
 static int check(std::mt19937& rng) {
   int bad = 0;
-  std::vector<uint8_t> region(1u << 16, 0);  // emulated 64 KB shared-memory table
+  // emulated shared-memory table: 64 KB, 128 KB for the b = 4 pair table
+  std::vector<uint8_t> region(PAIR ? pair_table_bytes(B) : (1u << 16), 0);
   for (int trial = 0; trial < 2000; ++trial) {
     const uint32_t r = rng() % 128;
     uint32_t P[B];
@@ -43,10 +45,11 @@ static int check(std::mt19937& rng) {
       return region[x] | (region[x + 1] << 8);
     };
     uint32_t out[16];
-    if constexpr (B <= 3) {
+    if constexpr (PAIR) {
       for (int v1 = 0; v1 < (1 << B); ++v1)
         for (int v2 = 0; v2 < (1 << B); ++v2) {
           const uint32_t off = pair_offset(v1, v2, B, r);
+          if (off % 4) { std::printf("pair entry not word aligned\n"); return 1; }
           if (!put16(off, lut[v1]) || !put16(off + 2, lut[v2])) { std::printf("offset out of range\n"); return 1; }
         }
       auto lds32 = [&](uint32_t x) -> uint32_t { return get16(x) | (get16(x + 2) << 16); };
@@ -96,14 +99,35 @@ static int check_layout() {
       bank[bk] = true;
     }
   }
+  // b = 4 pair table: every (v1, v2, r) has its own word, and a warp's 32 rows
+  // hit 32 banks
+  {
+    std::vector<uint8_t> seen(pair_table_bytes(4) / 4, 0);
+    for (uint32_t v1 = 0; v1 < 16; ++v1)
+      for (uint32_t v2 = 0; v2 < 16; ++v2)
+        for (uint32_t r = 0; r < 128; ++r) {
+          const uint32_t w = pair_offset(v1, v2, 4, r) / 4;
+          if (w >= seen.size() || seen[w]) ++bad;
+          else seen[w] = 1;
+        }
+    for (uint32_t q = 0; q < 4; ++q) {
+      bool bank[32] = {};
+      for (uint32_t l = 0; l < 32; ++l) {
+        const uint32_t bk = (pair_offset(l % 7, l % 11, 4, 32 * q + l) / 4) % 32;
+        if (bank[bk]) ++bad;
+        bank[bk] = true;
+      }
+    }
+  }
   if (bad) std::printf("layout: %d problems\n", bad);
   return bad;
 }
 
 int main() {
   std::mt19937 rng(12345);
-  int bad = check<1>(rng) + check<2>(rng) + check<3>(rng) + check<4>(rng) + check<5>(rng) +
-            check<6>(rng) + check<7>(rng) + check<8>(rng) + check_layout();
+  int bad = check<1, true>(rng) + check<2, true>(rng) + check<3, true>(rng) +
+            check<4, true>(rng) + check<4, false>(rng) + check<5, false>(rng) +
+            check<6, false>(rng) + check<7, false>(rng) + check<8, false>(rng) + check_layout();
   std::printf(bad ? "FAIL %d\n" : "ok\n", bad);
   return bad ? 1 : 0;
 }
