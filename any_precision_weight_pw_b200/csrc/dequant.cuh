@@ -13,22 +13,28 @@
 // Codes come from an 8x8 bit-matrix transpose of plane words: input row p
 // becomes bit p of every byte, so byte n of output row q collects column
 // 8n + q.  The byte then IS an address byte: one byte permute (PRMT) puts it
-// next to the thread's row byte, and one shared-memory load fetches the
-// entry.  Two tables, both for 128 local rows (threads):
-//   pair     b <= 4: the 32-bit entry for codes v1 (column c) and v2 (column
-//            c + 4) is the fp16 pair (LUT[v1], LUT[v2]) -- one load gives one
-//            output register.  For b <= 3 the byte holds
-//            (v1 << (b + 1)) | (v2 << 1) | h with the row half h = r >= 64,
-//            and the entry sits at byte (byte << 8) | 4 (r mod 64) (<= 64 KB);
-//            for b = 4 the byte is (v1 << 4) | v2 and h moves to the third
-//            address byte: (h << 16) | (byte << 8) | 4 (r mod 64) (128 KB).
-//   single   b >= 4: the byte holds v; the fp16 entry of row r is at
-//            byte (v << 8) | 4 (r mod 64) | 2h (rows r and r + 64 share a
-//            word, 64 KB).  Two loads and one multiply-add give one output
+// next to the thread's row bytes, and one shared-memory load fetches the
+// entry.  Two kinds of table serve 128 local rows (threads):
+//   pair     the 32-bit entry for codes v1 (column c) and v2 (column c + 4) is
+//            the fp16 pair (LUT[v1], LUT[v2]) -- one load gives one output
 //            register.
-// In both the 32 threads of a warp (32 consecutive rows) read 32 different
-// banks.  Shifts are written as multiplies (left) and high multiplies (right)
-// so they issue on the FMA pipe; the ALU pipe keeps the LOP3 and PRMT work.
+//   single   the fp16 entry for code v; two loads and one multiply-add give
+//            one output register.
+// and two layouts of them (h = r >= 64 is the row half):
+//   split    (128 KB region) pair tables for b <= 4, single for b >= 5.  The
+//            address is (h << 16) | (byte << 8) | 4 (r mod 64), with byte =
+//            (v1 << b) | v2 (pair) or v (single, entry in the low half of the
+//            word).  Every row owns its words in every table, so the threads
+//            of one row need not wait for any other row's threads when the
+//            table changes.
+//   packed   (64 KB region) pair tables for b <= 3 with byte =
+//            (v1 << (b + 1)) | (v2 << 1) | h at (byte << 8) | 4 (r mod 64);
+//            single tables for b >= 4 at (v << 8) | 4 (r mod 64) | 2h (rows r
+//            and r + 64 share a word).
+// In all of them the 32 threads of a warp (32 consecutive rows) read 32
+// different banks.  Shifts are written as multiplies (left) and high multiplies
+// (right) so they issue on the FMA pipe; the ALU pipe keeps the LOP3 and PRMT
+// work.
 //
 // Everything here is __host__ __device__ so the bit manipulation can be
 // checked on the CPU (tests/dequant_selftest.cpp) against a plain unpack.
@@ -118,39 +124,45 @@ PW_HD void transpose8_lo(uint32_t (&X)[8]) {
 }
 
 // Address of the entry for byte N of x: byte 0 = byte 0 of rowb (the row
-// byte), byte 1 = byte N of x, byte 2 = byte 1 of rowb (the row half for b = 4
-// pair tables, else zero), byte 3 = byte 2 of rowb (zero).
+// byte), byte 1 = byte N of x, byte 2 = byte 1 of rowb (the row half in the
+// split layout, else zero), byte 3 = byte 2 of rowb (zero).
 template <int N>
 PW_HD uint32_t code_addr(uint32_t x, uint32_t rowb) {
   return prmt(x, rowb, 0x6504u | (static_cast<uint32_t>(N) << 4));
 }
 
-// Row words: pair table 4 (r mod 64) (+ h << 8 for b = 4), single table
-// 4 (r mod 64) + 2h.
-PW_HD uint32_t pair_row_byte(uint32_t r, int b) {
-  return 4u * (r & 63u) | (b == 4 ? (r >> 6) << 8 : 0u);
+// Widest bitwidth served by a pair table.
+PW_HD constexpr int pair_max(bool split) { return split ? 4 : 3; }
+// Bytes a layout's tables span.
+PW_HD constexpr uint32_t table_bytes(bool split) { return split ? (2u << 16) : (1u << 16); }
+
+// Row words (bytes 0-1 of every address of row r).
+PW_HD uint32_t pair_row_byte(uint32_t r, bool split) {
+  return split ? (4u * (r & 63u) | ((r >> 6) << 8)) : 4u * (r & 63u);
 }
-PW_HD uint32_t single_row_byte(uint32_t r) { return 4u * (r & 63u) + 2u * (r >> 6); }
+PW_HD uint32_t single_row_byte(uint32_t r, bool split) {
+  return split ? (4u * (r & 63u) | ((r >> 6) << 8)) : 4u * (r & 63u) + 2u * (r >> 6);
+}
 
 // Byte offsets of table entries (for writing the tables).
-PW_HD uint32_t pair_offset(uint32_t v1, uint32_t v2, int b, uint32_t r) {
-  if (b == 4) return ((r >> 6) << 16) | (((v1 << 4) | v2) << 8) | 4u * (r & 63u);
+PW_HD uint32_t pair_offset(uint32_t v1, uint32_t v2, int b, uint32_t r, bool split) {
+  if (split) return ((r >> 6) << 16) | (((v1 << b) | v2) << 8) | 4u * (r & 63u);
   const uint32_t byte = (v1 << (b + 1)) | (v2 << 1) | (r >> 6);
-  return (byte << 8) | pair_row_byte(r, b);
+  return (byte << 8) | 4u * (r & 63u);
 }
-// Bytes a pair table of bitwidth b spans.
-PW_HD constexpr uint32_t pair_table_bytes(int b) { return b == 4 ? (2u << 16) : (1u << 16); }
-PW_HD uint32_t single_offset(uint32_t v, uint32_t r) { return (v << 8) | single_row_byte(r); }
+PW_HD uint32_t single_offset(uint32_t v, uint32_t r, bool split) {
+  return split ? ((r >> 6) << 16) | (v << 8) | 4u * (r & 63u) : (v << 8) | single_row_byte(r, false);
+}
 
-// b <= 4.  Lds32(x) returns the 32-bit entry at byte offset x.
-template <int B, class Lds32>
+// Pair-table bitwidths.  Lds32(x) returns the 32-bit entry at byte offset x.
+template <int B, bool SPLIT, class Lds32>
 PW_HD void dq_word_pair(const uint32_t (&P)[B], uint32_t r, Lds32 lds32, uint32_t* out) {
-  static_assert(B >= 1 && B <= 4, "pair tables serve b = 1..4");
+  static_assert(B >= 1 && B <= pair_max(SPLIT), "pair tables serve b = 1..3 (packed), 1..4 (split)");
   uint32_t X[8];
-  // b <= 3: byte bit 0 = row half; bits 1..B = code of column c + 4 (moved
-  // down 4 columns); bits B+1..2B = code of column c.  b = 4: bits 0..3 and
-  // 4..7 the two codes.  Plane 0 is the code's MSB.
-  constexpr int kH = B <= 3 ? 1 : 0;
+  // byte bits kH..kH+B-1 = code of column c + 4 (moved down 4 columns), bits
+  // kH+B..kH+2B-1 = code of column c; packed layout: bit 0 = row half.
+  // Plane 0 is the code's MSB.
+  constexpr int kH = SPLIT ? 0 : 1;
   if (kH) X[0] = (r >> 6) ? 0xFFFFFFFFu : 0u;
 #pragma unroll
   for (int j = 0; j < B; ++j) {
@@ -160,7 +172,7 @@ PW_HD void dq_word_pair(const uint32_t (&P)[B], uint32_t r, Lds32 lds32, uint32_
 #pragma unroll
   for (int p = kH + 2 * B; p < 8; ++p) X[p] = 0u;
   transpose8_lo(X);
-  const uint32_t rowb = pair_row_byte(r, B);
+  const uint32_t rowb = pair_row_byte(r, SPLIT);
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     // byte j of X[m]: columns 8j + m and 8j + m + 4
@@ -171,16 +183,16 @@ PW_HD void dq_word_pair(const uint32_t (&P)[B], uint32_t r, Lds32 lds32, uint32_
   }
 }
 
-// b >= 4.  Lds16(x) returns the 16-bit entry at byte offset x.
-template <int B, class Lds16>
+// Single-table bitwidths.  Lds16(x) returns the 16-bit entry at byte offset x.
+template <int B, bool SPLIT, class Lds16>
 PW_HD void dq_word_single(const uint32_t (&P)[B], uint32_t r, Lds16 lds16, uint32_t* out) {
-  static_assert(B >= 4 && B <= 8, "single tables serve b = 4..8");
+  static_assert(B > pair_max(SPLIT) && B <= 8, "single tables serve the wider bitwidths");
   uint32_t X[8];
   // byte bit p = code bit p (right-aligned code); plane 0 is the MSB
 #pragma unroll
   for (int p = 0; p < 8; ++p) X[p] = (p < B) ? P[(p < B) ? B - 1 - p : 0] : 0u;
   transpose8(X);
-  const uint32_t rowb = single_row_byte(r);
+  const uint32_t rowb = single_row_byte(r, SPLIT);
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     // columns 8j + m (X[m] byte j) and 8j + m + 4 (X[m + 4] byte j)

@@ -89,8 +89,10 @@ struct Cfg {
   static constexpr bool kPrefill = PF;
   static constexpr int kNSlot = 16;            // plane slots
   static constexpr int kNT = PF ? kTcPfTokens : kTcTokens;
-  static constexpr int kPairMax = PF ? 3 : 4;   // widest bitwidth with a pair table
-  static constexpr uint32_t kLutBytes = dq::pair_table_bytes(kPairMax);
+  // table layout (dequant.cuh): split (rows own their words, 128 KB) or packed
+  static constexpr bool kSplitRows = !PF;
+  static constexpr int kPairMax = dq::pair_max(kSplitRows);  // widest pair-table bitwidth
+  static constexpr uint32_t kLutBytes = dq::table_bytes(kSplitRows);
   static constexpr int kBStageK = PF ? 64 : 128;
   static constexpr int kBStageBytes = kNT * kBStageK * 2;
   static constexpr int kBPerStage = 256 / kBStageK;
@@ -102,7 +104,7 @@ struct Cfg {
   static constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
   static constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
   static constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
-  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 2 * kNDBuf + 2;
+  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 2 * kNDBuf + 1 + 4;
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
   static constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 8 * (kMaxGroups + 2);
   static constexpr uint32_t kSmemTotal = kOffSlotUser + 4 * kNSlot;
@@ -447,8 +449,8 @@ __device__ __forceinline__ uint4 read_plane_chunk(uint32_t slot_off, int r, int 
   return *reinterpret_cast<const uint4*>(pw_tc_smem + off);
 }
 
-// All dequantiser threads meet (a bounded wait, unlike a hardware barrier,
-// so a warp that gave up cannot leave the others blocked).
+// The dequantiser warps counted by `bar` meet (a bounded wait, unlike a
+// hardware barrier, so a warp that gave up cannot leave the others blocked).
 __device__ __forceinline__ bool dq_sync(uint64_t* bar, uint32_t& phase, const Ctl& ctl) {
   mbar_arrive_warp(bar);
   const bool ok = mbar_wait_warp(bar, phase, ctl);
@@ -499,11 +501,11 @@ __device__ bool dequant_stages(const Item& it, int grp, int quad,
     for (int h = 0; h < 2; ++h) {
       uint32_t out[32];
       if constexpr (B <= C::kPairMax) {
-        dq::dq_word_pair<B>(P[2 * h], ru, lds32, out);
-        dq::dq_word_pair<B>(P[2 * h + 1], ru, lds32, out + 16);
+        dq::dq_word_pair<B, C::kSplitRows>(P[2 * h], ru, lds32, out);
+        dq::dq_word_pair<B, C::kSplitRows>(P[2 * h + 1], ru, lds32, out + 16);
       } else {
-        dq::dq_word_single<B>(P[2 * h], ru, lds16, out);
-        dq::dq_word_single<B>(P[2 * h + 1], ru, lds16, out + 16);
+        dq::dq_word_single<B, C::kSplitRows>(P[2 * h], ru, lds16, out);
+        dq::dq_word_single<B, C::kSplitRows>(P[2 * h + 1], ru, lds16, out + 16);
       }
       tmem_st32(tcol + 32 * h, out);
     }
@@ -582,13 +584,14 @@ __device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int 
     };
     const int n = 1 << b, half = n >> 1;
     // offsets are linear in v2: base + v2 * step
-    const uint32_t step = dq::pair_offset(0, 1, b, ru) - dq::pair_offset(0, 0, b, ru);
+    const uint32_t step = dq::pair_offset(0, 1, b, ru, C::kSplitRows) -
+                          dq::pair_offset(0, 0, b, ru, C::kSplitRows);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (i >= half) break;
       const int v1 = grp * half + i;
       const uint32_t lo = pick(v1);
-      uint8_t* base = pw_tc_smem + kOffLut + dq::pair_offset(v1, 0, b, ru);
+      uint8_t* base = pw_tc_smem + kOffLut + dq::pair_offset(v1, 0, b, ru, C::kSplitRows);
 #pragma unroll
       for (int v2 = 0; v2 < 16; ++v2) {
         if (v2 >= n) break;
@@ -598,10 +601,10 @@ __device__ __forceinline__ void lut_install(const Item& it, const Pass& ps, int 
     }
     return;
   }
-  // single table: entry v of row r at dq::single_offset(v, r); this thread
+  // single table: entry v of row r at dq::single_offset(v, r, .); this thread
   // writes entries grp * half .. grp * half + half - 1
   auto put = [&](int v, uint32_t e) {
-    *reinterpret_cast<uint16_t*>(pw_tc_smem + kOffLut + dq::single_offset(v, ru)) =
+    *reinterpret_cast<uint16_t*>(pw_tc_smem + kOffLut + dq::single_offset(v, ru, C::kSplitRows)) =
         static_cast<uint16_t>(e);
   };
   const int half = 1 << (b - 1);
@@ -682,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   uint64_t* df = ae + kNA;
   uint64_t* de = df + kNDBuf;
   uint64_t* drain = de + kNDBuf;
-  uint64_t* dqbar = drain + 1;
+  uint64_t* dqbar = drain + 1;  // table syncs: [4] (split layout: one per row quarter)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_prefix = reinterpret_cast<int*>(smem + C::kOffMisc + 16);
@@ -711,7 +714,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       mbar_init(&ae[i], 1);
     }
     mbar_init(drain, 1);
-    mbar_init(dqbar, kDqThreads / 32);
+    // split layout: the two warps of a row quarter (K halves) share its
+    // tables; packed layout: all dequantisers
+    for (int i = 0; i < 4; ++i) mbar_init(&dqbar[i], C::kSplitRows ? 2 : kDqThreads / 32);
     for (int k = 0; k < C::kNSlot; ++k) slot_user[k] = 0u;
     // the table offsets assume a 1024-byte aligned dynamic shared memory base
     *s_abort = (smem_addr(smem) & 1023u) ? 1 : 0;
@@ -760,6 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     int gh[2] = {0, 0};
     const int grp = warp >> 2, quad = warp & 3;
     const int r = 32 * quad + lane;
+    // split layout: a row quarter's tables are touched only by its two warps,
+    // so they alone meet around a table change
+    uint64_t* tbar = C::kSplitRows ? &dqbar[quad] : dqbar;
     uint32_t sync_phase = 0;
     bool ok = true;
     // walk (item, pass) pairs; the next pass's LUT loads are issued before
@@ -773,10 +781,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     }
     while (i < total && ok) {
       const Pass ps = get_pass(p, it, q);
-      // every thread is done with the previous pass's table before it changes
-      if (!dq_sync(dqbar, sync_phase, ctl)) break;
+      // every reader of these rows' tables is done with the previous pass's
+      // table before it changes
+      if (!dq_sync(tbar, sync_phase, ctl)) break;
       lut_install<C>(it, ps, grp, r, pre);
-      if (!dq_sync(dqbar, sync_phase, ctl)) break;
+      if (!dq_sync(tbar, sync_phase, ctl)) break;
       const Item cur = it;
       int ni = i, nq = q + 1;
       if (nq >= it.npass) {

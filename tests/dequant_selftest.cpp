@@ -1,7 +1,9 @@
 // CPU check of the kernel's per-thread dequantisation routines
 // (any_precision_weight_pw_b200/csrc/dequant.cuh) against a plain unpack:
-// for every bitwidth, random planes and LUTs, every output half must equal
-// LUT[code] of the column the K order assigns to it.  Exit status 0 = pass.
+// for every bitwidth and both table layouts, random planes and LUTs, every
+// output half must equal LUT[code] of the column the K order assigns to it.
+// The layout checks cover bank spread and, for the split layout, that every
+// row's table words are its own in every format.  Exit status 0 = pass.
 #include <cstdio>
 #include <cstdlib>
 #include <algorithm>
@@ -19,12 +21,11 @@ static int code_of(const uint32_t* P, int B, int c) {
   return v;
 }
 
-// PAIR: take the pair table (b <= 4) rather than the single one (b >= 4).
-template <int B, bool PAIR>
+template <int B, bool SPLIT>
 static int check(std::mt19937& rng) {
+  constexpr bool kPair = B <= pair_max(SPLIT);
   int bad = 0;
-  // emulated shared-memory table: 64 KB, 128 KB for the b = 4 pair table
-  std::vector<uint8_t> region(PAIR ? pair_table_bytes(B) : (1u << 16), 0);
+  std::vector<uint8_t> region(table_bytes(SPLIT), 0);  // emulated shared-memory table region
   for (int trial = 0; trial < 2000; ++trial) {
     const uint32_t r = rng() % 128;
     uint32_t P[B];
@@ -45,26 +46,26 @@ static int check(std::mt19937& rng) {
       return region[x] | (region[x + 1] << 8);
     };
     uint32_t out[16];
-    if constexpr (PAIR) {
+    if constexpr (kPair) {
       for (int v1 = 0; v1 < (1 << B); ++v1)
         for (int v2 = 0; v2 < (1 << B); ++v2) {
-          const uint32_t off = pair_offset(v1, v2, B, r);
+          const uint32_t off = pair_offset(v1, v2, B, r, SPLIT);
           if (off % 4) { std::printf("pair entry not word aligned\n"); return 1; }
           if (!put16(off, lut[v1]) || !put16(off + 2, lut[v2])) { std::printf("offset out of range\n"); return 1; }
         }
       auto lds32 = [&](uint32_t x) -> uint32_t { return get16(x) | (get16(x + 2) << 16); };
-      dq_word_pair<B>(P, r, lds32, out);
+      dq_word_pair<B, SPLIT>(P, r, lds32, out);
     } else {
       for (int v = 0; v < (1 << B); ++v)
-        if (!put16(single_offset(v, r), lut[v])) { std::printf("offset out of range\n"); return 1; }
-      dq_word_single<B>(P, r, get16, out);
+        if (!put16(single_offset(v, r, SPLIT), lut[v])) { std::printf("offset out of range\n"); return 1; }
+      dq_word_single<B, SPLIT>(P, r, get16, out);
     }
     for (int pr = 0; pr < 16; ++pr) {
       const int m = pr >> 2, j = pr & 3;
       const int c0 = 8 * j + m, c1 = c0 + 4;
       const uint32_t want = lut[code_of(P, B, c0)] | (static_cast<uint32_t>(lut[code_of(P, B, c1)]) << 16);
       if (out[pr] != want) {
-        if (bad < 5) std::printf("b=%d trial %d pair %d: got %08x want %08x\n", B, trial, pr, out[pr], want);
+        if (bad < 5) std::printf("b=%d split=%d trial %d pair %d: got %08x want %08x\n", B, SPLIT, trial, pr, out[pr], want);
         ++bad;
       }
     }
@@ -72,62 +73,67 @@ static int check(std::mt19937& rng) {
   return bad;
 }
 
-// The tables of all rows of a warp-quarter: distinct rows never share a
-// 2-byte entry, and the 32 rows of a warp address 32 different banks.
-static int check_layout() {
+// Byte offsets of every entry of row r's table for bitwidth b (2 bytes each).
+static std::vector<uint32_t> entries(int b, uint32_t r, bool split) {
+  std::vector<uint32_t> o;
+  if (b <= pair_max(split)) {
+    for (uint32_t v1 = 0; v1 < (1u << b); ++v1)
+      for (uint32_t v2 = 0; v2 < (1u << b); ++v2) {
+        o.push_back(pair_offset(v1, v2, b, r, split));
+        o.push_back(pair_offset(v1, v2, b, r, split) + 2);
+      }
+  } else {
+    for (uint32_t v = 0; v < (1u << b); ++v) o.push_back(single_offset(v, r, split));
+  }
+  return o;
+}
+
+static int check_layout(bool split) {
   int bad = 0;
-  for (int b = 4; b <= 8; ++b)
-    for (uint32_t v = 0; v < (1u << b); ++v)
-      for (uint32_t r = 0; r < 128; ++r)
-        for (uint32_t r2 = r + 1; r2 < 128; ++r2)
-          if (single_offset(v, r) == single_offset(v, r2)) ++bad;
-  for (uint32_t q = 0; q < 4; ++q) {
-    bool bank[32] = {};
-    for (uint32_t l = 0; l < 32; ++l) {
-      const uint32_t r = 32 * q + l;
-      const uint32_t bk = (single_offset(l % 7, r) / 4) % 32;  // any codes
-      if (bank[bk]) ++bad;
-      bank[bk] = true;
-    }
-  }
-  for (uint32_t q = 0; q < 4; ++q) {
-    bool bank[32] = {};
-    for (uint32_t l = 0; l < 32; ++l) {
-      const uint32_t r = 32 * q + l;
-      const uint32_t bk = (pair_offset(l % 5, l % 3, 3, r) / 4) % 32;
-      if (bank[bk]) ++bad;
-      bank[bk] = true;
-    }
-  }
-  // b = 4 pair table: every (v1, v2, r) has its own word, and a warp's 32 rows
-  // hit 32 banks
-  {
-    std::vector<uint8_t> seen(pair_table_bytes(4) / 4, 0);
-    for (uint32_t v1 = 0; v1 < 16; ++v1)
-      for (uint32_t v2 = 0; v2 < 16; ++v2)
-        for (uint32_t r = 0; r < 128; ++r) {
-          const uint32_t w = pair_offset(v1, v2, 4, r) / 4;
-          if (w >= seen.size() || seen[w]) ++bad;
-          else seen[w] = 1;
-        }
+  for (int b = 1; b <= 8; ++b) {
+    // distinct rows never share a 2-byte entry, and every entry is in range
+    std::vector<int> owner(table_bytes(split) / 2, -1);
+    for (uint32_t r = 0; r < 128; ++r)
+      for (uint32_t off : entries(b, r, split)) {
+        if (off + 2 > table_bytes(split)) { ++bad; continue; }
+        if (owner[off / 2] >= 0 && owner[off / 2] != static_cast<int>(r)) ++bad;
+        owner[off / 2] = static_cast<int>(r);
+      }
+    // the 32 rows of a warp read 32 different banks, whatever their codes
     for (uint32_t q = 0; q < 4; ++q) {
       bool bank[32] = {};
       for (uint32_t l = 0; l < 32; ++l) {
-        const uint32_t bk = (pair_offset(l % 7, l % 11, 4, 32 * q + l) / 4) % 32;
+        const uint32_t r = 32 * q + l;
+        const uint32_t v1 = (l * 7) % (1u << b), v2 = (l * 5 + 3) % (1u << b);
+        const uint32_t off = b <= pair_max(split) ? pair_offset(v1, v2, b, r, split)
+                                                  : single_offset(v1, r, split);
+        const uint32_t bk = (off / 4) % 32;
         if (bank[bk]) ++bad;
         bank[bk] = true;
       }
     }
   }
-  if (bad) std::printf("layout: %d problems\n", bad);
+  if (split) {
+    // every 4-byte word of row r's tables, in every format, encodes r: row
+    // half in bit 14 of the word index, r mod 64 in bits 0-5
+    for (int b = 1; b <= 8; ++b)
+      for (uint32_t r = 0; r < 128; ++r)
+        for (uint32_t off : entries(b, r, true)) {
+          const uint32_t w = off / 4;
+          if ((((w >> 14) & 1u) << 6 | (w & 63u)) != r) ++bad;
+        }
+  }
+  if (bad) std::printf("layout (split=%d): %d problems\n", split, bad);
   return bad;
 }
 
 int main() {
   std::mt19937 rng(12345);
-  int bad = check<1, true>(rng) + check<2, true>(rng) + check<3, true>(rng) +
-            check<4, true>(rng) + check<4, false>(rng) + check<5, false>(rng) +
-            check<6, false>(rng) + check<7, false>(rng) + check<8, false>(rng) + check_layout();
+  int bad = check<1, false>(rng) + check<2, false>(rng) + check<3, false>(rng) + check<4, false>(rng) +
+            check<5, false>(rng) + check<6, false>(rng) + check<7, false>(rng) + check<8, false>(rng);
+  bad += check<1, true>(rng) + check<2, true>(rng) + check<3, true>(rng) + check<4, true>(rng) +
+         check<5, true>(rng) + check<6, true>(rng) + check<7, true>(rng) + check<8, true>(rng);
+  bad += check_layout(false) + check_layout(true);
   std::printf(bad ? "FAIL %d\n" : "ok\n", bad);
   return bad ? 1 : 0;
 }
