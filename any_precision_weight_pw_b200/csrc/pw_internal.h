@@ -9,6 +9,33 @@
 
 namespace pw {
 
+// Programmatic dependent launch.  The forward's kernels go on the stream with
+// the programmatic-serialisation attribute, so each can be scheduled while
+// its predecessor drains; every such kernel calls pdl_wait() before it reads
+// anything a predecessor wrote (or writes anything a predecessor reads), and
+// may call pdl_trigger() to let its own successor be scheduled early.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+#endif
+
 constexpr int kMaxBlocks = 3 * (PW_MAX_EXPERTS + 1);
 constexpr int kMaxGroups = PW_MAX_EXPERTS + 1;  // routed experts + shared
 

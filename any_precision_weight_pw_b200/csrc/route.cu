@@ -37,6 +37,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   const int warps_per_block = kRouteThreads / 32;
   const int E = p.E, H = p.H, T = p.T, k = p.k;
   const RouteWorkspace& ws = p.ws;
+  // the previous kernel on the stream may produce x and still read the
+  // workspace; the gather kernel may be scheduled from here on
+  pdl_wait();
+  pdl_trigger();
 
   const int total_pairs = T * E;
   for (int pair = blockIdx.x * warps_per_block + warp; pair < total_pairs;
@@ -46,18 +50,41 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
     const uint16_t* xr = p.x + static_cast<size_t>(t) * H;
     const float* wr = p.wr + static_cast<size_t>(e) * H;
     // loads in batches of 32 per lane (independent of the sum, so their
-    // latencies overlap); the fused multiply-adds stay in ascending i
+    // latencies overlap), the next batch issued before the current one is
+    // summed; the fused multiply-adds stay in ascending i
     float s = 0.0f;
     int i0 = lane;
-    for (; i0 + 32 * 31 < H; i0 += 32 * 32) {
-      float xv[32], wv[32];
+    float xv[32], wv[32];
+    bool have = i0 + 32 * 31 < H;
+    if (have) {
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
         xv[u] = bf16_bits_to_f32(xr[i0 + 32 * u]);
         wv[u] = wr[i0 + 32 * u];
       }
+    }
+    while (have) {
+      const int i1 = i0 + 32 * 32;
+      const bool more = i1 + 32 * 31 < H;
+      float xn[32], wn[32];
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          xn[u] = bf16_bits_to_f32(xr[i1 + 32 * u]);
+          wn[u] = wr[i1 + 32 * u];
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 32; ++u) s = __fmaf_rn(xv[u], wv[u], s);
+      i0 = i1;
+      have = more;
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          xv[u] = xn[u];
+          wv[u] = wn[u];
+        }
+      }
     }
     for (int i = i0; i < H; i += 32) s = __fmaf_rn(bf16_bits_to_f32(xr[i]), wr[i], s);
 #pragma unroll
@@ -208,6 +235,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
 // Stored atom-major, [ld / 64][rows][64], so one 3-D copy fetches a stage.
 // One 32-column group per thread.
 __global__ void gather_kernel(const GatherParams p) {
+  pdl_wait();
+  pdl_trigger();  // the tensor-core kernel may be scheduled (it waits for this grid)
   const int P = p.offsets[p.n_groups];
   const int wpr = p.H >> 5;
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < P * wpr;
@@ -245,6 +274,8 @@ __global__ void gather_kernel(const GatherParams p) {
 // out[t] = sum_j ysorted[pos(t, j)] (+ shared) in slot order, summing the
 // split-K partials of each position in split order; fp32, rounded to bf16.
 __global__ void combine_kernel(const CombineParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.y;
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (c >= p.H) return;
@@ -277,8 +308,7 @@ cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s) {
   int grid = (pairs + warps - 1) / warps;
   if (grid > 4 * n_sm) grid = 4 * n_sm;
   if (grid < 1) grid = 1;
-  route_kernel<<<grid, kRouteThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel, dim3(grid), dim3(kRouteThreads), 0, s, p);
 }
 
 cudaError_t launch_gather(const GatherParams& p, int max_rows, int n_sm, cudaStream_t s) {
@@ -286,15 +316,13 @@ cudaError_t launch_gather(const GatherParams& p, int max_rows, int n_sm, cudaStr
   int grid = (max_rows * (p.H >> 5) + threads - 1) / threads;
   if (grid > 4 * n_sm) grid = 4 * n_sm;
   if (grid < 1) grid = 1;
-  gather_kernel<<<grid, threads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gather_kernel, dim3(grid), dim3(threads), 0, s, p);
 }
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
   const int threads = 128;
   dim3 grid((p.H / 4 + threads - 1) / threads, p.T);
-  combine_kernel<<<grid, threads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, grid, dim3(threads), 0, s, p);
 }
 
 }  // namespace pw

@@ -695,6 +695,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = (p.mode == kTcLinear) ? 1 : p.n_groups;
+  // everything below reads what earlier kernels of the forward wrote (or
+  // writes what they read); the successor is not released early, so it
+  // cannot take SM resources while the grid's CTAs wait on one another
+  pdl_wait();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {
@@ -1185,8 +1189,7 @@ cudaError_t launch_cfg(const TcParams& p, int n_sm, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  tc_kernel<C><<<n_sm, kThreads, C::kSmemTotal, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(tc_kernel<C>, dim3(n_sm), dim3(kThreads), C::kSmemTotal, s, p);
 }
 
 cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s) {
