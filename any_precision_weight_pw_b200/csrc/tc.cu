@@ -106,7 +106,9 @@ struct Cfg {
   static constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
   static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 2 * kNDBuf + 1 + 4;
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
-  static constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 8 * (kMaxGroups + 2);
+  // misc: tmem holder, abort flag, then s_prefix, s_prefix2 and the group
+  // offsets (kMaxGroups + 2 ints each)
+  static constexpr uint32_t kOffSlotUser = kOffMisc + 16 + 12 * (kMaxGroups + 2);
   static constexpr uint32_t kSmemTotal = kOffSlotUser + 4 * kNSlot;
   static_assert(kSmemTotal <= 232448, "shared memory budget of one CTA");
   static_assert(kAColBase + kNA * kAColsPerSlot <= kTmemCols, "tensor memory budget");
@@ -359,7 +361,8 @@ __device__ __forceinline__ bool gate_or_up(int mode) {
 }
 
 // Items of a fused launch: [0, s_prefix[G]) gate/up, then the down items
-// listed by s_prefix2; gh holds one search hint per list.
+// listed by s_prefix2; gh holds one search hint per list.  The group offsets
+// (token positions) are the shared-memory copy that follows s_prefix2.
 template <class C>
 __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_prefix,
                                             const int* s_prefix2, int G, int i, Item& it,
@@ -392,8 +395,9 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
     const int Fg = (g == p.E) ? p.S : p.F;
     it.rows = gate_or_up(kind) ? Fg : p.H;
     it.cols = gate_or_up(kind) ? p.H : Fg;
-    pos0 = p.offsets[g];
-    n = p.offsets[g + 1] - pos0;
+    const int* offs = s_prefix2 + (kMaxGroups + 2);
+    pos0 = offs[g];
+    n = offs[g + 1] - pos0;
   }
   const int rt = (it.rows + kTileRows - 1) / kTileRows;
   const int stages = (((it.cols + 31) >> 5) + kStageWords - 1) / kStageWords;
@@ -690,6 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* s_prefix = reinterpret_cast<int*>(smem + C::kOffMisc + 16);
   int* s_prefix2 = s_prefix + (kMaxGroups + 2);  // fused launch: the down items
+  int* s_offs = s_prefix2 + (kMaxGroups + 2);    // group offsets (token positions)
   uint32_t* slot_user = reinterpret_cast<uint32_t*>(smem + C::kOffSlotUser);  // producer only
 
   const int warp = threadIdx.x >> 5;
@@ -699,6 +704,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   // writes what they read); the successor is not released early, so it
   // cannot take SM resources while the grid's CTAs wait on one another
   pdl_wait();
+  // group offsets into shared memory with one parallel load (the item
+  // counts below and every item decode read them)
+  if (p.mode != kTcLinear)
+    for (int g = threadIdx.x; g <= G; g += blockDim.x) s_offs[g] = p.offsets[g];
+  __syncthreads();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {
@@ -740,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         } else {
           const int Fg = (g == p.E) ? p.S : p.F;
           rows = gate_or_up(kind) ? Fg : p.H;
-          n = p.offsets[g + 1] - p.offsets[g];
+          n = s_offs[g + 1] - s_offs[g];
         }
         const int tt = (n + C::kNT - 1) / C::kNT;
         acc += ((rows + kTileRows - 1) / kTileRows) * tt * (kind == kTcDown ? p.n_split : 1);
