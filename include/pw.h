@@ -145,7 +145,11 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
                               pw_stream_t side_stream);
 
 /* y = MoE(x): d_x bf16 [T][H], d_router_w fp32 [E][H], d_router_bias fp32
- * [E] or NULL, d_y bf16 [T][H] (device).  0 <= T <= max_tokens. */
+ * [E] or NULL, d_y bf16 [T][H] (device).  0 <= T <= max_tokens.  The
+ * forward's kernels are launched with programmatic dependent launch: each
+ * may be scheduled while its predecessor on the stream drains, and waits for
+ * that predecessor's completion before it reads or writes anything; the
+ * stream order seen by the caller is unchanged. */
 pw_status_t pw_moe_forward(pw_moe_t* h, const uint16_t* d_x, int32_t T,
                            const float* d_router_w, const float* d_router_bias,
                            uint16_t* d_y, pw_stream_t stream);
