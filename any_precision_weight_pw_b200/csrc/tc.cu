@@ -25,18 +25,20 @@
 //   warp 10     token-tile loader: the item's token rows are contiguous in an
 //               fp16 buffer already in the A operand's K order (the gathered
 //               activations for gate/up, h = silu(g)*u for down), so one lane
-//               moves each stage's tile with ONE 3-D TMA box (decode: 4 atoms
-//               of 64 columns x 8, 16, 24 or 32 rows; prefill: 1 atom x 256
-//               rows; 128-byte swizzle = the MMA's K-major B layout).  A
-//               standalone linear converts its bf16 rows with all 32 lanes.
+//               moves each B stage with ONE 3-D TMA box (decode: 2 atoms of
+//               64 columns x 8, 16, 24 or 32 rows, two B stages per plane
+//               stage; prefill: 1 atom x 256 rows; 128-byte swizzle = the
+//               MMA's K-major B layout).  A standalone linear converts its
+//               bf16 rows with all 32 lanes.
 //   warps 0-7   dequantisers in two K halves: warps q and q+4 both own rows
 //               32q..32q+31 (thread <-> output row <-> TMEM lane); the first
 //               group takes columns 0-127 of every stage, the second
 //               columns 128-255.  Each thread unpacks its row's codes from the
 //               b plane words (a bit-matrix transpose), looks them up in the
-//               shared-memory table of the pass (pair table for b <= 3,
-//               single table above; see dequant.cuh) and writes fp16 weights
-//               into a TMEM ring slot (the MMA's A operand).
+//               shared-memory table of the pass (pair table up to b = 4 at
+//               decode and b = 3 at prefill, single table above; see
+//               dequant.cuh) and writes fp16 weights into a TMEM ring slot
+//               (the MMA's A operand).
 //   warp 9      MMA issuer: tcgen05.mma kind::f16, M=128, N=16/32 (decode)
 //               or 256 (prefill), K=16, fp32 accumulators in TMEM (decode:
 //               two buffers, alternating items, gate and up side by side).
@@ -44,6 +46,9 @@
 //               as fp16 in the down pass's K order (gate/up), the routing-
 //               weighted fp32 partials (down), g (prefill gate) or the fp32
 //               result (linear).
+// The forward's kernels are launched with programmatic dependent launch;
+// this kernel waits for its predecessor before it reads anything and does
+// not release its successor early.
 // Every wait is an mbarrier try_wait (with a suspend hint, so waiting warps
 // do not spin) bounded by a global-timer deadline; a timeout raises the CTA's
 // abort flag and the device error word, and every role drains what it has in
