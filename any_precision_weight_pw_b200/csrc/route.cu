@@ -19,6 +19,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kRouteThreads = 256;
 constexpr int kStageFloats = 4096;  // logits staged in shared memory (16 KB)
 constexpr int kStageSel = 16384;    // selections kept in shared memory (one byte each)
+constexpr int kStageW = 2048;       // routing weights kept in shared memory (8 KB)
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -29,8 +30,10 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
 // ascending order, then the 32 partial sums meet in a xor butterfly
 // (16, 8, 4, 2, 1), so every lane ends with the same value.  Phase 2 runs in
 // the block that finishes last (a ticket counter, no waiting): top-k and
-// softmax per token, then per-expert token lists built with warp ballots and
-// prefix counts, ordered by token.
+// softmax with a group of lanes per token (argmax rounds over the group; the
+// softmax denominator is a lane-wise sum met in a xor butterfly), then
+// per-expert counts from warp ballots, one warp-wide scan over the experts,
+// and per-expert token lists ordered by token.
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams p) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -100,14 +103,24 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   if (!s_last) return;
   __threadfence();
 
-  // ---- phase 2 (one block): top-k + softmax ------------------------------
+  // ---- phase 2 (one block): top-k + softmax, a lane group per token ------
   // The logits are staged in shared memory a chunk of tokens at a time with
-  // coalesced loads, so each thread's top-k reads shared memory instead of
-  // waiting on L2; the selections stay in shared memory (one byte each) for
-  // the bucketing below when they fit.
+  // coalesced loads.  A group of L lanes (a power of two with 4 L >= E and
+  // L >= k) serves one token: lane i of the group holds experts i + L q
+  // (q < 4); each of the k rounds is an argmax over the group under the
+  // ranking order (logit descending, index ascending), so every lane of the
+  // group ends with the same selection.  Selections and weights stay in
+  // shared memory for the bucketing below when they fit.
   __shared__ float s_logits[kStageFloats];
   __shared__ uint8_t s_idx[kStageSel];
+  __shared__ float s_w[kStageW];
   const bool sel_staged = T * k <= kStageSel;
+  const bool w_staged = T * k <= kStageW;
+  int L = 1;
+  while (4 * L < E || L < k) L <<= 1;
+  const int gl = lane & (L - 1);                       // lane within the group
+  const int gid = warp * (32 / L) + lane / L;          // group index in the block
+  const int n_groups_blk = warps_per_block * (32 / L);
   const int chunk = kStageFloats / E;  // tokens per staged chunk (>= 32)
   for (int t0 = 0; t0 < T; t0 += chunk) {
     const int nt = min(chunk, T - t0);
@@ -115,46 +128,70 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
     for (int j = threadIdx.x; j < nt * E; j += kRouteThreads)
       s_logits[j] = __ldcg(ws.logits + static_cast<size_t>(t0) * E + j);
     __syncthreads();
-    for (int tl = threadIdx.x; tl < nt; tl += kRouteThreads) {
-      const int t = t0 + tl;
-      const float* l = s_logits + tl * E;
+    // rounds are uniform over the block, so every lane takes every shuffle
+    for (int r0 = 0; r0 < nt; r0 += n_groups_blk) {
+      const int tl = r0 + gid;
+      const bool active = tl < nt;
+      const float* l = s_logits + (active ? tl : 0) * E;
+      float v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = gl + L * q;
+        v[q] = (active && e < E) ? l[e] : 0.0f;
+      }
+      uint32_t taken = 0u;  // bit q: expert gl + L q already selected
       int sel[PW_MAX_TOPK];
       float lsel[PW_MAX_TOPK];
-      uint64_t taken_lo = 0ull, taken_hi = 0ull;  // experts already selected (E <= 128)
 #pragma unroll
       for (int j = 0; j < PW_MAX_TOPK; ++j) {
         if (j >= k) break;
+        float bv = 0.0f;
         int bi = -1;
-        float best = 0.0f;
-        for (int e = 0; e < E; ++e) {
-          if ((((e < 64) ? taken_lo : taken_hi) >> (e & 63)) & 1ull) continue;
-          const float v = l[e];
-          if (bi < 0 || v > best) {  // strict: equal logits keep the lower index
-            best = v;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int e = gl + L * q;
+          if (active && e < E && !((taken >> q) & 1u) && (bi < 0 || v[q] > bv)) {
+            bv = v[q];
             bi = e;
           }
         }
-        if (bi < 64) taken_lo |= 1ull << bi; else taken_hi |= 1ull << (bi & 63);
+        for (int m = L >> 1; m >= 1; m >>= 1) {
+          const float ov = __shfl_xor_sync(kFull, bv, m);
+          const int oi = __shfl_xor_sync(kFull, bi, m);
+          if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oi < bi))) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        if (bi >= 0 && (bi & (L - 1)) == gl) taken |= 1u << (bi / L);
         sel[j] = bi;
-        lsel[j] = best;
+        lsel[j] = bv;
       }
       const float mx = lsel[0];
       float z = 0.0f;
-      for (int e = 0; e < E; ++e) z += expf(l[e] - mx);
-      float psel[PW_MAX_TOPK];
-      float ssum = 0.0f;
 #pragma unroll
-      for (int j = 0; j < PW_MAX_TOPK; ++j) {
-        if (j >= k) break;
-        psel[j] = expf(lsel[j] - mx) / z;
-        ssum += psel[j];
-      }
+      for (int q = 0; q < 4; ++q)
+        if (active && gl + L * q < E) z += expf(v[q] - mx);
+      for (int m = L >> 1; m >= 1; m >>= 1) z += __shfl_xor_sync(kFull, z, m);
+      if (active && gl == 0) {
+        const int t = t0 + tl;
+        float psel[PW_MAX_TOPK];
+        float ssum = 0.0f;
 #pragma unroll
-      for (int j = 0; j < PW_MAX_TOPK; ++j) {
-        if (j >= k) break;
-        ws.topk_idx[t * k + j] = sel[j];
-        ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
-        if (sel_staged) s_idx[t * k + j] = static_cast<uint8_t>(sel[j]);
+        for (int j = 0; j < PW_MAX_TOPK; ++j) {
+          if (j >= k) break;
+          psel[j] = expf(lsel[j] - mx) / z;
+          ssum += psel[j];
+        }
+#pragma unroll
+        for (int j = 0; j < PW_MAX_TOPK; ++j) {
+          if (j >= k) break;
+          const float w = p.renorm ? psel[j] / ssum : psel[j];
+          ws.topk_idx[t * k + j] = sel[j];
+          ws.topk_w[t * k + j] = w;
+          if (sel_staged) s_idx[t * k + j] = static_cast<uint8_t>(sel[j]);
+          if (w_staged) s_w[t * k + j] = w;
+        }
       }
     }
   }
@@ -179,22 +216,41 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   }
   __syncthreads();
   const int G = E + (p.has_shared ? 1 : 0);
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < E; ++e) {
-      s_off[e] = run;
-      run += s_cnt[e];
+  if (warp == 0) {
+    // exclusive scan over the experts: lane holds experts 4 lane .. 4 lane + 3
+    int c4[4], run = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = 4 * lane + q;
+      c4[q] = e < E ? s_cnt[e] : 0;
+      run += c4[q];
     }
-    s_off[E] = run;
-    if (p.has_shared) {
-      s_cnt[E] = T;
-      s_off[E + 1] = run + T;
+    int incl = run;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const int o = __shfl_up_sync(kFull, incl, m);
+      if (lane >= m) incl += o;
     }
-    for (int g = 0; g <= G; ++g) ws.offsets[g] = s_off[g];
-    for (int j = 0; j < p.n_zero; ++j) p.zero_words[j] = 0;
-    *ws.ticket = 0u;  // ready for the next forward (kernels on a stream do not overlap)
+    int base = incl - run;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = 4 * lane + q;
+      if (e < E) s_off[e] = base;
+      base += c4[q];
+    }
+    const int routed = __shfl_sync(kFull, incl, 31);
+    if (lane == 0) {
+      s_off[E] = routed;
+      if (p.has_shared) {
+        s_cnt[E] = T;
+        s_off[E + 1] = routed + T;
+      }
+      *ws.ticket = 0u;  // ready for the next forward (kernels on a stream do not overlap)
+    }
   }
   __syncthreads();
+  for (int g = threadIdx.x; g <= G; g += kRouteThreads) ws.offsets[g] = s_off[g];
+  for (int j = threadIdx.x; j < p.n_zero; j += kRouteThreads) p.zero_words[j] = 0;
 
   // ---- bucketing: lists ordered by token ----------------------------------
   const unsigned lt_mask = (1u << lane) - 1u;
@@ -211,6 +267,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
         const int pos = run + __popc(m & lt_mask);
         ws.slot_token[pos] = t;
         ws.token_pos[t * k + slot] = pos;
+        if (w_staged) ws.slot_w[pos] = s_w[t * k + slot];
       }
       run += __popc(m);
     }
@@ -223,10 +280,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       ws.token_pos[T * k + t] = pos;
     }
   }
-  // routing weight of every routed position (independent loads, all threads)
-  __syncthreads();
-  for (int j = threadIdx.x; j < T * k; j += kRouteThreads)
-    ws.slot_w[__ldcg(ws.token_pos + j)] = __ldcg(ws.topk_w + j);
+  if (!w_staged) {
+    // routing weight of every routed position (independent loads, all threads)
+    __syncthreads();
+    for (int j = threadIdx.x; j < T * k; j += kRouteThreads)
+      ws.slot_w[__ldcg(ws.token_pos + j)] = __ldcg(ws.topk_w + j);
+  }
 }
 
 // x_sorted row pos = the activations of token slot_token[pos] as fp16, each
