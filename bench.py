@@ -336,7 +336,10 @@ def run_ours(args, rank, world, local_rank):
     bytes_down = sum(bts[i % N_BATCHES]["down"] for i in range(steps))
     tok_s = whole_job_rate(world, steps, T, ms_max)
     fwd_gbs = bytes_total / (ms / 1e3) / 1e9
-    # dominant kernel: the tensor-core dequant-GEMM (its gate/up and down launches)
+    # dominant kernel: the tensor-core dequant-GEMM.  Launch slots 1 and 2 hold the
+    # gather launch and the tensor-core launch(es) (one fused launch at decode),
+    # so the duration includes the small gather kernel: achieved is a slight
+    # underestimate of the tensor-core kernel alone.
     tc_ms = per_launch[1] + per_launch[2]
     tc_gbs = (bytes_gu + bytes_down) / (tc_ms / 1e3) / 1e9 if tc_ms > 0 else None
     traffic = None
