@@ -203,8 +203,7 @@ pw_status_t pw_check_device_error(pw_moe_t* h);
 /* Per-launch timing for benchmarks.  While enabled, every forward records
  * CUDA events between its launch slots: route; gather + gate/up (the one
  * fused launch at decode, both prefill launches at prefill); down (empty
- * when fused); combine.  Events between launches also keep the slots from
- * overlapping through programmatic dependent launch.
+ * when fused); combine.
  * pw_profile_read synchronises on them and writes, for each launch slot, the
  * milliseconds summed over the forwards issued since the previous read (ms
  * has room for n >= 4 floats); *n_forwards receives how many were summed. */
