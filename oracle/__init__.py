@@ -60,6 +60,7 @@ def lib():
         _lib.pwo_topk_softmax.argtypes = [P, i, i, i, i, P, P]
         _lib.pwo_expert_ffn.argtypes = [C.POINTER(_Layer), i, P, P, P, i]
         _lib.pwo_moe_forward.argtypes = [C.POINTER(_Layer), P, i, P, P, P, P, P, i]
+        _lib.pwo_routing_stats.argtypes = [P, P, i, i, i, P, P]
     return _lib
 
 
@@ -134,6 +135,20 @@ def topk_softmax(logits: np.ndarray, k: int, renorm: bool):
     _check(lib().pwo_topk_softmax(_ptr(logits), T, E, k, int(renorm), _ptr(idx), _ptr(w)),
            "topk")
     return idx, w
+
+
+def routing_stats(idx: np.ndarray, w: np.ndarray, n_experts: int, counts=None, mass=None):
+    """Per-expert assignment counts and routing-weight sums of a batch,
+    added to (counts, mass) when given (accumulation over forwards)."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    T, k = idx.shape
+    counts = np.zeros(n_experts, np.uint64) if counts is None else counts
+    mass = np.zeros(n_experts, np.float64) if mass is None else mass
+    assert counts.dtype == np.uint64 and mass.dtype == np.float64
+    _check(lib().pwo_routing_stats(_ptr(idx), _ptr(w), T, k, n_experts, _ptr(counts),
+                                   _ptr(mass)), "routing_stats")
+    return counts, mass
 
 
 class Layer:

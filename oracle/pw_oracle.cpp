@@ -35,6 +35,9 @@
 //                                       closed forms for E=2 and k=E)
 //   pwo_expert_ffn / pwo_moe_forward    pinned (hand-worked 2-expert example,
 //                                       shared-expert linearity, SiLU limits)
+//   pwo_routing_stats                   pinned (hand-worked example, totals
+//                                       T*k and T, k = E column sums equal
+//                                       a softmax written out in numpy)
 
 #include <cmath>
 #include <cstdint>
@@ -241,6 +244,25 @@ int pwo_topk_softmax(const float* logits, int T, int E, int k, int renorm,
       w[static_cast<size_t>(t) * k + j] = renorm ? pj / sel : pj;
     }
   }
+  return 0;
+}
+
+// Routing statistics of a batch: the online "routing mass" the planner
+// weighs (legiblepapers summary, "Summary & Methodology Analysis": routing
+// mass is how frequently an expert is used).  Reading: per expert e, the
+// number of (token, slot) assignments to e and the sum of their routing
+// weights, ADDED to counts[e] and mass[e] so that calls accumulate over
+// forwards.  idx / w are [T][k] as pwo_topk_softmax returns them.
+int pwo_routing_stats(const int32_t* idx, const double* w, int T, int k, int E,
+                      uint64_t* counts, double* mass) {
+  if ((T > 0 && (!idx || !w)) || !counts || !mass || k < 1 || E < 1) return 1;
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[static_cast<size_t>(t) * k + j];
+      if (e < 0 || e >= E) return 1;
+      counts[e] += 1;
+      mass[e] += w[static_cast<size_t>(t) * k + j];
+    }
   return 0;
 }
 

@@ -119,3 +119,47 @@ def test_routing_weights_closed_forms(oracle):
     # renorm divides by the selected mass
     _, wr = oracle.topk_softmax(l, 2, renorm=True)
     np.testing.assert_allclose(wr, wa / wa.sum(axis=1, keepdims=True), rtol=1e-14)
+
+
+# ---- routing statistics (the planner's online routing mass) ---------------
+
+def test_routing_stats_hand_example(oracle):
+    """The hand example's routing: t0 -> (0, 1) with weights (s, 1-s), t1 ->
+    (1, 0) with (s, 1-s), t2 -> (0, 1) with (1/2, 1/2), s the logistic of 1.
+    Each expert is used three times with weight mass s + (1-s) + 1/2 = 3/2;
+    a second call adds the same again."""
+    s = 1.0 / (1.0 + math.exp(-1.0))
+    idx = np.array([[0, 1], [1, 0], [0, 1]], np.int32)
+    w = np.array([[s, 1 - s], [s, 1 - s], [0.5, 0.5]])
+    counts, mass = oracle.routing_stats(idx, w, 2)
+    assert counts.tolist() == [3, 3]
+    np.testing.assert_allclose(mass, [1.5, 1.5], rtol=1e-15)
+    counts, mass = oracle.routing_stats(idx, w, 2, counts, mass)
+    assert counts.tolist() == [6, 6]
+    np.testing.assert_allclose(mass, [3.0, 3.0], rtol=1e-15)
+
+
+def test_routing_stats_totals_and_unused_experts(oracle):
+    """Totals: T*k assignments; with renormalised weights the mass sums to T.
+    An expert that is never selected keeps zero count and mass."""
+    rng = np.random.default_rng(9)
+    l = rng.normal(size=(50, 8)).astype(np.float32)
+    l[:, 5] = -100.0                      # expert 5 never wins a slot
+    idx, w = oracle.topk_softmax(l, 3, renorm=True)
+    counts, mass = oracle.routing_stats(idx, w, 8)
+    assert int(counts.sum()) == 150 and counts[5] == 0 and mass[5] == 0.0
+    assert mass.sum() == pytest.approx(50.0, rel=1e-13)
+
+
+def test_routing_stats_k_equals_e_is_the_softmax_column_sum(oracle):
+    """k = E without renormalisation: every expert is in every token's list
+    with its full softmax probability, so mass[e] = sum_t softmax(l_t)[e],
+    written here directly with numpy in float64."""
+    rng = np.random.default_rng(10)
+    l = rng.normal(size=(40, 6)).astype(np.float32)
+    idx, w = oracle.topk_softmax(l, 6, renorm=False)
+    counts, mass = oracle.routing_stats(idx, w, 6)
+    z = np.exp(l.astype(np.float64) - l.max(axis=1, keepdims=True))
+    p = z / z.sum(axis=1, keepdims=True)
+    assert counts.tolist() == [40] * 6
+    np.testing.assert_allclose(mass, p.sum(axis=0), rtol=1e-13)
