@@ -23,6 +23,7 @@ EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy"
             "pw_moe_forward_host", "pw_linear", "pw_get_block_bits", "pw_get_routing",
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
             "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
+            "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats",
             "pw_last_error", "pw_abi_version"]
 
 
@@ -62,6 +63,9 @@ def lib():
         L.pw_moe_forward_host.argtypes = [P, P, i32, P, P, P, P]
         L.pw_linear.argtypes = [P, P, i32, i32, i32, i32, P, i32, P, P]
         L.pw_get_block_bits.argtypes = [P, i32, C.POINTER(i32), C.POINTER(i32)]
+        L.pw_get_forward_bits.argtypes = [P, C.POINTER(i32), i32]
+        L.pw_set_switch_lag.argtypes = [P, i32]
+        L.pw_routing_stats.argtypes = [P, P, P, i32, P]
         L.pw_get_routing.argtypes = [P, P, P, P]
         L.pw_check_device_error.argtypes = [P]
         L.pw_profile_enable.argtypes = [P, i32]
@@ -193,9 +197,19 @@ class MoELayer:
         check(lib().pw_set_block_bits(self.h, block, bits, side_stream.cuda_stream))
 
     def get_block_bits(self, block: int):
-        nxt, pend = C.c_int32(), C.c_int32()
-        check(lib().pw_get_block_bits(self.h, block, C.byref(nxt), C.byref(pend)))
-        return nxt.value, pend.value
+        """(bitwidth as of the last issued forward, pending width or 0)."""
+        cur, pend = C.c_int32(), C.c_int32()
+        check(lib().pw_get_block_bits(self.h, block, C.byref(cur), C.byref(pend)))
+        return cur.value, pend.value
+
+    def forward_bits(self) -> List[int]:
+        """Bitwidth of every block in the most recently issued forward."""
+        out = (C.c_int32 * self.n_blocks)()
+        check(lib().pw_get_forward_bits(self.h, out, self.n_blocks))
+        return list(out)
+
+    def set_switch_lag(self, max_lag: int) -> None:
+        check(lib().pw_set_switch_lag(self.h, max_lag))
 
     def routing(self, T: int, stream=None):
         import torch
@@ -204,6 +218,15 @@ class MoELayer:
         w = torch.empty((T, k), dtype=torch.float32, device="cuda")
         check(lib().pw_get_routing(self.h, _ptr(idx), _ptr(w), _stream(stream)))
         return idx, w
+
+    def routing_stats(self, reset: bool = False, stream=None):
+        """(counts uint64 [E], mass float64 [E]) accumulated over forwards."""
+        E = self.cfg["n_experts"]
+        counts = np.zeros(E, dtype=np.uint64)
+        mass = np.zeros(E, dtype=np.float64)
+        check(lib().pw_routing_stats(self.h, counts.ctypes.data, mass.ctypes.data,
+                                     1 if reset else 0, _stream(stream)))
+        return counts, mass
 
     def check_device_error(self) -> None:
         check(lib().pw_check_device_error(self.h))
@@ -234,10 +257,10 @@ class MoELayer:
 
 
 def upload_synth_layer(layer, max_tokens: int, host_copies: bool = False,
-                       device: str = "cuda") -> MoELayer:
+                       device: str = "cuda", host_planes: bool = True) -> MoELayer:
     """Put a synth.Layer's pages on the device and create the library layer.
-    With host_copies, pinned master copies of all planes and every LUT width
-    are kept for bitwidth switches."""
+    With host_copies, pinned master copies of every LUT width, and of all
+    planes unless host_planes is False, are kept for bitwidth switches."""
     import torch
     wl = layer.wl
     planes, slots, hp, hl = [], [], [], []
@@ -251,8 +274,9 @@ def upload_synth_layer(layer, max_tokens: int, host_copies: bool = False,
         lt = layer.lut(blk, layer.bits[blk])
         s0[: lt.size].copy_(torch.from_numpy(lt.reshape(-1).view(np.int16)))
         slots.append((s0, s1))
-        if host_copies:
+        if host_copies and host_planes:
             hp.append(paged.cpu().pin_memory())
+        if host_copies:
             hl.append({b: torch.from_numpy(layer.lut(blk, b).reshape(-1).view(np.int16)).pin_memory()
                        for b in range(1, wl.n_max + 1)})
     cfg = dict(hidden=wl.hidden, ffn=wl.ffn, n_experts=wl.n_experts, top_k=wl.top_k,

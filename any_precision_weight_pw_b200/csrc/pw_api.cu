@@ -135,11 +135,13 @@ struct pw_moe {
     const uint16_t* h_lut[PW_MAX_BITS + 1];
     int bits, slot;            // active bitwidth and LUT slot
     int pend_bits;             // 0 = none
-    long long pend_due;        // forward index from which the change applies
+    long long pend_req;        // forwards issued when the change was requested
     cudaEvent_t ready;
   };
   std::vector<Blk> blk;
   long long n_forwards = 0;
+  int max_lag = 8;                   // forwards a page move may stay pending
+  std::vector<int32_t> fwd_bits;     // bitwidths of the most recent forward
   cudaEvent_t fwd_done = nullptr;
   bool any_forward = false;
   // workspace
@@ -156,6 +158,8 @@ struct pw_moe {
   bool pf = false;                   // the prefill passes are available
   float* ysorted = nullptr;
   int* err = nullptr;
+  unsigned long long* stat_count = nullptr;  // routing statistics [E]
+  double* stat_mass = nullptr;               // [E]
   uint16_t* stage_x = nullptr;
   uint16_t* stage_y = nullptr;
   int P_max = 0, gu_stride = 0, max_split = 8, last_T = 0;
@@ -277,7 +281,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
     d.bits = b.bits;
     d.slot = 0;
     d.pend_bits = 0;
-    d.pend_due = 0;
+    d.pend_req = 0;
     d.ready = nullptr;
     if (cudaEventCreateWithFlags(&d.ready, cudaEventDisableTiming) != cudaSuccess) {
       free_all(h);
@@ -312,6 +316,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const size_t o_tk = off; off += al(sizeof(uint32_t) * 4);
   const size_t o_err = off; off += al(sizeof(int) * 4);
   const size_t o_gd = off; off += al(sizeof(int) * (h->G + 1));
+  const size_t o_sc = off; off += al(sizeof(unsigned long long) * E);
+  const size_t o_sm = off; off += al(sizeof(double) * E);
   const size_t o_gu = off; off += al(sizeof(float) * size_t(h->P_max) * h->gu_stride);
   const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->x_ld);
   const size_t o_hp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->h_perm_ld);
@@ -336,6 +342,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->ws.ticket = reinterpret_cast<uint32_t*>(w + o_tk);
   h->err = reinterpret_cast<int*>(w + o_err);
   h->gu_done = reinterpret_cast<int*>(w + o_gd);
+  h->stat_count = reinterpret_cast<unsigned long long*>(w + o_sc);
+  h->stat_mass = reinterpret_cast<double*>(w + o_sm);
   h->gu = reinterpret_cast<float*>(w + o_gu);
   h->x_sorted = reinterpret_cast<uint16_t*>(w + o_xp);
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
@@ -343,7 +351,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->gbuf = reinterpret_cast<float*>(w + o_gb);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
   h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
-  if (cudaMemset(w + o_tk, 0, o_gd + al(sizeof(int) * (h->G + 1)) - o_tk) != cudaSuccess ||
+  if (cudaMemset(w + o_tk, 0, o_sm + al(sizeof(double) * E) - o_tk) != cudaSuccess ||
       cudaMemset(w + o_xp, 0, o_sx - o_xp) != cudaSuccess) {
     free_all(h);
     return fail(PW_ERR_CUDA, "cudaMemset failed");
@@ -393,19 +401,33 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
                           cudaMemcpyHostToDevice, s));
   PW_CUDA(cudaEventRecord(b.ready, s));
   b.pend_bits = new_bits;
-  b.pend_due = h->n_forwards + 1;
+  b.pend_req = h->n_forwards;
   return PW_OK;
 }
 
-pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_next,
+pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_active,
                               int32_t* bits_pending) {
-  if (!h || !bits_next) return fail(PW_ERR_INVALID_ARG, "null argument");
+  if (!h || !bits_active) return fail(PW_ERR_INVALID_ARG, "null argument");
   if (block_id < 0 || block_id >= h->n_blocks)
     return fail(PW_ERR_INVALID_ARG, "block id %d out of range", block_id);
   const auto& b = h->blk[block_id];
-  const bool due = b.pend_bits && b.pend_due <= h->n_forwards;
-  *bits_next = due ? b.pend_bits : b.bits;
-  if (bits_pending) *bits_pending = due ? 0 : b.pend_bits;
+  *bits_active = b.bits;
+  if (bits_pending) *bits_pending = b.pend_bits;
+  return PW_OK;
+}
+
+pw_status_t pw_get_forward_bits(const pw_moe_t* h, int32_t* bits, int32_t n) {
+  if (!h || !bits) return fail(PW_ERR_INVALID_ARG, "null argument");
+  if (n < h->n_blocks) return fail(PW_ERR_INVALID_ARG, "need room for %d bitwidths", h->n_blocks);
+  for (int i = 0; i < h->n_blocks; ++i)
+    bits[i] = h->fwd_bits.empty() ? h->blk[i].bits : h->fwd_bits[i];
+  return PW_OK;
+}
+
+pw_status_t pw_set_switch_lag(pw_moe_t* h, int32_t max_lag) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  if (max_lag < 0) return fail(PW_ERR_INVALID_ARG, "max_lag must be >= 0");
+  h->max_lag = max_lag;
   return PW_OK;
 }
 
@@ -413,15 +435,23 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
                                 const float* d_wr, const float* d_bias, uint16_t* d_y,
                                 cudaStream_t s) {
   const pw_moe_config_t& c = h->cfg;
-  // page moves that are due: the stream waits for their copies
+  // pending page moves: one whose copy has already completed takes effect
+  // now, without any wait; one that has stayed pending for max_lag forwards
+  // takes effect now too, and the stream waits for its copy
   for (auto& b : h->blk) {
-    if (b.pend_bits && b.pend_due <= h->n_forwards) {
-      PW_CUDA(cudaStreamWaitEvent(s, b.ready, 0));
-      b.bits = b.pend_bits;
-      b.slot ^= 1;
-      b.pend_bits = 0;
-    }
+    if (!b.pend_bits) continue;
+    const cudaError_t q = cudaEventQuery(b.ready);
+    if (q != cudaSuccess && q != cudaErrorNotReady)
+      return fail(PW_ERR_CUDA, "cudaEventQuery (page move) failed: %s", cudaGetErrorString(q));
+    const bool landed = q == cudaSuccess;
+    if (!landed && h->n_forwards - b.pend_req < h->max_lag) continue;
+    if (!landed) PW_CUDA(cudaStreamWaitEvent(s, b.ready, 0));
+    b.bits = b.pend_bits;
+    b.slot ^= 1;
+    b.pend_bits = 0;
   }
+  h->fwd_bits.resize(h->n_blocks);
+  for (int i = 0; i < h->n_blocks; ++i) h->fwd_bits[i] = h->blk[i].bits;
   h->n_forwards++;
   h->last_T = T;
   if (T == 0) {
@@ -470,6 +500,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   rp.ws = h->ws;
   rp.zero_words = fused ? h->gu_done : nullptr;
   rp.n_zero = fused ? h->G : 0;
+  rp.stat_count = h->stat_count;
+  rp.stat_mass = h->stat_mass;
   PW_CUDA(pw::launch_route(rp, h->n_sm, s));
   PW_CUDA(mark(1));
 
@@ -506,6 +538,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.err = h->err;
     if (fused) {
       tp.n_split = down_splits(h, T, 6);
+      tp.cooperative = env_int("PW_COOP", 0);
       for (int i = 0; i < 4; ++i) tp.h_maps[i] = h->h_maps[i];
       tp.gu_done = h->gu_done;
       tp.ysorted = h->ysorted;
@@ -708,6 +741,22 @@ pw_status_t pw_get_routing(const pw_moe_t* h, int32_t* d_idx, float* d_w, pw_str
     PW_CUDA(cudaMemcpyAsync(d_idx, h->ws.topk_idx, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s));
     PW_CUDA(cudaMemcpyAsync(d_w, h->ws.topk_w, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
   }
+  return PW_OK;
+}
+
+pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_t reset,
+                             pw_stream_t stream) {
+  if (!h || !counts || !mass) return fail(PW_ERR_INVALID_ARG, "null argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int E = h->cfg.n_experts;
+  static_assert(sizeof(uint64_t) == sizeof(unsigned long long), "64-bit counters");
+  PW_CUDA(cudaMemcpyAsync(counts, h->stat_count, sizeof(uint64_t) * E, cudaMemcpyDeviceToHost, s));
+  PW_CUDA(cudaMemcpyAsync(mass, h->stat_mass, sizeof(double) * E, cudaMemcpyDeviceToHost, s));
+  if (reset) {
+    PW_CUDA(cudaMemsetAsync(h->stat_count, 0, sizeof(uint64_t) * E, s));
+    PW_CUDA(cudaMemsetAsync(h->stat_mass, 0, sizeof(double) * E, s));
+  }
+  PW_CUDA(cudaStreamSynchronize(s));
   return PW_OK;
 }
 

@@ -19,20 +19,29 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// cooperative: the grid's CTAs are all resident at once or the launch fails
+// (for kernels whose CTAs wait on one another).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t s, Args&&... args) {
+cudaError_t launch_pdl_ex(bool cooperative, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+                          size_t smem, cudaStream_t s, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cooperative ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  return launch_pdl_ex(false, kernel, grid, block, smem, s, static_cast<Args&&>(args)...);
 }
 #endif
 
@@ -76,6 +85,8 @@ struct RouteParams {
   RouteWorkspace ws;
   int* zero_words;         // counters of the launches that follow, set to zero
   int n_zero;              // (may be null / 0)
+  unsigned long long* stat_count;  // [E] routing statistics, accumulated over
+  double* stat_mass;               // forwards (both null: none kept)
 };
 
 struct GatherParams {

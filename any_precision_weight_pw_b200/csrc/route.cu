@@ -253,9 +253,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   for (int j = threadIdx.x; j < p.n_zero; j += kRouteThreads) p.zero_words[j] = 0;
 
   // ---- bucketing: lists ordered by token ----------------------------------
+  // With routing statistics on, the warp of expert e also sums the weights of
+  // e's slots (in double: per 32-token block a xor butterfly, blocks in token
+  // order) and adds its count and weight sum to the handle's counters; one
+  // warp owns each expert, so the counters need no atomics.
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int e = warp; e < E; e += warps_per_block) {
     int run = s_off[e];
+    double mass = 0.0;
     for (int base = 0; base < T; base += 32) {
       const int t = base + lane;
       int slot = -1;
@@ -263,13 +268,27 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
         for (int j = 0; j < k; ++j)
           if (sel_of(t, j) == e) slot = j;
       const unsigned m = __ballot_sync(kFull, slot >= 0);
+      double wm = 0.0;
       if (slot >= 0) {
         const int pos = run + __popc(m & lt_mask);
         ws.slot_token[pos] = t;
         ws.token_pos[t * k + slot] = pos;
-        if (w_staged) ws.slot_w[pos] = s_w[t * k + slot];
+        const float w = w_staged       ? s_w[t * k + slot]
+                        : p.stat_count ? __ldcg(ws.topk_w + t * k + slot)
+                                       : 0.0f;
+        if (w_staged) ws.slot_w[pos] = w;
+        wm = static_cast<double>(w);
+      }
+      if (p.stat_count) {
+#pragma unroll
+        for (int sh = 16; sh >= 1; sh >>= 1) wm += __shfl_xor_sync(kFull, wm, sh);
+        mass += wm;
       }
       run += __popc(m);
+    }
+    if (p.stat_count && lane == 0) {
+      p.stat_count[e] += static_cast<unsigned long long>(s_off[e + 1] - s_off[e]);
+      p.stat_mass[e] += mass;
     }
   }
   if (p.has_shared) {

@@ -11,8 +11,10 @@
 // have no counterpart of this call; it is a library convenience.
 //
 // The scratch is one array per device for the whole process.  Its address is
-// looked up once per device, on the first call there, with
-// cudaGetSymbolAddress; later calls only read the cached pointer.
+// looked up with cudaGetSymbolAddress on every call made outside a stream
+// capture (so a module reloaded after cudaDeviceReset is found again) and
+// cached per device; a call made while its stream is being captured uses the
+// cached address, so the first call on a device must come before any capture.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -69,10 +71,16 @@ extern "C" pw_status_t pw_route_static(const uint16_t* d_x, const float* d_route
   if (dev < 0 || dev >= kMaxDevices)
     return pw::record_error(PW_ERR_UNSUPPORTED, "pw_route_static: device ordinal >= 64");
 
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap);
+  if (e != cudaSuccess) return pw::record_error(PW_ERR_CUDA, cudaGetErrorString(e));
   unsigned char* base;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (cap != cudaStreamCaptureStatusNone && !g_scratch_ptr[dev])
+      return pw::record_error(PW_ERR_STATE,
+                              "pw_route_static: first call on a device inside a stream capture");
+    if (cap == cudaStreamCaptureStatusNone) {
       void* p = nullptr;
       e = cudaGetSymbolAddress(&p, g_route_scratch);
       if (e != cudaSuccess || !p) {

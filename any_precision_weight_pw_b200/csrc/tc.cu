@@ -57,6 +57,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "dequant.cuh"
 #include "pages.h"
 #include "pw_internal.h"
@@ -1195,16 +1197,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
 
 }  // namespace
 
+// The shared-memory attribute is per device context: set it once per device
+// (under a lock, since handles on different devices may launch from
+// different threads).
 template <class C>
 cudaError_t launch_cfg(const TcParams& p, int n_sm, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::kSmemTotal));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(C::kSmemTotal));
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
   }
-  return launch_pdl(tc_kernel<C>, dim3(n_sm), dim3(kThreads), C::kSmemTotal, s, p);
+  // a fused launch's down items wait on other CTAs' gate/up items: launched
+  // cooperatively, so either every CTA is resident or the launch fails
+  const bool coop = p.mode == kTcFused && p.cooperative;
+  return launch_pdl_ex(coop, tc_kernel<C>, dim3(n_sm), dim3(kThreads), C::kSmemTotal, s, p);
 }
 
 cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s) {

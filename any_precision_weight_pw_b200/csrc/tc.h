@@ -50,6 +50,7 @@ struct TcParams {
   float* gbuf;                   // prefill: gate outputs [rows][gbuf_ld] fp32
   int gbuf_ld;
   int* err;                      // device error word (may be null)
+  int cooperative;               // fused mode: launch with the cooperative attribute
 };
 
 cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s);

@@ -189,9 +189,14 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
     sched = synth.switch_schedule(wl, layer.bits, total, every=10)
     pb = [binding.plane_bytes(*layer.shape(blk)) for blk in range(wl.n_blocks)]
 
-    def run(with_switches):
+    def run(with_switches, track=False):
+        # track: also read back, after every forward, the widths it used, to
+        # count how many forwards each switch takes to apply (an extra host
+        # call per forward, so only in an untimed pass)
         bits = list(layer.bits) if with_switches else None
         moved = 0
+        lags = []        # forwards from a switch's request until all of it applies
+        waiting = []     # (forward of the request, widths after it)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(total)]
         for f in range(total):
@@ -202,17 +207,30 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
                     if f >= warmup:
                         moved += max(nb - bits[blk], 0) * pb[blk] + rows * (1 << nb) * 2
                     bits[blk] = nb
+                if track:
+                    waiting.append((f, list(bits)))
             evs[f][0].record(stream)
             d.forward(xs[f % N_BATCHES], wr, None, ys[f % N_BATCHES])
             evs[f][1].record(stream)
+            if waiting:
+                used = d.forward_bits()
+                while waiting and used == waiting[0][1]:
+                    lags.append(f - waiting.pop(0)[0])
         torch.cuda.synchronize()
         d.check_device_error()
         lat = np.array([a.elapsed_time(b) for a, b in evs[warmup:]])
         span = evs[warmup][0].elapsed_time(evs[-1][1])
-        return lat, span, moved
+        return lat, span, moved, lags
 
-    base_lat, base_span, _ = run(False)
-    lat, span, moved = run(True)
+    base_lat, base_span, _, _ = run(False)
+    lat, span, moved, _ = run(True)
+    # widths back to the starting table, then the untimed pass that counts lags
+    for blk in range(wl.n_blocks):
+        d.set_block_bits(blk, layer.bits[blk], side)
+    for _ in range(10):
+        d.forward(xs[0], wr, None, ys[0])
+        torch.cuda.synchronize()
+    _, _, _, lags = run(True, track=True)
     n_switch = sum(1 for f in sched if f >= warmup)
     out = {"workload": "qwen15_moe_a27b decode T=%d, 25%% of blocks switch every 10 forwards" % T,
            "forwards": n_forwards, "tokens_per_s": round(n_forwards * T / (span / 1e3), 1),
@@ -222,9 +240,76 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
            "ms_per_forward_max": round(float(lat.max()), 4),
            "page_bytes_per_switch": int(moved / max(n_switch, 1)),
            "blocks_per_switch": len(next(iter(sched.values()))),
+           "forwards_until_applied": {"mean": round(float(np.mean(lags)), 2) if lags else None,
+                                      "max": int(max(lags)) if lags else None,
+                                      "max_lag": 8},
            "no_switch": {"tokens_per_s": round(n_forwards * T / (base_span / 1e3), 1),
                          "ms_per_forward_p99": round(float(np.percentile(base_lat, 99)), 4)}}
     d.close()
+    return out
+
+
+def time_flushed(d, xs, ys, wr, bias, flush, n=20, warmup=3):
+    """Median ms of single forwards, each after an L2 flush (CUDA events on
+    the forward stream)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    times = []
+    for i in range(warmup + n):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        d.forward(xs[i % len(xs)], wr, bias, ys[i % len(ys)])
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(a.elapsed_time(b))
+    d.check_device_error()
+    return float(np.median(times))
+
+
+def uniform_vs_mixed(dev, hbm_peak):
+    """Mixed per-block bitwidths against uniform ones, at kernel level: the
+    same layer shape and token batches with every block at one width b (for
+    each b of the workload's set), then with the workload's mixed table.
+    The pages report at most 4.1% throughput loss of the mixed system
+    against uniform quantisation (legiblepapers FAQ Q7; hardware unstated);
+    here the comparable figure is the achieved GB/s of the mixed table
+    against the uniform widths' (same bytes-per-second machinery, different
+    bytes per forward)."""
+    import torch
+    from any_precision_weight_pw_b200 import binding, synth
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = []
+    for name, T in (("mixtral_8x7b", 16), ("qwen15_moe_a27b", 32)):
+        wl = synth.WORKLOADS[name]
+        mixed = synth.Layer(wl, seed=0)
+        rows = []
+        for tag, bits in [("uniform %d" % b, [b] * wl.n_blocks) for b in wl.bit_choices
+                          if b in (3, 4, 6)] + [("mixed", None)]:
+            layer = mixed if bits is None else synth.Layer(wl, seed=0, bits=bits)
+            d = binding.upload_synth_layer(layer, max_tokens=T)
+            wr = torch.from_numpy(layer.router_w).to(dev)
+            xs_np = [synth.tokens(wl, T, seed=0, batch=b) for b in range(N_BATCHES)]
+            xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x in xs_np]
+            ys = [torch.empty_like(x) for x in xs]
+            mb = []
+            for x, y in zip(xs, ys):
+                d.forward(x, wr, None, y)
+                idx, _ = d.routing(T)
+                mb.append(algorithmic_bytes(layer, idx.cpu().numpy())["total"])
+            ms = time_flushed(d, xs, ys, wr, None, flush)
+            gbs = float(np.mean(mb)) / (ms / 1e3) / 1e9
+            rows.append({"bits": tag, "avg_bits": round(float(np.mean(layer.bits)), 3),
+                         "ms": round(ms, 4), "tokens_per_s": round(T / (ms / 1e3), 1),
+                         "gbs": round(gbs, 1), "frac_of_measured_hbm": round(gbs / hbm_peak, 4)})
+            d.close()
+            del xs, ys
+        uni = [r["gbs"] for r in rows if r["bits"] != "mixed"]
+        mix = [r["gbs"] for r in rows if r["bits"] == "mixed"][0]
+        out.append({"workload": "%s decode T=%d" % (name, T), "runs": rows,
+                    "mixed_gbs_vs_uniform_mean": round(mix / float(np.mean(uni)), 4)})
+    del flush
     return out
 
 
@@ -374,6 +459,7 @@ def run_ours(args, rank, world, local_rank):
     sweep = []
     page_move = None
     prefill = None
+    uniform = None
     if rank == 0 and not args.no_sweep:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         cur = (name, layer, d, wr, bias)
@@ -383,18 +469,7 @@ def run_ours(args, rank, world, local_rank):
                 cur = (wname,) + prepare_layer(wname, seed=rank)
             _, lay, dd, wr2, b2 = cur
             xs2, _, ys2, bts2 = prepare_batches(lay, dd, wr2, b2, wT, seed=rank)
-            times = []
-            for i in range(3 + 20):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                dd.forward(xs2[i % N_BATCHES], wr2, b2, ys2[i % N_BATCHES])
-                b.record(stream)
-                torch.cuda.synchronize()
-                if i >= 3:
-                    times.append(a.elapsed_time(b))
-            dd.check_device_error()
-            med = float(np.median(times))
+            med = time_flushed(dd, xs2, ys2, wr2, b2, flush)
             mb = float(np.mean([bb["total"] for bb in bts2]))
             sweep.append({"workload": wname, "tokens": wT, "ms_median": round(med, 4),
                           "tokens_per_s": round(wT / (med / 1e3), 1),
@@ -406,6 +481,7 @@ def run_ours(args, rank, world, local_rank):
         del flush
         page_move = page_move_stress(dev)
         prefill = prefill_measure(dev)
+        uniform = uniform_vs_mixed(dev, hbm_peak)
     else:
         d.close()
 
@@ -451,6 +527,7 @@ def run_ours(args, rank, world, local_rank):
         "sweep": sweep,
         "page_move": page_move,
         "prefill": prefill,
+        "uniform_vs_mixed": uniform,
     }
     return out
 

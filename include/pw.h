@@ -138,9 +138,18 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
  * raising b -> b' copies planes b..b'-1 and LUT_b' from the host copies;
  * lowering copies LUT_b' only (the top b' planes are already resident).  The
  * LUT lands in the idle slot, so no forward ever reads memory being written.
- * Lag: with N forwards issued, forward N still uses the old bitwidth and
- * forward N+1 waits for the copy and uses the new one.  PW_ERR_STATE while an
- * earlier change of the same block has not taken effect yet. */
+ * When it takes effect (PagedWeight, legiblepapers "Summary & Methodology
+ * Analysis": pages move asynchronously to hide latency): every forward issued
+ * afterwards checks, without blocking (cudaEventQuery), whether the copy has
+ * completed; the first forward that finds it complete uses the new bitwidth.
+ * A change still pending after max_lag more forwards (pw_set_switch_lag,
+ * default 8) takes effect at the next forward, which then waits on the GPU
+ * for the copy.  pw_get_forward_bits reports the bitwidths each forward used.
+ * Forwards of one handle go on one stream (the copy is ordered after the
+ * last issued forward through an event on that stream).  PW_ERR_STATE while
+ * an earlier change of the same block has not taken effect yet;
+ * PW_ERR_INVALID_ARG (nothing enqueued) when the host LUT for new_bits is
+ * NULL, or when raising the width of a block whose host planes are NULL. */
 pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
                               pw_stream_t side_stream);
 
@@ -187,14 +196,40 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
                       int32_t cols, int32_t n_max, int32_t bits, const uint16_t* d_x,
                       int32_t T, float* d_y, pw_stream_t stream);
 
-/* Bitwidth the next forward will use, and the pending one (0 if none). */
-pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_next,
+/* Bitwidth of a block as of the most recently issued forward (the one the
+ * create call set, before any forward), and the width of a change still
+ * pending (0 if none). */
+pw_status_t pw_get_block_bits(const pw_moe_t* h, int32_t block_id, int32_t* bits_active,
                               int32_t* bits_pending);
+
+/* The bitwidth every block had in the most recently issued forward (the
+ * create-time widths before any forward), in block-id order; bits has room
+ * for n >= 3E (+3) entries.  Lets a caller replay exactly what each forward
+ * computed while page moves land asynchronously. */
+pw_status_t pw_get_forward_bits(const pw_moe_t* h, int32_t* bits, int32_t n);
+
+/* Largest number of forwards a page move may stay pending before a forward
+ * waits for its copy (>= 0; 0 = the next forward always waits and uses the
+ * new width). */
+pw_status_t pw_set_switch_lag(pw_moe_t* h, int32_t max_lag);
 
 /* Routing of the most recent forward: d_idx int32 [T][k] (selection order)
  * and d_w fp32 [T][k], copied device-to-device on stream. */
 pw_status_t pw_get_routing(const pw_moe_t* h, int32_t* d_idx, float* d_w,
                            pw_stream_t stream);
+
+/* Online routing statistics: the planner's "routing mass", how often each
+ * expert is used (PagedWeight, legiblepapers "Summary & Methodology
+ * Analysis" and FAQ Q4/Q8: damage per released byte weighs offline
+ * sensitivity, online routing mass and prompt residuals).  Every forward's
+ * route kernel adds, for each routed expert e, the number of (token, slot)
+ * assignments to e and the sum of their routing weights (the weights the
+ * combine applies), accumulated on the device in 64-bit counters and
+ * doubles.  This call copies them into the host arrays counts [E] and mass
+ * [E] after the forwards issued so far on stream, zeroes them if reset != 0,
+ * and returns once the copies have landed (it synchronises stream). */
+pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_t reset,
+                             pw_stream_t stream);
 
 /* Synchronises the device and reports a device-side error flag of the handle
  * (PW_ERR_TIMEOUT if a bounded wait gave up) and clears it. */
@@ -231,9 +266,11 @@ int32_t pw_forward_launches(const pw_moe_t* h, int32_t T);
  *   0 <= T <= PW_ROUTE_STATIC_MAX_TOKENS, 1 <= top_k <= min(n_experts, 8),
  *   n_experts <= 128, renorm_topk 0 or 1; anything else is PW_ERR_INVALID_ARG
  *   with nothing enqueued.  T = 0 returns PW_OK at once.
- * The first call on a device looks up the array's address
- * (cudaGetSymbolAddress; PW_ERR_CUDA if that fails) and caches it; make that
- * first call before any stream capture on the device begins.
+ * Every call made outside a stream capture looks up the array's address
+ * (cudaGetSymbolAddress; PW_ERR_CUDA if that fails), so the address stays
+ * right after a cudaDeviceReset, and caches it per device; a call made while
+ * its stream is being captured uses the cached address, so make the first
+ * call on a device before any stream capture there (PW_ERR_STATE otherwise).
  * Races: the array is shared by every call on the device in the process.  Two
  * calls whose kernels can overlap (different streams without an event between
  * them, or several host threads) corrupt each other's scratch and results;

@@ -219,7 +219,7 @@ def test_qwen_shaped_layer(pw, oracle, T):
     assert_output_close(y, ref)
 
 
-@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("T", [1, 16, 64])
 def test_mixtral_shaped_layer(pw, oracle, T):
     layer = synth.Layer(synth.WORKLOADS["mixtral_8x7b"], seed=0)
     y, idx, w, x = _run_layer(pw, layer, T, batch=T)
@@ -252,18 +252,21 @@ def test_zero_tokens_and_bad_T(pw):
     dev.close()
 
 
-def test_bitwidth_switch_lag_and_parity(pw, oracle):
-    """A switch requested after N forwards: forward N keeps the old widths,
-    forward N+1 uses the new ones; both match the oracle at those widths."""
+def test_bitwidth_switch_waits_at_lag_zero(pw, oracle):
+    """max_lag 0: the forward issued right after the requests waits for the
+    page moves and uses the new widths; it and the next match the oracle at
+    those widths, and the widths reported before it are the old ones."""
     wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
     layer = synth.Layer(wl, seed=3)
     dev = pw.upload_synth_layer(layer, max_tokens=16, host_copies=True)
+    dev.set_switch_lag(0)
     wr = torch.from_numpy(layer.router_w).cuda()
     side = torch.cuda.Stream()
     changes = {0: 8, 4: 2, 5: 6, 11: 1, 23: 8}
     x0 = synth.tokens(wl, 16, seed=3, batch=0)
     dev.forward(_dev_bf16(x0), wr)                      # forward 0
     old = list(layer.bits)
+    assert dev.forward_bits() == old
     for blk, b in changes.items():
         dev.set_block_bits(blk, b, side)
         assert dev.get_block_bits(blk) == (old[blk], b)
@@ -272,18 +275,135 @@ def test_bitwidth_switch_lag_and_parity(pw, oracle):
     new = list(old)
     for blk, b in changes.items():
         new[blk] = b
-    for f, bits in ((1, old), (2, new), (3, new)):
+    for f in (1, 2):
         x = synth.tokens(wl, 16, seed=3, batch=f)
         y = dev.forward(_dev_bf16(x), wr)
+        assert dev.forward_bits() == new
         torch.cuda.synchronize()
-        yf = _to_f32(y)
-        ref, _, _ = oracle_layer(oracle, layer, bits).forward(x, layer.router_w, threads=8)
-        assert_output_close(yf, ref)
-        if f == 1:
-            for blk, b in changes.items():
-                assert dev.get_block_bits(blk) == (b, 0)
+        ref, _, _ = oracle_layer(oracle, layer, new).forward(x, layer.router_w, threads=8)
+        assert_output_close(_to_f32(y), ref)
+    for blk, b in changes.items():
+        assert dev.get_block_bits(blk) == (b, 0)
     dev.check_device_error()
     dev.close()
+
+
+def test_bitwidth_switch_async_replay(pw, oracle):
+    """Default lag: a change takes effect at the first forward issued after
+    its copy has landed (at the latest max_lag forwards after the request);
+    every forward matches the oracle at the widths it reports."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=6)
+    dev = pw.upload_synth_layer(layer, max_tokens=16, host_copies=True)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    side = torch.cuda.Stream()
+    sched = {1: [(2, 8), (7, 1)], 3: [(2, 3), (13, 7), (20, 2)]}
+    want = list(layer.bits)
+    for f in range(12):
+        for blk, b in sched.get(f, []):
+            dev.set_block_bits(blk, b, side)
+            want[blk] = b
+        x = synth.tokens(wl, 16, seed=6, batch=f)
+        y = dev.forward(_dev_bf16(x), wr)
+        used = dev.forward_bits()
+        torch.cuda.synchronize()   # lets the copies land before the next forward
+        ref, _, _ = oracle_layer(oracle, layer, used).forward(x, layer.router_w, threads=8)
+        assert_output_close(_to_f32(y), ref)
+        if f in (2, 4) or f > 4:
+            # the previous forward's synchronize let every copy requested
+            # before it land, so this forward found them complete
+            assert used == want, (f, used, want)
+    dev.check_device_error()
+    dev.close()
+
+
+def test_switch_stress_replay_qwen_shaped(pw, oracle):
+    """The Qwen-shaped switch stress (decode batch 32; before every 10th
+    forward a quarter of the blocks change width, page moves on a side
+    stream), 41 forwards issued back to back.  The widths each forward
+    reports are replayed through the oracle: forward 0, every 10th, and the
+    first forwards after each switch at which part and all of its changes
+    had landed are compared."""
+    wl = synth.WORKLOADS["qwen15_moe_a27b_switch"]
+    T = wl.tokens[0]
+    layer = synth.Layer(wl, seed=0)
+    dev = pw.upload_synth_layer(layer, max_tokens=T, host_copies=True)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    side = torch.cuda.Stream()
+    n = 41
+    sched = synth.switch_schedule(wl, layer.bits, n, every=10)
+    assert all(len(v) == round(0.25 * wl.n_blocks) for v in sched.values())
+    ys, used, want_after = [], [], {}
+    want = list(layer.bits)
+    for f in range(n):
+        for blk, b in sched.get(f, []):
+            dev.set_block_bits(blk, b, side)
+            want[blk] = b
+        if f in sched:
+            want_after[f] = list(want)
+        x = synth.tokens(wl, T, seed=0, batch=f)
+        ys.append(dev.forward(_dev_bf16(x), wr))
+        used.append(dev.forward_bits())
+    torch.cuda.synchronize()
+    dev.check_device_error()
+    lag = 8
+    pick = {0} | {f for f in range(0, n, 10)}
+    for f0, w in want_after.items():
+        # every change of the switch took effect within the lag
+        full = [f for f in range(f0, min(n, f0 + lag + 1)) if used[f] == w]
+        assert full, "switch before forward %d never completed within the lag" % f0
+        pick.add(full[0])
+        part = [f for f in range(f0, full[0] + 1) if used[f] != used[f - 1]]
+        if part:
+            pick.add(part[0])
+    assert used[-1] == want
+    for f in sorted(pick):
+        x = synth.tokens(wl, T, seed=0, batch=f)
+        ref, ridx, _ = oracle_layer(oracle, layer, used[f]).forward(x, layer.router_w, threads=32)
+        assert_output_close(_to_f32(ys[f]), ref)
+    dev.close()
+
+
+def test_switch_rejects_missing_host_copies(pw):
+    """Raising the width of a block without host planes, and a width without
+    a host LUT, are rejected with nothing enqueued; the layer keeps working."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=0)
+    side = torch.cuda.Stream()
+    b0 = layer.bits[0]
+    bare = pw.upload_synth_layer(layer, max_tokens=4)     # no host copies at all
+    with pytest.raises(pw.PwError) as e:
+        bare.set_block_bits(0, b0 - 1, side)              # no host LUT for that width
+    assert e.value.status == 1 and "LUT" in str(e.value)
+    bare.close()
+    dev = pw.upload_synth_layer(layer, max_tokens=4, host_copies=True, host_planes=False)
+    with pytest.raises(pw.PwError) as e:
+        dev.set_block_bits(0, b0 + 1, side)               # raising needs the host planes
+    assert e.value.status == 1 and "planes" in str(e.value)
+    assert dev.get_block_bits(0) == (b0, 0)
+    dev.set_block_bits(0, b0 - 1, side)                   # lowering needs only the LUT
+    assert dev.get_block_bits(0) == (b0, b0 - 1)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    dev.forward(_dev_bf16(synth.tokens(wl, 4, seed=0)), wr)
+    torch.cuda.synchronize()
+    dev.check_device_error()
+    dev.close()
+
+
+def test_destroy_with_work_in_flight(pw):
+    """pw_destroy while a forward and a page move are still queued waits for
+    them and returns PW_OK."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=0)
+    dev = pw.upload_synth_layer(layer, max_tokens=16, host_copies=True)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    side = torch.cuda.Stream()
+    x = _dev_bf16(synth.tokens(wl, 16, seed=0))
+    dev.forward(x, wr)
+    dev.set_block_bits(1, 8, side)
+    dev.forward(x, wr)
+    dev.close()                                          # raises on a non-OK status
+    torch.cuda.synchronize()
 
 
 def test_forward_host_matches_device(pw):
@@ -299,10 +419,12 @@ def test_forward_host_matches_device(pw):
 
 
 def test_prefill_scale_layer_sampled(pw, oracle):
-    """Mixtral-shaped layer at prefill scale (4096 tokens, Zipf-skewed expert
-    usage, experts 0 and 1 at 8 bits, the rest at 4): every token's routing
-    is compared with the oracle's, and the outputs of a sample of tokens
-    (the oracle computes each token on its own)."""
+    """Mixtral-shaped layer at prefill scale (4096 tokens, Zipf(1.2)-skewed
+    expert usage, experts 0 and 1 at 8 bits, the rest at 4): every token's
+    routing is compared with the oracle's, expert 0's top-1 share is Zipf's
+    0.429 +- 0.02, and the outputs of a stratified sample of 256 tokens (32
+    whose first choice is each expert, so both 8-bit experts and every
+    other) are compared (the oracle computes each token on its own)."""
     wl = synth.WORKLOADS["mixtral_8x7b_prefill"]
     layer = synth.Layer(wl, seed=0)
     T = 4096
@@ -311,13 +433,16 @@ def test_prefill_scale_layer_sampled(pw, oracle):
     ridx, rw = oracle.topk_softmax(logits, wl.top_k, bool(wl.renorm_topk))
     np.testing.assert_array_equal(idx, ridx)
     np.testing.assert_allclose(w, rw, rtol=1e-5, atol=1e-7)
-    counts = np.bincount(idx.reshape(-1), minlength=wl.n_experts)
-    assert counts[0] == counts.max() and counts[0] > 2 * np.sort(counts)[-3]  # skewed usage
+    top1 = np.bincount(idx[:, 0], minlength=wl.n_experts) / T
+    assert abs(top1[0] - synth.zipf_pmf(wl.n_experts, wl.zipf_s)[0]) <= 0.02, top1
     rng = np.random.default_rng(7)
-    heavy = np.flatnonzero(idx[:, 0] == 0)[:4]          # tokens on the 8-bit expert 0
-    sample = np.unique(np.concatenate([heavy, rng.choice(T, 12, replace=False), [0, T - 1]]))
+    per = 256 // wl.n_experts
+    sample = np.sort(np.concatenate([
+        rng.choice(np.flatnonzero(idx[:, 0] == e), per, replace=False)
+        for e in range(wl.n_experts)]))
+    assert sample.size == 256
     L = oracle_layer(oracle, layer)
-    ref, sidx, _ = L.forward(x[sample], layer.router_w, layer.router_bias, threads=32)
+    ref, sidx, _ = L.forward(x[sample], layer.router_w, layer.router_bias, threads=64)
     np.testing.assert_array_equal(sidx, idx[sample])
     assert_output_close(y[sample], ref)
 
@@ -368,3 +493,33 @@ def test_prefill_passes_qwen_shaped_sampled(pw, oracle):
     L = oracle_layer(oracle, layer)
     ref, _, _ = L.forward(x[sample], layer.router_w, None, threads=32)
     assert_output_close(y[sample], ref)
+
+
+@pytest.mark.parametrize("name,T,n_fwd", [("tiny_h256_f512_e8k2", 16, 1000),
+                                          ("qwen15_moe_a27b", 32, 20)])
+def test_routing_stats_accumulate_over_forwards(pw, oracle, name, T, n_fwd):
+    """The route kernel's per-expert counters (assignments and routing-weight
+    mass, the planner's online routing mass) over many forwards of distinct
+    batches: counts equal the oracle's exactly, mass within 1e-5 relative;
+    a read with reset zeroes them."""
+    wl = synth.WORKLOADS[name]
+    layer = synth.Layer(wl, seed=8)
+    dev = pw.upload_synth_layer(layer, max_tokens=T)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    counts = np.zeros(wl.n_experts, np.uint64)
+    mass = np.zeros(wl.n_experts, np.float64)
+    y = torch.empty((T, wl.hidden), dtype=torch.int16, device="cuda")
+    for f in range(n_fwd):
+        x = synth.tokens(wl, T, seed=8, batch=f)
+        dev.forward(_dev_bf16(x), wr, None, y)
+        idx, w = oracle.topk_softmax(oracle.router_logits(x, layer.router_w, None), wl.top_k,
+                                     bool(wl.renorm_topk))
+        oracle.routing_stats(idx, w, wl.n_experts, counts, mass)
+    got_c, got_m = dev.routing_stats(reset=True)
+    dev.check_device_error()
+    np.testing.assert_array_equal(got_c, counts)
+    np.testing.assert_allclose(got_m, mass, rtol=1e-5, atol=1e-9)
+    assert int(got_c.sum()) == n_fwd * T * wl.top_k
+    c2, m2 = dev.routing_stats()
+    assert not c2.any() and not m2.any()
+    dev.close()
