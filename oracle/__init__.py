@@ -61,6 +61,8 @@ def lib():
         _lib.pwo_expert_ffn.argtypes = [C.POINTER(_Layer), i, P, P, P, i]
         _lib.pwo_moe_forward.argtypes = [C.POINTER(_Layer), P, i, P, P, P, P, P, i]
         _lib.pwo_routing_stats.argtypes = [P, P, i, i, i, P, P]
+        _lib.pwo_plan_greedy.argtypes = [P, i, C.c_int64, P, P, P]
+        _lib.pwo_plan_exact.argtypes = [P, i, C.c_int64, P, P, P]
     return _lib
 
 
@@ -149,6 +151,48 @@ def routing_stats(idx: np.ndarray, w: np.ndarray, n_experts: int, counts=None, m
     _check(lib().pwo_routing_stats(_ptr(idx), _ptr(w), T, k, n_experts, _ptr(counts),
                                    _ptr(mass)), "routing_stats")
     return counts, mass
+
+
+class PlanBlock(C.Structure):
+    """One block as the planner sees it (see pwo_plan_greedy)."""
+    _fields_ = [("bits", C.c_int32), ("min_bits", C.c_int32), ("plane_bytes", C.c_int64),
+                ("rows", C.c_int32), ("mass", C.c_double), ("resid", C.c_double),
+                ("sens", C.c_double * 9)]
+
+
+def _plan_array(blocks):
+    arr = (PlanBlock * len(blocks))()
+    for j, b in enumerate(blocks):
+        arr[j].bits, arr[j].min_bits = int(b["bits"]), int(b["min_bits"])
+        arr[j].plane_bytes, arr[j].rows = int(b["plane_bytes"]), int(b["rows"])
+        arr[j].mass, arr[j].resid = float(b["mass"]), float(b.get("resid", 0.0))
+        for k in range(9):
+            arr[j].sens[k] = float(b["sens"][k]) if k < len(b["sens"]) else 0.0
+    return arr
+
+
+def _plan(fn, blocks, target):
+    arr = _plan_array(blocks)
+    n = len(blocks)
+    bits = (C.c_int32 * max(n, 1))()
+    rel = C.c_int64()
+    dmg = C.c_double()
+    rc = fn(arr, n, int(target), bits, C.byref(rel), C.byref(dmg))
+    if rc == 1:
+        raise ValueError("oracle planner rejected its arguments")
+    return {"bits": list(bits)[:n], "released": rel.value, "damage": dmg.value,
+            "reached": rc == 0}
+
+
+def plan_greedy(blocks, target):
+    """Greedy least-damage-per-byte release plan (dicts with bits, min_bits,
+    plane_bytes, rows, mass, resid, sens[0..8])."""
+    return _plan(lib().pwo_plan_greedy, blocks, target)
+
+
+def plan_exact(blocks, target):
+    """The brute-force optimum of the same problem (tiny instances)."""
+    return _plan(lib().pwo_plan_exact, blocks, target)
 
 
 class Layer:

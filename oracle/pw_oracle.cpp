@@ -35,6 +35,10 @@
 //                                       closed forms for E=2 and k=E)
 //   pwo_expert_ffn / pwo_moe_forward    pinned (hand-worked 2-expert example,
 //                                       shared-expert linearity, SiLU limits)
+//   pwo_plan_greedy / pwo_plan_exact    pinned (hand-worked instance; greedy
+//                                       equals the brute-force optimum where
+//                                       the exchange argument holds; greedy
+//                                       never beats the optimum)
 //   pwo_routing_stats                   pinned (hand-worked example, totals
 //                                       T*k and T, k = E column sums equal
 //                                       a softmax written out in numpy)
@@ -263,6 +267,115 @@ int pwo_routing_stats(const int32_t* idx, const double* w, int T, int k, int E,
       counts[e] += 1;
       mass[e] += w[static_cast<size_t>(t) * k + j];
     }
+  return 0;
+}
+
+// ---- the quality-aware planner (host-side decision) ------------------------
+//
+// legiblepapers summary, "Summary & Methodology Analysis" and FAQ Q8: the
+// runtime planner takes a target number of bytes to free and greedily picks
+// weight quantisation actions with the least damage per released byte; the
+// damage combines offline sensitivity, online routing mass and prompt
+// residuals.  The pages give no formula; the reading taken here:
+//   action (i, b): lower block i from b to b - 1 bits (b > min_bits[i]); it
+//     releases plane page b - 1 and shrinks the LUT from 2^b to 2^(b-1)
+//     fp16 entries per row:  bytes(i, b) = plane_bytes[i] + rows[i] * 2^(b-1) * 2
+//   damage(i, b) = sens[i][b] * mass[i] * (1 + resid[i])   (in double, in
+//     this order), sens[i][b] the offline sensitivity of that step, mass[i]
+//     the routing mass of the block's expert, resid[i] >= 0 a prompt-residual
+//     weight.
+//   greedy: while released < target, take the action with the smallest
+//     damage / bytes (double division; ties to the lower block index) and
+//     apply it.
+typedef struct {
+  int32_t bits, min_bits;   // current width, lowest allowed width
+  int64_t plane_bytes;      // bytes of one plane page of the block
+  int32_t rows;             // LUT rows
+  double mass, resid;       // routing mass of the block's expert, residual weight
+  double sens[9];           // sens[b]: damage of the step b -> b - 1 (b = 1..8)
+} pwo_plan_block_t;
+
+static int64_t plan_step_bytes(const pwo_plan_block_t& k, int b) {
+  return k.plane_bytes + static_cast<int64_t>(k.rows) * (int64_t{1} << (b - 1)) * 2;
+}
+static double plan_step_damage(const pwo_plan_block_t& k, int b) {
+  return k.sens[b] * k.mass * (1.0 + k.resid);
+}
+
+// Greedy: new_bits[n], *released, *damage.  Returns 0 when the target was
+// reached, 2 when no action was left before reaching it (new_bits then holds
+// every block at its lowest width), 1 on bad arguments.
+int pwo_plan_greedy(const pwo_plan_block_t* blocks, int n, int64_t target, int32_t* new_bits,
+                    int64_t* released, double* damage) {
+  if (!blocks || !new_bits || !released || !damage || n < 0) return 1;
+  for (int i = 0; i < n; ++i) {
+    if (blocks[i].bits < 1 || blocks[i].bits > 8 || blocks[i].min_bits < 1 ||
+        blocks[i].min_bits > blocks[i].bits)
+      return 1;
+    new_bits[i] = blocks[i].bits;
+  }
+  *released = 0;
+  *damage = 0.0;
+  while (*released < target) {
+    int best = -1;
+    double best_ratio = 0.0;
+    for (int i = 0; i < n; ++i) {
+      const int b = new_bits[i];
+      if (b <= blocks[i].min_bits) continue;
+      const double ratio = plan_step_damage(blocks[i], b) /
+                           static_cast<double>(plan_step_bytes(blocks[i], b));
+      if (best < 0 || ratio < best_ratio) {
+        best = i;
+        best_ratio = ratio;
+      }
+    }
+    if (best < 0) return 2;
+    const int b = new_bits[best];
+    *released += plan_step_bytes(blocks[best], b);
+    *damage += plan_step_damage(blocks[best], b);
+    new_bits[best] = b - 1;
+  }
+  return 0;
+}
+
+// The exact optimum of the same problem by brute force over every width
+// vector (min_bits[i] .. bits[i] per block): the smallest total damage whose
+// released bytes reach the target (ties: the first vector in lexicographic
+// order of (w_0, w_1, ...) descending from the current widths).  For tiny
+// instances only.  Returns 0, or 2 if no vector reaches the target.
+int pwo_plan_exact(const pwo_plan_block_t* blocks, int n, int64_t target, int32_t* best_bits,
+                   int64_t* released, double* damage) {
+  if (!blocks || !best_bits || !released || !damage || n < 0 || n > 12) return 1;
+  std::vector<int> w(n);
+  for (int i = 0; i < n; ++i) w[i] = blocks[i].bits;
+  bool found = false;
+  double best_d = 0.0;
+  int64_t best_r = 0;
+  while (true) {
+    int64_t r = 0;
+    double d = 0.0;
+    for (int i = 0; i < n; ++i)
+      for (int b = blocks[i].bits; b > w[i]; --b) {
+        r += plan_step_bytes(blocks[i], b);
+        d += plan_step_damage(blocks[i], b);
+      }
+    if (r >= target && (!found || d < best_d)) {
+      found = true;
+      best_d = d;
+      best_r = r;
+      for (int i = 0; i < n; ++i) best_bits[i] = w[i];
+    }
+    int i = n - 1;  // next vector: odometer, each digit counting down
+    while (i >= 0 && w[i] == blocks[i].min_bits) {
+      w[i] = blocks[i].bits;
+      --i;
+    }
+    if (i < 0) break;
+    --w[i];
+  }
+  if (!found) return 2;
+  *released = best_r;
+  *damage = best_d;
   return 0;
 }
 
