@@ -23,7 +23,7 @@ EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy"
             "pw_moe_forward_host", "pw_linear", "pw_get_block_bits", "pw_get_routing",
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
             "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
-            "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats",
+            "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats", "pw_plan_release",
             "pw_last_error", "pw_abi_version"]
 
 
@@ -37,6 +37,12 @@ class Config(C.Structure):
     _fields_ = [("hidden", C.c_int32), ("ffn", C.c_int32), ("n_experts", C.c_int32),
                 ("top_k", C.c_int32), ("shared_ffn", C.c_int32), ("n_max", C.c_int32),
                 ("renorm_topk", C.c_int32), ("max_tokens", C.c_int32)]
+
+
+class PlanBlock(C.Structure):
+    _fields_ = [("bits", C.c_int32), ("min_bits", C.c_int32), ("plane_bytes", C.c_int64),
+                ("rows", C.c_int32), ("mass", C.c_double), ("resid", C.c_double),
+                ("sens", C.c_double * (PW_MAX_BITS + 1))]
 
 
 class BlockDesc(C.Structure):
@@ -66,6 +72,9 @@ def lib():
         L.pw_get_forward_bits.argtypes = [P, C.POINTER(i32), i32]
         L.pw_set_switch_lag.argtypes = [P, i32]
         L.pw_routing_stats.argtypes = [P, P, P, i32, P]
+        L.pw_plan_release.argtypes = [C.POINTER(PlanBlock), i32, C.c_int64, C.POINTER(i32),
+                                      C.POINTER(C.c_int64), C.POINTER(C.c_double),
+                                      C.POINTER(i32)]
         L.pw_get_routing.argtypes = [P, P, P, P]
         L.pw_check_device_error.argtypes = [P]
         L.pw_profile_enable.argtypes = [P, i32]
@@ -147,6 +156,26 @@ def route_static(x, router_w, top_k: int, renorm_topk: int, router_bias=None, id
     check(lib().pw_route_static(_ptr(x), _ptr(router_w), _ptr(router_bias), T, H, E, top_k,
                                 renorm_topk, _ptr(idx), _ptr(w), _stream(stream)))
     return idx, w
+
+
+def plan_release(blocks, target_bytes: int):
+    """Greedy release plan through pw_plan_release.  blocks: dicts with bits,
+    min_bits, plane_bytes, rows, mass, resid, sens (sens[b] for b = 0..8).
+    Returns {"bits", "released", "damage", "reached"}."""
+    n = len(blocks)
+    arr = (PlanBlock * max(n, 1))()
+    for j, b in enumerate(blocks):
+        arr[j].bits, arr[j].min_bits = int(b["bits"]), int(b["min_bits"])
+        arr[j].plane_bytes, arr[j].rows = int(b["plane_bytes"]), int(b["rows"])
+        arr[j].mass, arr[j].resid = float(b["mass"]), float(b.get("resid", 0.0))
+        for k in range(PW_MAX_BITS + 1):
+            arr[j].sens[k] = float(b["sens"][k]) if k < len(b["sens"]) else 0.0
+    bits = (C.c_int32 * max(n, 1))()
+    rel, dmg, reached = C.c_int64(), C.c_double(), C.c_int32()
+    check(lib().pw_plan_release(arr, n, int(target_bytes), bits, C.byref(rel), C.byref(dmg),
+                                C.byref(reached)))
+    return {"bits": list(bits)[:n], "released": rel.value, "damage": dmg.value,
+            "reached": bool(reached.value)}
 
 
 class MoELayer:

@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpw_b200.so")
-SOURCES = ["pw_api.cu", "route.cu", "simple.cu", "tc.cu", "repack.cu", "route_static.cu"]
+SOURCES = ["pw_api.cu", "route.cu", "simple.cu", "tc.cu", "repack.cu", "route_static.cu",
+           "planner.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -29,7 +30,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(tmpdir, exist_ok=True)
     objs = []
     for src in SOURCES:
-        obj = os.path.join(tmpdir, src.replace(".cu", ".o"))
+        obj = os.path.join(tmpdir, os.path.splitext(src)[0] + ".o")
         cmd = [nvcc, "-std=c++17", "-O3", "-lineinfo", *ARCH, "-Xcompiler", "-fPIC",
                "-I", os.path.join(ROOT, "include"), "-c", os.path.join(SRC, src), "-o", obj]
         if verbose:

@@ -231,6 +231,39 @@ pw_status_t pw_get_routing(const pw_moe_t* h, int32_t* d_idx, float* d_w,
 pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_t reset,
                              pw_stream_t stream);
 
+/* ---- the quality-aware release planner (host only) --------------------- */
+
+/* One linear-block as the planner sees it. */
+typedef struct {
+  int32_t bits;          /* current bitwidth, 1..8 */
+  int32_t min_bits;      /* lowest width the planner may choose, 1..bits */
+  int64_t plane_bytes;   /* bytes of one plane page (pw_plane_bytes) */
+  int32_t rows;          /* LUT rows (the block's output rows) */
+  double mass;           /* routing mass of the block's expert (from
+                            pw_routing_stats; the shared expert's is the
+                            token count), >= 0 */
+  double resid;          /* prompt-residual weight, >= 0 */
+  double sens[PW_MAX_BITS + 1]; /* sens[b]: offline damage of the step b -> b-1 */
+} pw_plan_block_t;
+
+/* Greedy release plan (PagedWeight, legiblepapers "Summary & Methodology
+ * Analysis" and FAQ Q8: the planner frees a target number of bytes by
+ * picking, one at a time, the quantisation action with the least damage per
+ * released byte; damage combines offline sensitivity, online routing mass
+ * and prompt residuals).  Reading of the pages: an action lowers one block
+ * by one bit, b -> b-1 (b > min_bits), releasing its plane page b-1 and half
+ * of its LUT: plane_bytes + rows * 2^(b-1) * 2 bytes; its damage is
+ * sens[b] * mass * (1 + resid), evaluated in double in that order; the
+ * action with the smallest damage / bytes (double division) goes first,
+ * ties to the lower block index; actions stop once the released bytes
+ * reach target_bytes.  Writes the chosen width of every block to new_bits
+ * [n], the bytes released and the summed damage, and *reached = 1 if the
+ * target was met (0: every block ended at min_bits short of it).  Pure host
+ * computation; apply the plan with pw_set_block_bits. */
+pw_status_t pw_plan_release(const pw_plan_block_t* blocks, int32_t n, int64_t target_bytes,
+                            int32_t* new_bits, int64_t* released, double* damage,
+                            int32_t* reached);
+
 /* Synchronises the device and reports a device-side error flag of the handle
  * (PW_ERR_TIMEOUT if a bounded wait gave up) and clears it. */
 pw_status_t pw_check_device_error(pw_moe_t* h);
