@@ -24,6 +24,7 @@ EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy"
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
             "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
             "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats", "pw_plan_release",
+            "pw_enable_paging", "pw_resident_bytes",
             "pw_last_error", "pw_abi_version"]
 
 
@@ -72,6 +73,8 @@ def lib():
         L.pw_get_forward_bits.argtypes = [P, C.POINTER(i32), i32]
         L.pw_set_switch_lag.argtypes = [P, i32]
         L.pw_routing_stats.argtypes = [P, P, P, i32, P]
+        L.pw_enable_paging.argtypes = [P, P]
+        L.pw_resident_bytes.argtypes = [P, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.pw_plan_release.argtypes = [C.POINTER(PlanBlock), i32, C.c_int64, C.POINTER(i32),
                                       C.POINTER(C.c_int64), C.POINTER(C.c_double),
                                       C.POINTER(i32)]
@@ -247,6 +250,17 @@ class MoELayer:
         w = torch.empty((T, k), dtype=torch.float32, device="cuda")
         check(lib().pw_get_routing(self.h, _ptr(idx), _ptr(w), _stream(stream)))
         return idx, w
+
+    def enable_paging(self, stream=None) -> None:
+        """Library-owned plane storage holding only each block's resident
+        planes (the caller's plane buffers may be freed afterwards)."""
+        check(lib().pw_enable_paging(self.h, _stream(stream)))
+
+    def resident_bytes(self, trim: bool = False):
+        """(plane bytes resident, pool bytes reserved after a trim or None)."""
+        pb, pr = C.c_int64(), C.c_int64()
+        check(lib().pw_resident_bytes(self.h, C.byref(pb), C.byref(pr) if trim else None))
+        return pb.value, (pr.value if trim else None)
 
     def routing_stats(self, reset: bool = False, stream=None):
         """(counts uint64 [E], mass float64 [E]) accumulated over forwards."""

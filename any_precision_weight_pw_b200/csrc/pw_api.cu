@@ -134,11 +134,16 @@ struct pw_moe {
     const uint32_t* h_planes;
     const uint16_t* h_lut[PW_MAX_BITS + 1];
     int bits, slot;            // active bitwidth and LUT slot
+    int stride;                // planes per tile group of d_planes
+    bool owned;                // d_planes is library storage (paging)
     int pend_bits;             // 0 = none
     long long pend_req;        // forwards issued when the change was requested
+    uint32_t* pend_planes;     // paging: the storage the pending change fills
     cudaEvent_t ready;
   };
   std::vector<Blk> blk;
+  bool paging = false;               // plane storage owned by the library
+  cudaMemPool_t pool = nullptr;      // paging: the plane pages' memory pool
   long long n_forwards = 0;
   int max_lag = 8;                   // forwards a page move may stay pending
   std::vector<int32_t> fwd_bits;     // bitwidths of the most recent forward
@@ -189,8 +194,12 @@ void free_all(pw_moe* h) {
   for (auto& v : h->ev_pending)
     for (auto e : v) cudaEventDestroy(e);
   for (auto e : h->ev_pool) cudaEventDestroy(e);
-  for (auto& b : h->blk)
+  for (auto& b : h->blk) {
     if (b.ready) cudaEventDestroy(b.ready);
+    if (b.owned && b.d_planes) cudaFree(b.d_planes);
+    if (b.pend_planes) cudaFree(b.pend_planes);
+  }
+  if (h->pool) cudaMemPoolDestroy(h->pool);
   if (h->fwd_done) cudaEventDestroy(h->fwd_done);
   if (h->ws_base) cudaFree(h->ws_base);
   delete h;
@@ -280,8 +289,11 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
     for (int k = 0; k <= PW_MAX_BITS; ++k) d.h_lut[k] = b.h_lut[k];
     d.bits = b.bits;
     d.slot = 0;
+    d.stride = c.n_max;
+    d.owned = false;
     d.pend_bits = 0;
     d.pend_req = 0;
+    d.pend_planes = nullptr;
     d.ready = nullptr;
     if (cudaEventCreateWithFlags(&d.ready, cudaEventDisableTiming) != cudaSuccess) {
       free_all(h);
@@ -314,6 +326,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   const size_t o_sw = off; off += al(sizeof(float) * h->P_max);
   const size_t o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
   const size_t o_tk = off; off += al(sizeof(uint32_t) * 4);
+  const size_t o_tc = off; off += al(sizeof(uint32_t) * T);
   const size_t o_err = off; off += al(sizeof(int) * 4);
   const size_t o_gd = off; off += al(sizeof(int) * (h->G + 1));
   const size_t o_sc = off; off += al(sizeof(unsigned long long) * E);
@@ -340,6 +353,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->ws.slot_w = reinterpret_cast<float*>(w + o_sw);
   h->ws.token_pos = reinterpret_cast<int32_t*>(w + o_tp);
   h->ws.ticket = reinterpret_cast<uint32_t*>(w + o_tk);
+  h->ws.tok_ctr = reinterpret_cast<uint32_t*>(w + o_tc);
   h->err = reinterpret_cast<int*>(w + o_err);
   h->gu_done = reinterpret_cast<int*>(w + o_gd);
   h->stat_count = reinterpret_cast<unsigned long long*>(w + o_sc);
@@ -387,7 +401,32 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
     return fail(PW_ERR_INVALID_ARG, "block %d: raising bits needs the host planes", block_id);
   cudaStream_t s = static_cast<cudaStream_t>(side_stream);
   if (h->any_forward) PW_CUDA(cudaStreamWaitEvent(s, h->fwd_done, 0));
-  if (new_bits > b.bits) {
+  if (h->paging) {
+    // new storage holding exactly new_bits planes per tile group: the kept
+    // planes come from the current storage, raised ones from the host copy;
+    // the current storage is freed once the change has taken effect
+    const size_t tile = pw::pages::kTileBytes;
+    const size_t groups = static_cast<size_t>(pw::pages::groups_of(b.rows, b.cols));
+    void* np = nullptr;
+    if (cudaMallocFromPoolAsync(&np, static_cast<size_t>(new_bits) * groups * tile, h->pool, s) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return fail(PW_ERR_OOM, "block %d: no room in the plane-page pool for %d planes", block_id,
+                  new_bits);
+    }
+    uint32_t* dst = static_cast<uint32_t*>(np);
+    const int keep = new_bits < b.bits ? new_bits : b.bits;
+    PW_CUDA(cudaMemcpy2DAsync(dst, new_bits * tile, b.d_planes, b.stride * tile, keep * tile, groups,
+                              cudaMemcpyDeviceToDevice, s));
+    if (new_bits > b.bits) {
+      const size_t pitch = static_cast<size_t>(h->cfg.n_max) * tile;
+      const size_t off = static_cast<size_t>(b.bits) * (tile / 4);
+      PW_CUDA(cudaMemcpy2DAsync(dst + off, new_bits * tile, b.h_planes + off, pitch,
+                                static_cast<size_t>(new_bits - b.bits) * tile, groups,
+                                cudaMemcpyHostToDevice, s));
+    }
+    b.pend_planes = dst;
+  } else if (new_bits > b.bits) {
     // planes b.bits .. new_bits-1 are tiles b.bits.. of every tile group
     const size_t pitch = static_cast<size_t>(h->cfg.n_max) * pw::pages::kTileBytes;
     const size_t groups = static_cast<size_t>(pw::pages::groups_of(b.rows, b.cols));
@@ -446,6 +485,15 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     const bool landed = q == cudaSuccess;
     if (!landed && h->n_forwards - b.pend_req < h->max_lag) continue;
     if (!landed) PW_CUDA(cudaStreamWaitEvent(s, b.ready, 0));
+    if (b.pend_planes) {
+      // paging: the forwards issued so far may still read the old storage;
+      // this stream-ordered free runs after them and before this forward
+      if (b.owned) PW_CUDA(cudaFreeAsync(b.d_planes, s));
+      b.d_planes = b.pend_planes;
+      b.stride = b.pend_bits;
+      b.owned = true;
+      b.pend_planes = nullptr;
+    }
     b.bits = b.pend_bits;
     b.slot ^= 1;
     b.pend_bits = 0;
@@ -464,6 +512,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     pt.blk[i].planes = h->blk[i].d_planes;
     pt.blk[i].lut = h->blk[i].d_lut[h->blk[i].slot];
     pt.bits[i] = static_cast<uint8_t>(h->blk[i].bits);
+    pt.stride[i] = static_cast<uint8_t>(h->blk[i].stride);
   }
   const int has_shared = c.shared_ffn > 0 ? 1 : 0;
   const bool prefill = h->tc && use_prefill(h, T);
@@ -536,9 +585,17 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_perm_ld = h->h_perm_ld;
     tp.h_rows = h->P_max;
     tp.err = h->err;
+    tp.test_stall_group = -1;
     if (fused) {
+      // test switches: a shorter wait limit, and one group's down items
+      // waiting for a count that never arrives (failure-detection tests)
+      tp.wait_ns = static_cast<unsigned long long>(env_int("PW_TEST_WAIT_US", 0)) * 1000ull;
+      tp.test_stall_group = env_int("PW_TEST_STALL_GROUP", -1);
       tp.n_split = down_splits(h, T, 6);
-      tp.cooperative = env_int("PW_COOP", 0);
+      // down items wait on other CTAs' gate/up items, so every CTA must be
+      // resident: the launch is cooperative (refused rather than stalled when
+      // the grid cannot be co-resident); PW_COOP=0 drops the attribute
+      tp.cooperative = env_int("PW_COOP", 1);
       for (int i = 0; i < 4; ++i) tp.h_maps[i] = h->h_maps[i];
       tp.gu_done = h->gu_done;
       tp.ysorted = h->ysorted;
@@ -582,6 +639,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     n_split = prefill ? 1 : down_splits(h, T, 4);
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
+    tp.test_stall_group = -1;
     tp.pt = pt;
     tp.mode = prefill ? pw::kTcPfDown : pw::kTcDown;
     tp.pf_map = h->h_pf_map;
@@ -686,6 +744,7 @@ pw_status_t pw_linear(const uint32_t* d_planes, const uint16_t* d_lut, int32_t r
   if (tc_shape_ok(cols) && env_int("PW_FORCE_SIMPLE", 0) == 0) {
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
+    tp.test_stall_group = -1;
     tp.mode = pw::kTcLinear;
     tp.n_groups = 1;
     tp.n_split = 1;
@@ -757,6 +816,81 @@ pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_
     PW_CUDA(cudaMemsetAsync(h->stat_mass, 0, sizeof(double) * E, s));
   }
   PW_CUDA(cudaStreamSynchronize(s));
+  return PW_OK;
+}
+
+pw_status_t pw_enable_paging(pw_moe_t* h, pw_stream_t stream) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  if (h->paging) return PW_OK;
+  for (int i = 0; i < h->n_blocks; ++i) {
+    if (!h->blk[i].h_planes)
+      return fail(PW_ERR_INVALID_ARG, "block %d: paging needs the host copy of its planes", i);
+    if (h->blk[i].pend_bits)
+      return fail(PW_ERR_STATE, "block %d: a bitwidth change is still pending", i);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaMemPoolProps props = {};
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = h->device;
+  PW_CUDA(cudaMemPoolCreate(&h->pool, &props));
+  const size_t tile = pw::pages::kTileBytes;
+  std::vector<uint32_t*> fresh(h->n_blocks, nullptr);
+  for (int i = 0; i < h->n_blocks; ++i) {
+    auto& b = h->blk[i];
+    const size_t groups = static_cast<size_t>(pw::pages::groups_of(b.rows, b.cols));
+    void* np = nullptr;
+    if (cudaMallocFromPoolAsync(&np, static_cast<size_t>(b.bits) * groups * tile, h->pool, s) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      for (auto q : fresh)
+        if (q) cudaFreeAsync(q, s);
+      cudaStreamSynchronize(s);
+      cudaMemPoolDestroy(h->pool);
+      h->pool = nullptr;
+      return fail(PW_ERR_OOM, "block %d: plane-page pool allocation failed", i);
+    }
+    fresh[i] = static_cast<uint32_t*>(np);
+    PW_CUDA(cudaMemcpy2DAsync(np, b.bits * tile, b.d_planes, b.stride * tile, b.bits * tile, groups,
+                              cudaMemcpyDeviceToDevice, s));
+  }
+  // the copies have landed and no forward issued so far still reads the
+  // caller's storage
+  PW_CUDA(cudaStreamSynchronize(s));
+  if (h->any_forward) PW_CUDA(cudaEventSynchronize(h->fwd_done));
+  for (int i = 0; i < h->n_blocks; ++i) {
+    auto& b = h->blk[i];
+    b.d_planes = fresh[i];
+    b.stride = b.bits;
+    b.owned = true;
+  }
+  h->paging = true;
+  return PW_OK;
+}
+
+pw_status_t pw_resident_bytes(pw_moe_t* h, int64_t* plane_bytes, int64_t* pool_reserved) {
+  if (!h || !plane_bytes) return fail(PW_ERR_INVALID_ARG, "null argument");
+  int64_t total = 0;
+  for (const auto& b : h->blk) {
+    const int64_t groups = pw::pages::groups_of(b.rows, b.cols);
+    const int64_t planes = (b.owned || !h->paging) ? b.stride : 0;
+    total += planes * groups * pw::pages::kTileBytes;
+    if (b.pend_planes) total += static_cast<int64_t>(b.pend_bits) * groups * pw::pages::kTileBytes;
+  }
+  *plane_bytes = total;
+  if (pool_reserved) {
+    *pool_reserved = 0;
+    if (h->pool) {
+      // hand memory the pool no longer uses back to the device first
+      if (h->fwd_done) PW_CUDA(cudaEventSynchronize(h->fwd_done));
+      for (auto& b : h->blk)
+        if (b.pend_bits) PW_CUDA(cudaEventSynchronize(b.ready));
+      PW_CUDA(cudaMemPoolTrimTo(h->pool, 0));
+      cuuint64_t v = 0;
+      PW_CUDA(cudaMemPoolGetAttribute(h->pool, cudaMemPoolAttrReservedMemCurrent, &v));
+      *pool_reserved = static_cast<int64_t>(v);
+    }
+  }
   return PW_OK;
 }
 

@@ -60,6 +60,8 @@ struct BlockRef {
 struct PageTable {
   BlockRef blk[kMaxBlocks];
   uint8_t bits[kMaxBlocks];
+  uint8_t stride[kMaxBlocks];  // planes stored per tile group: n_max for caller
+                               // storage, the resident count for paged storage
 };
 
 // Routing results and per-group token lists, written by the route kernel.
@@ -75,6 +77,7 @@ struct RouteWorkspace {
   float* slot_w;        // [P] routing weight of each sorted position
   int32_t* token_pos;   // [T][k] (+ [T] shared) sorted position of (t, j)
   uint32_t* ticket;     // last-block-done counter (self-resetting)
+  uint32_t* tok_ctr;    // [T] logits written per token (self-resetting)
 };
 
 struct RouteParams {

@@ -17,7 +17,6 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kRouteThreads = 256;
-constexpr int kStageFloats = 4096;  // logits staged in shared memory (16 KB)
 constexpr int kStageSel = 16384;    // selections kept in shared memory (one byte each)
 constexpr int kStageW = 2048;       // routing weights kept in shared memory (8 KB)
 
@@ -25,15 +24,85 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// Top-k and softmax of token t by one warp, once all E logits of t are in
+// global memory: lane i holds experts i + 32 q (q < 4); each of the k rounds
+// is an argmax over the warp under the ranking order (logit descending,
+// index ascending); the softmax denominator is a lane-wise sum met in a xor
+// butterfly.  Lane 0 writes the selections and their weights.
+__device__ void topk_token(const RouteParams& p, int t, int lane) {
+  const int E = p.E, k = p.k;
+  const float* l = p.ws.logits + static_cast<size_t>(t) * E;
+  float v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = lane + 32 * q;
+    v[q] = e < E ? __ldcg(l + e) : 0.0f;
+  }
+  uint32_t taken = 0u;  // bit q: expert lane + 32 q already selected
+  int sel[PW_MAX_TOPK];
+  float lsel[PW_MAX_TOPK];
+#pragma unroll
+  for (int j = 0; j < PW_MAX_TOPK; ++j) {
+    if (j >= k) break;
+    float bv = 0.0f;
+    int bi = -1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = lane + 32 * q;
+      if (e < E && !((taken >> q) & 1u) && (bi < 0 || v[q] > bv)) {
+        bv = v[q];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+      const float ov = __shfl_xor_sync(kFull, bv, m);
+      const int oi = __shfl_xor_sync(kFull, bi, m);
+      if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi >= 0 && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    sel[j] = bi;
+    lsel[j] = bv;
+  }
+  const float mx = lsel[0];
+  float z = 0.0f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (lane + 32 * q < E) z += expf(v[q] - mx);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) z += __shfl_xor_sync(kFull, z, m);
+  if (lane == 0) {
+    float psel[PW_MAX_TOPK];
+    float ssum = 0.0f;
+#pragma unroll
+    for (int j = 0; j < PW_MAX_TOPK; ++j) {
+      if (j >= k) break;
+      psel[j] = expf(lsel[j] - mx) / z;
+      ssum += psel[j];
+    }
+#pragma unroll
+    for (int j = 0; j < PW_MAX_TOPK; ++j) {
+      if (j >= k) break;
+      p.ws.topk_idx[t * k + j] = sel[j];
+      p.ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
+    }
+  }
+}
+
 // One launch.  Phase 1: every warp computes router logits for (token,
 // expert) pairs; lane j owns columns j, j+32, ... and fuses them in
 // ascending order, then the 32 partial sums meet in a xor butterfly
-// (16, 8, 4, 2, 1), so every lane ends with the same value.  Phase 2 runs in
-// the block that finishes last (a ticket counter, no waiting): top-k and
-// softmax with a group of lanes per token (argmax rounds over the group; the
-// softmax denominator is a lane-wise sum met in a xor butterfly), then
-// per-expert counts from warp ballots, one warp-wide scan over the experts,
-// and per-expert token lists ordered by token.
+// (16, 8, 4, 2, 1), so every lane ends with the same value.  A per-token
+// counter finds the warp that writes a token's last logit; that warp takes
+// the token's top-k and softmax at once (topk_token), so the selections of
+// all tokens are made in parallel.  Phase 2 runs in the block that finishes
+// last (a ticket counter, no waiting): per-expert counts from warp ballots
+// over the staged selections, one warp-wide scan over the experts, and
+// per-expert token lists ordered by token; it also puts the counters back
+// to zero for the next launch.
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams p) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -92,7 +161,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
     for (int i = i0; i < H; i += 32) s = __fmaf_rn(bf16_bits_to_f32(xr[i]), wr[i], s);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) s = s + __shfl_xor_sync(kFull, s, m);
-    if (lane == 0) ws.logits[pair] = p.bias ? s + p.bias[e] : s;
+    int last = 0;
+    if (lane == 0) {
+      ws.logits[pair] = p.bias ? s + p.bias[e] : s;
+      __threadfence();
+      last = atomicAdd(ws.tok_ctr + t, 1u) == static_cast<unsigned>(E - 1);
+    }
+    if (__shfl_sync(kFull, last, 0)) {
+      __threadfence();
+      topk_token(p, t, lane);
+    }
   }
 
   __shared__ int s_last;
@@ -103,98 +181,19 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
   if (!s_last) return;
   __threadfence();
 
-  // ---- phase 2 (one block): top-k + softmax, a lane group per token ------
-  // The logits are staged in shared memory a chunk of tokens at a time with
-  // coalesced loads.  A group of L lanes (a power of two with 4 L >= E and
-  // L >= k) serves one token: lane i of the group holds experts i + L q
-  // (q < 4); each of the k rounds is an argmax over the group under the
-  // ranking order (logit descending, index ascending), so every lane of the
-  // group ends with the same selection.  Selections and weights stay in
-  // shared memory for the bucketing below when they fit.
-  __shared__ float s_logits[kStageFloats];
+  // ---- phase 2 (one block): bucketing ------------------------------------
+  // Every token's selections are in global memory; they are staged in shared
+  // memory (one byte each) with coalesced loads, with the weights when they
+  // fit, and the token counters go back to zero for the next launch.
   __shared__ uint8_t s_idx[kStageSel];
   __shared__ float s_w[kStageW];
   const bool sel_staged = T * k <= kStageSel;
   const bool w_staged = T * k <= kStageW;
-  int L = 1;
-  while (4 * L < E || L < k) L <<= 1;
-  const int gl = lane & (L - 1);                       // lane within the group
-  const int gid = warp * (32 / L) + lane / L;          // group index in the block
-  const int n_groups_blk = warps_per_block * (32 / L);
-  const int chunk = kStageFloats / E;  // tokens per staged chunk (>= 32)
-  for (int t0 = 0; t0 < T; t0 += chunk) {
-    const int nt = min(chunk, T - t0);
-    __syncthreads();
-    for (int j = threadIdx.x; j < nt * E; j += kRouteThreads)
-      s_logits[j] = __ldcg(ws.logits + static_cast<size_t>(t0) * E + j);
-    __syncthreads();
-    // rounds are uniform over the block, so every lane takes every shuffle
-    for (int r0 = 0; r0 < nt; r0 += n_groups_blk) {
-      const int tl = r0 + gid;
-      const bool active = tl < nt;
-      const float* l = s_logits + (active ? tl : 0) * E;
-      float v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = gl + L * q;
-        v[q] = (active && e < E) ? l[e] : 0.0f;
-      }
-      uint32_t taken = 0u;  // bit q: expert gl + L q already selected
-      int sel[PW_MAX_TOPK];
-      float lsel[PW_MAX_TOPK];
-#pragma unroll
-      for (int j = 0; j < PW_MAX_TOPK; ++j) {
-        if (j >= k) break;
-        float bv = 0.0f;
-        int bi = -1;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int e = gl + L * q;
-          if (active && e < E && !((taken >> q) & 1u) && (bi < 0 || v[q] > bv)) {
-            bv = v[q];
-            bi = e;
-          }
-        }
-        for (int m = L >> 1; m >= 1; m >>= 1) {
-          const float ov = __shfl_xor_sync(kFull, bv, m);
-          const int oi = __shfl_xor_sync(kFull, bi, m);
-          if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oi < bi))) {
-            bv = ov;
-            bi = oi;
-          }
-        }
-        if (bi >= 0 && (bi & (L - 1)) == gl) taken |= 1u << (bi / L);
-        sel[j] = bi;
-        lsel[j] = bv;
-      }
-      const float mx = lsel[0];
-      float z = 0.0f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (active && gl + L * q < E) z += expf(v[q] - mx);
-      for (int m = L >> 1; m >= 1; m >>= 1) z += __shfl_xor_sync(kFull, z, m);
-      if (active && gl == 0) {
-        const int t = t0 + tl;
-        float psel[PW_MAX_TOPK];
-        float ssum = 0.0f;
-#pragma unroll
-        for (int j = 0; j < PW_MAX_TOPK; ++j) {
-          if (j >= k) break;
-          psel[j] = expf(lsel[j] - mx) / z;
-          ssum += psel[j];
-        }
-#pragma unroll
-        for (int j = 0; j < PW_MAX_TOPK; ++j) {
-          if (j >= k) break;
-          const float w = p.renorm ? psel[j] / ssum : psel[j];
-          ws.topk_idx[t * k + j] = sel[j];
-          ws.topk_w[t * k + j] = w;
-          if (sel_staged) s_idx[t * k + j] = static_cast<uint8_t>(sel[j]);
-          if (w_staged) s_w[t * k + j] = w;
-        }
-      }
-    }
+  for (int j = threadIdx.x; j < T * k; j += kRouteThreads) {
+    if (sel_staged) s_idx[j] = static_cast<uint8_t>(__ldcg(ws.topk_idx + j));
+    if (w_staged) s_w[j] = __ldcg(ws.topk_w + j);
   }
+  for (int t = threadIdx.x; t < T; t += kRouteThreads) ws.tok_ctr[t] = 0u;
   __syncthreads();
   auto sel_of = [&](int t, int j) -> int {
     return sel_staged ? static_cast<int>(s_idx[t * k + j]) : __ldcg(ws.topk_idx + t * k + j);

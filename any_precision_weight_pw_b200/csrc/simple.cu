@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kWarps * 32) simple_kernel(const SimpleParams 
     rows = (proj < 2) ? Fg : p.H;
     cols = (proj < 2) ? p.H : Fg;
     bits = p.pt.bits[blk];
-    n_max = p.n_max;
+    n_max = p.pt.stride[blk];
     planes = p.pt.blk[blk].planes;
     lut = p.pt.blk[blk].lut;
     pos0 = p.offsets[group];

@@ -174,6 +174,7 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
 struct Ctl {
   volatile int* abort;  // shared
   int* err;             // global, may be null
+  unsigned long long wait_ns;  // limit of one wait
 };
 
 // Wait for the phase with the given parity; false on timeout or abort.
@@ -182,7 +183,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, const 
   while (true) {
     if (mbar_try(b, parity)) return true;
     if (*c.abort) return false;
-    if (global_ns() - t0 > kWaitNs) {
+    if (global_ns() - t0 > c.wait_ns) {
       *c.abort = 1;
       if (c.err) atomicExch(c.err, PW_ERR_TIMEOUT);
       return false;
@@ -229,11 +230,14 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 // A fused launch's down item of group g reads h rows that other CTAs' gate/up
 // epilogues write: wait (bounded) until all of g's gate/up items are counted,
 // then order the TMA reads that follow after those writes.
+// (A test switch, p.test_stall_group, makes one group's down items wait for
+// one count more than will ever arrive, so the bounded wait runs out.)
 __device__ __noinline__ bool wait_gate_up(const TcParams& p, int g, int need, const Ctl& c) {
+  if (g == p.test_stall_group) ++need;
   const unsigned long long t0 = global_ns();
   while (ld_acquire_gpu(p.gu_done + g) < need) {
     if (*c.abort) return false;
-    if (global_ns() - t0 > kWaitNs) {
+    if (global_ns() - t0 > c.wait_ns) {
       *c.abort = 1;
       if (c.err) atomicExch(c.err, PW_ERR_TIMEOUT);
       return false;
@@ -355,6 +359,7 @@ struct Pass {
   int blk, bits;
   const uint16_t* lut;
   const uint32_t* planes;  // plane pages (pages.h)
+  int stride;              // planes stored per tile group
 };
 struct Item {
   int g, row0, tok0, ntok, pos0, split, rows, cols, npass, s_begin, s_end;
@@ -442,12 +447,12 @@ __device__ __forceinline__ void decode_item(const TcParams& p, const int* s_pref
 
 // Block, bitwidth, LUT and plane tensor map of pass q of an item.
 __device__ __forceinline__ Pass get_pass(const TcParams& p, const Item& it, int q) {
-  if (p.mode == kTcLinear) return Pass{-1, p.lin_bits, p.lin_lut, p.lin_planes};
+  if (p.mode == kTcLinear) return Pass{-1, p.lin_bits, p.lin_lut, p.lin_planes, p.lin_n_max};
   const int proj = (it.kind == kTcGateUp) ? q
                    : (it.kind == kTcPfGate) ? 0
                    : (it.kind == kTcPfUp) ? 1 : 2;
   const int blk = 3 * it.g + proj;
-  return Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.pt.blk[blk].planes};
+  return Pass{blk, p.pt.bits[blk], p.pt.blk[blk].lut, p.pt.blk[blk].planes, p.pt.stride[blk]};
 }
 
 // ---------------------------------------------------------------- dequant
@@ -778,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   const uint32_t tmem_base = *tmem_holder;
   const int total =
       *s_abort ? 0 : s_prefix[G] + (p.mode == kTcFused ? s_prefix2[G] : 0);
-  const Ctl ctl{s_abort, p.err};
+  const Ctl ctl{s_abort, p.err, p.wait_ns ? p.wait_ns : kWaitNs};
 
   if (warp < 8) {
     // ------------------------------------------------ dequantisers
@@ -834,7 +839,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       uint32_t t = 0, ring_end = 0;
       int gh[2] = {0, 0};
       bool ok = true;
-      const int n_max = (p.mode == kTcLinear) ? p.lin_n_max : p.n_max;
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
         decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
@@ -871,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             const uint32_t bytes = static_cast<uint32_t>(ps.bits) * kSlotBytes;
             mbar_arrive_tx(&sf[e], bytes);
             bulk_load(smem_addr(smem + C::kOffSlots + start * kSlotBytes),
-                      ps.planes + grp_idx * n_max * (kSlotBytes / 4), bytes, &sf[e]);
+                      ps.planes + grp_idx * ps.stride * (kSlotBytes / 4), bytes, &sf[e]);
           }
         }
       }

@@ -51,6 +51,9 @@ struct TcParams {
   int gbuf_ld;
   int* err;                      // device error word (may be null)
   int cooperative;               // fused mode: launch with the cooperative attribute
+  unsigned long long wait_ns;    // limit of one device-side wait (0: 2 s)
+  int test_stall_group;          // test switch: this group's down items wait for
+                                 // a count that never arrives (-1: off)
 };
 
 cudaError_t launch_tc(const TcParams& p, int n_sm, cudaStream_t s);

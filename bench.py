@@ -313,6 +313,82 @@ def uniform_vs_mixed(dev, hbm_peak):
     return out
 
 
+def paging_measure(dev, hbm_peak, T=16, n_fwd=200):
+    """Residency paging on the Mixtral-shaped layer (decode batch 16): the
+    layer switched to library-owned plane storage (only each block's
+    resident planes on the device), then the planner frees 25% and then 50%
+    of the resident plane bytes (damage = synthetic offline sensitivity x
+    the routing mass the library counted over the warm-up forwards), the
+    plan is applied as page moves, and each table is reported as resident
+    plane bytes, pool bytes after a trim, device free memory, and forward
+    tokens/s (back to back, inputs larger than L2)."""
+    import torch
+    from any_precision_weight_pw_b200 import binding, synth
+    wl = synth.WORKLOADS["mixtral_8x7b"]
+    layer = synth.Layer(wl, seed=0)
+    d = binding.upload_synth_layer(layer, max_tokens=T, host_copies=True)
+    d.enable_paging()
+    d._keep[0] = None                      # the caller's plane buffers are released
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    wr = torch.from_numpy(layer.router_w).to(dev)
+    xs = [torch.from_numpy(synth.tokens(wl, T, seed=0, batch=b).view(np.int16)).to(dev)
+          for b in range(N_BATCHES)]
+    ys = [torch.empty_like(x) for x in xs]
+    side = torch.cuda.Stream()
+    rng = np.random.default_rng(0)
+    base = rng.random(wl.n_blocks) + 0.5
+
+    def timed():
+        for i in range(10):
+            d.forward(xs[i % N_BATCHES], wr, None, ys[i % N_BATCHES])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n_fwd):
+            d.forward(xs[i % N_BATCHES], wr, None, ys[i % N_BATCHES])
+        e1.record()
+        torch.cuda.synchronize()
+        d.check_device_error()
+        return e0.elapsed_time(e1) / n_fwd
+
+    rows_out = []
+    d.routing_stats(reset=True)
+    ms = timed()
+    _, mass = d.routing_stats()
+    bits = list(layer.bits)
+    resident0 = None
+    for frac in (0.0, 0.25, 0.5):
+        if frac > 0:
+            blocks = []
+            for blk in range(wl.n_blocks):
+                rows, cols = layer.shape(blk)
+                sens = [0.0] + [float(base[blk]) * 2.0 ** (8 - b) for b in range(1, 9)]
+                blocks.append(dict(bits=bits[blk], min_bits=2,
+                                   plane_bytes=binding.plane_bytes(rows, cols), rows=rows,
+                                   mass=float(mass[blk // 3]), resid=0.0, sens=sens))
+            plan = binding.plan_release(blocks, int(resident0 * frac) - (resident0 - resident))
+            d.set_switch_lag(0)
+            for blk, b in enumerate(plan["bits"]):
+                d.set_block_bits(blk, b, side)
+            bits = plan["bits"]
+            d.forward(xs[0], wr, None, ys[0])
+            torch.cuda.synchronize()
+            ms = timed()
+        resident, reserved = d.resident_bytes(trim=True)
+        if resident0 is None:
+            resident0 = resident
+        free_b, total_b = torch.cuda.mem_get_info(dev)
+        rows_out.append({"released_target": frac, "resident_plane_bytes": int(resident),
+                         "pool_reserved_bytes": int(reserved), "device_free_bytes": int(free_b),
+                         "avg_bits": round(float(np.mean(bits)), 3),
+                         "ms_per_forward": round(ms, 4),
+                         "tokens_per_s": round(T / (ms / 1e3), 1)})
+    d.close()
+    return {"workload": "mixtral_8x7b decode T=%d, paged planes, planner releases 25%% / 50%%" % T,
+            "steps": rows_out}
+
+
 def prefill_measure(dev, steps=5, warmup=2):
     """The Mixtral-shaped layer at prefill scale (4096 tokens, Zipf-skewed
     routing): forward time with CUDA events, tokens/s and achieved TFLOP/s of
@@ -410,6 +486,7 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
         ms = e0.elapsed_time(e1)
+    y0 = ys[0].view(torch.int16).cpu().numpy().view(np.uint16)  # the output for batch 0
     per_launch, n_fwd = d.profile_read()
     d.profile(False)
     launches_per_forward = d.launches(T)
@@ -460,6 +537,7 @@ def run_ours(args, rank, world, local_rank):
     page_move = None
     prefill = None
     uniform = None
+    paging = None
     if rank == 0 and not args.no_sweep:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         cur = (name, layer, d, wr, bias)
@@ -482,11 +560,24 @@ def run_ours(args, rank, world, local_rank):
         page_move = page_move_stress(dev)
         prefill = prefill_measure(dev)
         uniform = uniform_vs_mixed(dev, hbm_peak)
+        paging = paging_measure(dev, hbm_peak)
     else:
         d.close()
 
-    cpu = cpu_baseline(layer, xs_np[0], T) if (rank == 0 and world == 1 and not args.no_cpu) \
-        else None
+    cpu, accuracy = None, None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu, ref = cpu_baseline(layer, xs_np[0], T)
+        # the same tokens' GPU outputs against the oracle's (bf16 output
+        # rounding included in norm_max_rel; arith_excess is what lies beyond
+        # each output's half-ulp)
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from pw_testutil import output_errors
+        yg = (y0[:len(ref)].astype(np.uint32) << 16).view(np.float32)
+        e = output_errors(yg, np.asarray(ref))
+        accuracy = {"tokens": len(ref), "vs": "CPU oracle (float64)",
+                    "norm_max_rel": round(e["norm_max_rel"], 6),
+                    "arith_excess": round(e["arith_excess"], 6),
+                    "rne_mismatch": round(e["rne_mismatch"], 4), "tolerance_ok": e["excess"] <= 0}
     if rank != 0:
         return None
     wl = layer.wl
@@ -519,6 +610,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": traffic,
                      "launch_ms_per_forward": [round(m / max(n_fwd, 1), 5) for m in per_launch]},
         "cpu_baseline": cpu,
+        "accuracy": accuracy,
         "e2e": {"value": round(e2e_tok_s, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(T * wl.hidden * 2),
                 "d2h_bytes_per_step": int(T * wl.hidden * 2)},
@@ -528,6 +620,7 @@ def run_ours(args, rank, world, local_rank):
         "page_move": page_move,
         "prefill": prefill,
         "uniform_vs_mixed": uniform,
+        "paging": paging,
     }
     return out
 
@@ -541,14 +634,17 @@ def cpu_baseline(layer, x_np, T, budget_s=12.0):
     threads = oracle.default_threads()
     L = oracle_layer(oracle, layer)
     done = 0
+    outs = []
     t0 = time.perf_counter()
     while done < T and (time.perf_counter() - t0) < budget_s:
-        L.forward(x_np[done:done + 1], layer.router_w, layer.router_bias, threads=threads)
+        o, _, _ = L.forward(x_np[done:done + 1], layer.router_w, layer.router_bias,
+                            threads=threads)
+        outs.append(o[0])
         done += 1
     dt = time.perf_counter() - t0
-    return {"value": round(done / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": "%d of the %d tokens of one batch, one token per oracle call, %.1f s"
-                      % (done, T, dt)}
+    return ({"value": round(done / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+             "sample": "%d of the %d tokens of one batch, one token per oracle call, %.1f s"
+                       % (done, T, dt)}, outs)
 
 
 def run_reference(args):

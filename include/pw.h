@@ -68,10 +68,19 @@
  *   launches with the gate output kept in a workspace buffer; the result is
  *   the same computation (PW_PREFILL=0/1 in the environment forces either).
  *   At decode both tensor-core passes run in one launch (gate/up items, then
- *   down items, each down item waiting on its expert's gate/up items).
+ *   down items, each down item waiting on its expert's gate/up items).  That
+ *   launch has one CTA per SM and is cooperative: the driver either makes
+ *   every CTA resident at once or refuses the launch (PW_ERR_CUDA), so the
+ *   waits cannot stall on a CTA that never started (for instance when MPS or
+ *   another context holds SMs).
  *   Environment switches, for tests and measurements only: PW_FUSED=0 (two
  *   decode launches), PW_PREFILL=0/1, PW_DOWN_SPLIT=n (K splits of the down
- *   items), PW_FORCE_SIMPLE=1 (CUDA-core kernel; read at pw_moe_create).
+ *   items), PW_FORCE_SIMPLE=1 (CUDA-core kernel; read at pw_moe_create),
+ *   PW_COOP=0 (fused launch without the cooperative attribute), and for the
+ *   failure-detection test PW_TEST_WAIT_US=n (device wait limit, default 2 s)
+ *   with PW_TEST_STALL_GROUP=g (expert g's down items wait for a gate/up count
+ *   that never arrives, so the bounded wait runs out and the forward reports
+ *   PW_ERR_TIMEOUT through pw_check_device_error).
  */
 #ifndef PW_H_
 #define PW_H_
@@ -231,6 +240,35 @@ pw_status_t pw_get_routing(const pw_moe_t* h, int32_t* d_idx, float* d_w,
 pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_t reset,
                              pw_stream_t stream);
 
+/* ---- residency paging --------------------------------------------------- */
+
+/* Switch the handle to library-owned plane storage (PagedWeight,
+ * legiblepapers "Summary & Methodology Analysis": the bit-plane buffers are
+ * GPU-resident pages that are reloaded or offloaded asynchronously; cortexa
+ * abstract: freeing weight memory for the KV cache).  Every block then holds
+ * exactly its current bitwidth's planes on the device, in the paged layout
+ * with that many planes per tile group, in a memory pool the library
+ * creates on the handle's device.  Lowering a block's width offloads planes
+ * (new storage with fewer planes replaces the old one, which is freed to
+ * the pool once no issued forward can read it); raising it reloads planes
+ * from the host master copy, so every block needs h_planes (else
+ * PW_ERR_INVALID_ARG).  The switch semantics of pw_set_block_bits are
+ * unchanged; a pool allocation that fails there is PW_ERR_OOM with nothing
+ * changed.  The call copies the resident planes out of the caller's
+ * d_planes on stream and returns after those copies and every forward
+ * issued so far have finished: the caller may then free its plane buffers
+ * (the LUT slots stay caller-owned).  PW_ERR_STATE while a bitwidth change
+ * is pending.  Idempotent. */
+pw_status_t pw_enable_paging(pw_moe_t* h, pw_stream_t stream);
+
+/* Device bytes of plane pages the handle keeps resident (a block's
+ * resident planes x its plane page size, plus the storage of pending
+ * changes; without paging, n_max planes per block).  If pool_reserved is
+ * not NULL, the call first waits for the handle's issued work, returns the
+ * pool's unused memory to the device (cudaMemPoolTrimTo) and reports what
+ * the pool still reserves. */
+pw_status_t pw_resident_bytes(pw_moe_t* h, int64_t* plane_bytes, int64_t* pool_reserved);
+
 /* ---- the quality-aware release planner (host only) --------------------- */
 
 /* One linear-block as the planner sees it. */
@@ -310,7 +348,7 @@ int32_t pw_forward_launches(const pw_moe_t* h, int32_t T);
  * the caller serialises calls per device, e.g. by issuing them all on one
  * stream. */
 #define PW_ROUTE_STATIC_MAX_TOKENS 256
-#define PW_ROUTE_STATIC_SCRATCH_BYTES 156672 /* logits 128 KB + lists and counter */
+#define PW_ROUTE_STATIC_SCRATCH_BYTES 157696 /* logits 128 KB + lists and counters */
 pw_status_t pw_route_static(const uint16_t* d_x, const float* d_router_w,
                             const float* d_router_bias, int32_t T, int32_t hidden,
                             int32_t n_experts, int32_t top_k, int32_t renorm_topk,

@@ -8,7 +8,9 @@ where y_ref is the oracle's float64 result.  The first term is the rounding
 of a correctly rounded bf16 output (the output format's own error); the
 second is the 2e-3 budget for the path's arithmetic, taken relative to the
 largest output because a per-element relative error is ill-conditioned at
-outputs near zero.
+outputs near zero.  output_errors also reports that arithmetic part on its
+own (arith_excess) and how often the output differs from the correctly
+rounded oracle value (rne_mismatch).
 """
 import numpy as np
 
@@ -20,15 +22,33 @@ def bf16_half_ulp(v):
     return 2.0 ** (np.floor(np.log2(a)) - 8)
 
 
+def bf16_round(v):
+    """Round float64 values to the nearest bf16 (ties to even), as float64
+    (normal range; the outputs here are far from under- and overflow)."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    ulp = 2.0 ** (np.floor(np.log2(a)) - 7)
+    return np.round(v / ulp) * ulp      # v / ulp is exact; np.round ties to even
+
+
 def output_errors(y_gpu, y_ref):
+    """norm_max_rel: max |y_gpu - y_ref| / max |y_ref|, the bf16 output
+    rounding included (alone it can reach 2^-8 of scale when the largest
+    output sits just above a power of two).  arith_excess: the largest error
+    beyond the output's own half-ulp, / max |y_ref| -- a bound on the path's
+    arithmetic error before the final rounding.  rne_mismatch: the fraction
+    of outputs that differ from the correctly rounded oracle value."""
     y_gpu = np.asarray(y_gpu, dtype=np.float64)
     y_ref = np.asarray(y_ref, dtype=np.float64)
     scale = float(np.max(np.abs(y_ref))) if y_ref.size else 0.0
     err = np.abs(y_gpu - y_ref)
-    bound = bf16_half_ulp(np.maximum(np.abs(y_ref), np.abs(y_gpu))) + REL_TOL * scale
+    half = bf16_half_ulp(np.maximum(np.abs(y_ref), np.abs(y_gpu)))
+    bound = half + REL_TOL * scale
     return {
         "max_abs": float(err.max()) if err.size else 0.0,
         "norm_max_rel": float(err.max() / scale) if scale > 0 else 0.0,
+        "arith_excess": float(max(0.0, (err - half).max()) / scale) if scale > 0 else 0.0,
+        "rne_mismatch": float(np.mean(y_gpu != bf16_round(y_ref))) if y_ref.size else 0.0,
         "rel_l2": float(np.linalg.norm(err) / max(np.linalg.norm(y_ref), 1e-300)),
         "excess": float((err - bound).max()) if err.size else -1.0,
     }

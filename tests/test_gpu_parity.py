@@ -523,3 +523,143 @@ def test_routing_stats_accumulate_over_forwards(pw, oracle, name, T, n_fwd):
     c2, m2 = dev.routing_stats()
     assert not c2.any() and not m2.any()
     dev.close()
+
+
+def _plane_total(pw, layer, bits):
+    return sum(b * pw.plane_bytes(*layer.shape(blk)) for blk, b in enumerate(bits))
+
+
+def test_paging_offload_reload_parity(pw, oracle):
+    """Library-owned plane storage: after pw_enable_paging the caller's plane
+    buffers are overwritten with garbage and the layer still matches the
+    oracle; lowering widths offloads planes (resident bytes fall by exactly
+    the released plane pages), raising them reloads planes from the host
+    copies, and every forward matches the oracle at the widths it used."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=11)
+    dev = pw.upload_synth_layer(layer, max_tokens=16, host_copies=True)
+    dev.set_switch_lag(0)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    side = torch.cuda.Stream()
+    assert dev.resident_bytes()[0] == 8 * _plane_total(pw, layer, [1] * wl.n_blocks)
+    dev.enable_paging()
+    bits = list(layer.bits)
+    assert dev.resident_bytes()[0] == _plane_total(pw, layer, bits)
+    for t in dev._keep[0]:                 # the caller's plane buffers
+        t.fill_(-1)
+    torch.cuda.synchronize()
+
+    def check(f):
+        x = synth.tokens(wl, 16, seed=11, batch=f)
+        y = dev.forward(_dev_bf16(x), wr)
+        used = dev.forward_bits()
+        torch.cuda.synchronize()
+        ref, _, _ = oracle_layer(oracle, layer, used).forward(x, layer.router_w, threads=8)
+        assert_output_close(_to_f32(y), ref)
+        return used
+
+    assert check(0) == bits
+    down = {0: 1, 1: 2, 5: 1, 9: 2, 16: 1, 23: 2}
+    for blk, b in down.items():
+        dev.set_block_bits(blk, b, side)
+        bits[blk] = b
+    assert check(1) == bits
+    assert dev.resident_bytes()[0] == _plane_total(pw, layer, bits)
+    up = {0: 8, 5: 6, 9: 3, 12: 7}
+    for blk, b in up.items():
+        dev.set_block_bits(blk, b, side)
+        bits[blk] = b
+    assert check(2) == bits
+    assert check(3) == bits
+    plane, reserved = dev.resident_bytes(trim=True)
+    assert plane == _plane_total(pw, layer, bits) and reserved >= plane
+    dev.check_device_error()
+    dev.close()
+
+
+def test_paging_planner_frees_device_memory(pw, oracle):
+    """Qwen-shaped layer with paging: routing mass from the library's own
+    counters over 20 forwards, the planner frees a quarter of the resident
+    plane bytes, the plan is applied as page moves, and (a) resident bytes
+    fall by what the planner released in plane pages, (b) the pool still
+    covers what stays resident after a trim, (c) the next forwards match the oracle
+    at the widths they used.  (The pool reserves memory in 2 MB mappings,
+    so how much of the released bytes it can hand back depends on
+    fragmentation; only the accounting is exact.)"""
+    wl = synth.WORKLOADS["qwen15_moe_a27b"]
+    layer = synth.Layer(wl, seed=12)
+    T = 32
+    dev = pw.upload_synth_layer(layer, max_tokens=T, host_copies=True)
+    dev.enable_paging()
+    for t in dev._keep[0]:
+        t.fill_(-1)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    for f in range(20):
+        dev.forward(_dev_bf16(synth.tokens(wl, T, seed=12, batch=f)), wr)
+    counts, mass = dev.routing_stats()
+    resident0, reserved0 = dev.resident_bytes(trim=True)
+    rng = np.random.default_rng(12)
+    blocks = []
+    for blk in range(wl.n_blocks):
+        rows, cols = layer.shape(blk)
+        e = blk // 3
+        sens = [0.0] + [float(rng.random() + 0.5) * 2.0 ** (8 - b) for b in range(1, 9)]
+        blocks.append(dict(bits=layer.bits[blk], min_bits=2, plane_bytes=pw.plane_bytes(rows, cols),
+                           rows=rows, mass=float(mass[e]) if e < wl.n_experts else 20.0 * T,
+                           resid=0.0, sens=sens))
+    plan = pw.plan_release(blocks, resident0 // 4)
+    assert plan["reached"] and plan == oracle.plan_greedy(blocks, resident0 // 4)
+    side = torch.cuda.Stream()
+    dev.set_switch_lag(0)
+    for blk, b in enumerate(plan["bits"]):
+        dev.set_block_bits(blk, b, side)
+    x = synth.tokens(wl, T, seed=12, batch=99)
+    y = dev.forward(_dev_bf16(x), wr)
+    used = dev.forward_bits()
+    assert used == plan["bits"]
+    torch.cuda.synchronize()
+    released_planes = sum((layer.bits[i] - b) * blocks[i]["plane_bytes"]
+                          for i, b in enumerate(plan["bits"]))
+    resident1, reserved1 = dev.resident_bytes(trim=True)
+    assert resident1 == resident0 - released_planes
+    assert 0 < reserved1 and resident1 <= reserved1
+    ref, _, _ = oracle_layer(oracle, layer, used).forward(x, layer.router_w, threads=32)
+    assert_output_close(_to_f32(y), ref)
+    dev.check_device_error()
+    dev.close()
+
+
+def test_bounded_wait_times_out_and_the_handle_recovers(pw, oracle):
+    """Failure detection without a fault: with the test switches, one
+    expert's down items in the fused decode launch wait for a gate/up count
+    that never arrives, under a 5 ms limit.  The wait gives up, every role of
+    the CTA drains what it has in flight, the kernel returns, and
+    pw_check_device_error reports PW_ERR_TIMEOUT once (then the word is
+    clear).  The same handle's next forward, switches off, matches the
+    oracle."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=0)
+    dev = pw.upload_synth_layer(layer, max_tokens=16)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    x = synth.tokens(wl, 16, seed=0)
+    idx_ref, _ = oracle.topk_softmax(oracle.router_logits(x, layer.router_w, None), wl.top_k,
+                                     bool(wl.renorm_topk))
+    stalled = int(idx_ref[0, 0])            # an expert with routed tokens
+    os.environ["PW_TEST_WAIT_US"] = "5000"
+    os.environ["PW_TEST_STALL_GROUP"] = str(stalled)
+    try:
+        dev.forward(_dev_bf16(x), wr)
+        torch.cuda.synchronize()
+    finally:
+        os.environ.pop("PW_TEST_WAIT_US", None)
+        os.environ.pop("PW_TEST_STALL_GROUP", None)
+    with pytest.raises(pw.PwError) as e:
+        dev.check_device_error()
+    assert e.value.status == 4                 # PW_ERR_TIMEOUT
+    dev.check_device_error()                   # cleared
+    y = dev.forward(_dev_bf16(x), wr)
+    torch.cuda.synchronize()
+    dev.check_device_error()
+    ref, _, _ = oracle_layer(oracle, layer).forward(x, layer.router_w, threads=8)
+    assert_output_close(_to_f32(y), ref)
+    dev.close()

@@ -168,3 +168,19 @@ def test_dense_restatement_matches(oracle):
     want = Ws[2] @ (g / (1 + np.exp(-g)) * u)
     y, _ = layer.expert_ffn(0, x)
     np.testing.assert_allclose(y, want, rtol=1e-10, atol=1e-14)
+
+
+def test_bf16_round_helper():
+    """The tests' bf16 rounding of oracle outputs: exact values stay, halfway
+    cases go to the even significand, and it agrees with a float32 round
+    trip through the bf16 bit pattern on random values."""
+    import pw_testutil as tu
+    assert tu.bf16_round(np.array([1.0, -3.0, 0.5]))[:].tolist() == [1.0, -3.0, 0.5]
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to even -> 1
+    assert tu.bf16_round(np.array([1.0 + 2.0 ** -8]))[0] == 1.0
+    # 1 + 3 * 2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: -> 1 + 2^-6
+    assert tu.bf16_round(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2.0 ** -6
+    rng = np.random.default_rng(1)
+    v = rng.normal(size=1000).astype(np.float32)
+    want = synth.bf16_bits_to_float(synth.to_bf16_bits(v)).astype(np.float64)
+    np.testing.assert_array_equal(tu.bf16_round(v.astype(np.float64)), want)
