@@ -24,7 +24,7 @@ EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy"
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
             "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
             "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats", "pw_plan_release",
-            "pw_enable_paging", "pw_resident_bytes",
+            "pw_enable_paging", "pw_resident_bytes", "pw_workspace_bytes",
             "pw_last_error", "pw_abi_version"]
 
 
@@ -74,6 +74,7 @@ def lib():
         L.pw_set_switch_lag.argtypes = [P, i32]
         L.pw_routing_stats.argtypes = [P, P, P, i32, P]
         L.pw_enable_paging.argtypes = [P, P]
+        L.pw_workspace_bytes.argtypes = [C.POINTER(Config), C.POINTER(C.c_int64)]
         L.pw_resident_bytes.argtypes = [P, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.pw_plan_release.argtypes = [C.POINTER(PlanBlock), i32, C.c_int64, C.POINTER(i32),
                                       C.POINTER(C.c_int64), C.POINTER(C.c_double),
@@ -159,6 +160,15 @@ def route_static(x, router_w, top_k: int, renorm_topk: int, router_bias=None, id
     check(lib().pw_route_static(_ptr(x), _ptr(router_w), _ptr(router_bias), T, H, E, top_k,
                                 renorm_topk, _ptr(idx), _ptr(w), _stream(stream)))
     return idx, w
+
+
+def workspace_bytes(cfg: dict) -> int:
+    """Device workspace bytes a layer with this config allocates."""
+    c = Config(cfg["hidden"], cfg["ffn"], cfg["n_experts"], cfg["top_k"], cfg["shared_ffn"],
+               cfg["n_max"], cfg["renorm_topk"], cfg["max_tokens"])
+    out = C.c_int64()
+    check(lib().pw_workspace_bytes(C.byref(c), C.byref(out)))
+    return out.value
 
 
 def plan_release(blocks, target_bytes: int):

@@ -2,11 +2,13 @@
 // per-block page table, the asynchronous bitwidth switch, workspace and the
 // launch sequence of one forward.
 //
-// PagedWeight (legiblepapers summary, "Summary & Methodology Analysis"): the
-// bit-plane and LUT buffers are GPU-resident pages reloaded or offloaded
-// asynchronously to hide latency; (arxivlens abstract) asynchronous page
-// movement overlaps with serving.  Here a bitwidth change is a page move on a
-// side stream that the forward after next waits for (see pw_set_block_bits).
+// PagedWeight (legiblepapers summary, "Summary & Methodology Analysis"; the
+// arxivlens abstract): the bit-plane and LUT buffers are GPU-resident pages
+// that move between host and device asynchronously while the layer keeps
+// serving.  Here a bitwidth change is a page move on a side stream; a
+// forward uses the new width once it finds the move complete, or waits for
+// it after a bounded number of forwards (see pw_set_block_bits); with paging
+// on, lowering a width also frees the dropped planes' device memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -167,7 +169,9 @@ struct pw_moe {
   double* stat_mass = nullptr;               // [E]
   uint16_t* stage_x = nullptr;
   uint16_t* stage_y = nullptr;
-  int P_max = 0, gu_stride = 0, max_split = 8, last_T = 0;
+  int P_max = 0, gu_stride = 0, last_T = 0;
+  size_t ys_floats = 0;   // capacity of the down partials (shared with gbuf)
+  size_t ws_bytes = 0;
   bool tc = false;  // both expert passes on the tensor-core kernel
   void* ws_base = nullptr;
   // per-launch timing (pw_profile_*): 5 events per forward bracket 4 launches
@@ -205,21 +209,107 @@ void free_all(pw_moe* h) {
   delete h;
 }
 
+constexpr int kMaxSplit = 8;  // K splits of the down pass at most
+
 // K splits of the down items: enough items for `per_sm` rounds of the grid
 // (more in the fused launch, where down items also fill the gate/up tail).
-int down_splits(const pw_moe* h, int T, int per_sm) {
-  const pw_moe_config_t& c = h->cfg;
-  const int forced = env_int("PW_DOWN_SPLIT", 0);
-  if (forced > 0) return forced < h->max_split ? forced : h->max_split;
+int splits_for(const pw_moe_config_t& c, int n_sm, int T, int per_sm) {
   const int row_tiles = (c.hidden + 127) / 128;
   int groups = T * c.top_k < c.n_experts ? T * c.top_k : c.n_experts;
   if (c.shared_ffn > 0) groups += 1;
   const int items = row_tiles * groups;
-  int ns = (per_sm * h->n_sm + items - 1) / items;
+  int ns = (per_sm * n_sm + items - 1) / items;
   const int stages = ((c.ffn + 31) / 32 + 7) / 8;
   if (ns > stages) ns = stages;
-  if (ns > h->max_split) ns = h->max_split;
+  if (ns > kMaxSplit) ns = kMaxSplit;
   if (ns < 1) ns = 1;
+  return ns;
+}
+
+// Sorted positions of a forward of T tokens (routed slots + shared rows).
+size_t positions(const pw_moe_config_t& c, int T) {
+  return static_cast<size_t>(T) * c.top_k + (c.shared_ffn > 0 ? T : 0);
+}
+
+// The prefill passes are the default when the routed slots average at least
+// 64 tokens per expert.
+bool prefill_default(const pw_moe_config_t& c, int T) {
+  return static_cast<long long>(T) * c.top_k >= 64ll * c.n_experts;
+}
+
+// The workspace of a handle: one allocation, every piece 256-byte aligned.
+// The down pass's per-split partials and the prefill gate outputs share one
+// region (the gate outputs are dead once the up pass has run, before the
+// down pass writes), sized for the larger of: one split of every position
+// at max_tokens, the splits the decode passes choose at each token count
+// they serve, and the prefill gate outputs.
+struct Layout {
+  bool tc = false, pf = false;
+  int P_max = 0, gu_stride = 0, x_ld = 0, h_perm_ld = 0, gbuf_ld = 0;
+  size_t ys_floats = 0;
+  size_t o_logits, o_tki, o_tkw, o_off, o_st, o_sw, o_tp, o_tk, o_tc, o_err, o_gd, o_sc, o_sm,
+      o_gu, o_xp, o_hp, o_ys, o_sx, o_sy, total;
+};
+
+Layout make_layout(const pw_moe_config_t& c, int n_sm) {
+  Layout L;
+  const int T = c.max_tokens, E = c.n_experts, k = c.top_k, S = c.shared_ffn;
+  const int G = E + (S > 0 ? 1 : 0);
+  L.P_max = static_cast<int>(positions(c, T));
+  const int Fmax = c.ffn > S ? c.ffn : S;
+  L.tc = tc_shape_ok(c.hidden) && tc_shape_ok(c.ffn) && (S == 0 || tc_shape_ok(S)) &&
+         env_int("PW_FORCE_SIMPLE", 0) == 0;
+  L.gu_stride = L.tc ? 0 : 2 * Fmax;
+  // rows padded to whole 256-column stages, zero past the end
+  L.x_ld = L.tc ? (c.hidden + 255) / 256 * 256 : 0;
+  L.h_perm_ld = L.tc ? (Fmax + 255) / 256 * 256 : 0;
+  L.pf = L.tc && L.P_max >= pw::kTcPfTokens;
+  L.gbuf_ld = L.pf ? Fmax : 0;
+  size_t ys = static_cast<size_t>(L.P_max) * c.hidden;
+  if (L.tc)
+    for (int t = 1; t <= T; ++t) {
+      if (L.pf && prefill_default(c, t)) break;
+      int ns = splits_for(c, n_sm, t, 6);
+      const int ns4 = splits_for(c, n_sm, t, 4);
+      if (ns4 > ns) ns = ns4;
+      const size_t need = ns * positions(c, t) * c.hidden;
+      if (need > ys) ys = need;
+    }
+  const size_t gb = static_cast<size_t>(L.P_max) * L.gbuf_ld;
+  L.ys_floats = ys;
+  auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
+  size_t off = 0;
+  L.o_logits = off; off += al(sizeof(float) * T * E);
+  L.o_tki = off; off += al(sizeof(int32_t) * T * k);
+  L.o_tkw = off; off += al(sizeof(float) * T * k);
+  L.o_off = off; off += al(sizeof(int32_t) * (G + 1));
+  L.o_st = off; off += al(sizeof(int32_t) * L.P_max);
+  L.o_sw = off; off += al(sizeof(float) * L.P_max);
+  L.o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
+  L.o_tk = off; off += al(sizeof(uint32_t) * 4);
+  L.o_tc = off; off += al(sizeof(uint32_t) * T);
+  L.o_err = off; off += al(sizeof(int) * 4);
+  L.o_gd = off; off += al(sizeof(int) * (G + 1));
+  L.o_sc = off; off += al(sizeof(unsigned long long) * E);
+  L.o_sm = off; off += al(sizeof(double) * E);
+  L.o_gu = off; off += al(sizeof(float) * size_t(L.P_max) * L.gu_stride);
+  L.o_xp = off; off += al(sizeof(uint16_t) * size_t(L.P_max) * L.x_ld);
+  L.o_hp = off; off += al(sizeof(uint16_t) * size_t(L.P_max) * L.h_perm_ld);
+  L.o_ys = off; off += al(sizeof(float) * (ys > gb ? ys : gb));
+  L.o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
+  L.o_sy = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
+  L.total = off;
+  return L;
+}
+
+// Splits of the down pass for a forward of T tokens: the automatic choice
+// (or PW_DOWN_SPLIT), never more than the partials region holds.
+int down_splits(const pw_moe* h, int T, int per_sm) {
+  const int forced = env_int("PW_DOWN_SPLIT", 0);
+  int ns = forced > 0 ? (forced < kMaxSplit ? forced : kMaxSplit)
+                      : splits_for(h->cfg, h->n_sm, T, per_sm);
+  const size_t per_split = positions(h->cfg, T) * h->cfg.hidden;
+  while (ns > 1 && ns * per_split > h->ys_floats) --ns;
   return ns;
 }
 
@@ -229,7 +319,7 @@ bool use_prefill(const pw_moe* h, int T) {
   if (!h->pf) return false;
   const int forced = env_int("PW_PREFILL", -1);
   if (forced >= 0) return forced != 0;
-  return static_cast<long long>(T) * h->cfg.top_k >= 64ll * h->cfg.n_experts;
+  return prefill_default(h->cfg, T);
 }
 
 }  // namespace
@@ -237,6 +327,18 @@ bool use_prefill(const pw_moe* h, int T) {
 extern "C" {
 
 int32_t pw_abi_version(void) { return PW_ABI_VERSION; }
+
+pw_status_t pw_workspace_bytes(const pw_moe_config_t* cfg, int64_t* bytes) {
+  if (!cfg || !bytes) return fail(PW_ERR_INVALID_ARG, "null argument");
+  if (cfg->max_tokens < 1 || cfg->hidden < 8 || cfg->n_experts < 1 || cfg->top_k < 1 ||
+      cfg->ffn < 1 || cfg->shared_ffn < 0)
+    return fail(PW_ERR_INVALID_ARG, "bad config");
+  int dev = 0, n_sm = 0;
+  PW_CUDA(cudaGetDevice(&dev));
+  PW_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  *bytes = static_cast<int64_t>(make_layout(*cfg, n_sm).total);
+  return PW_OK;
+}
 const char* pw_last_error(void) { return g_err.c_str(); }
 
 pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blocks,
@@ -306,40 +408,21 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   }
 
   // workspace, one allocation
-  const int T = c.max_tokens, E = c.n_experts, k = c.top_k;
-  const int S = c.shared_ffn;
-  h->P_max = T * k + (S > 0 ? T : 0);
-  const int Fmax = c.ffn > S ? c.ffn : S;
-  h->tc = tc_shape_ok(c.hidden) && tc_shape_ok(c.ffn) && (S == 0 || tc_shape_ok(S)) &&
-          env_int("PW_FORCE_SIMPLE", 0) == 0;
-  h->gu_stride = h->tc ? 0 : 2 * Fmax;
-  // rows padded to whole 256-column stages, zero past the end
-  h->x_ld = h->tc ? (c.hidden + 255) / 256 * 256 : 0;
-  h->h_perm_ld = h->tc ? (Fmax + 255) / 256 * 256 : 0;
-  auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
-  size_t off = 0;
-  const size_t o_logits = off; off += al(sizeof(float) * T * E);
-  const size_t o_tki = off; off += al(sizeof(int32_t) * T * k);
-  const size_t o_tkw = off; off += al(sizeof(float) * T * k);
-  const size_t o_off = off; off += al(sizeof(int32_t) * (h->G + 1));
-  const size_t o_st = off; off += al(sizeof(int32_t) * h->P_max);
-  const size_t o_sw = off; off += al(sizeof(float) * h->P_max);
-  const size_t o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
-  const size_t o_tk = off; off += al(sizeof(uint32_t) * 4);
-  const size_t o_tc = off; off += al(sizeof(uint32_t) * T);
-  const size_t o_err = off; off += al(sizeof(int) * 4);
-  const size_t o_gd = off; off += al(sizeof(int) * (h->G + 1));
-  const size_t o_sc = off; off += al(sizeof(unsigned long long) * E);
-  const size_t o_sm = off; off += al(sizeof(double) * E);
-  const size_t o_gu = off; off += al(sizeof(float) * size_t(h->P_max) * h->gu_stride);
-  const size_t o_xp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->x_ld);
-  const size_t o_hp = off; off += al(sizeof(uint16_t) * size_t(h->P_max) * h->h_perm_ld);
-  const size_t o_ys = off; off += al(sizeof(float) * size_t(h->max_split) * h->P_max * c.hidden);
-  h->pf = h->tc && h->P_max >= pw::kTcPfTokens;
-  h->gbuf_ld = h->pf ? Fmax : 0;
-  const size_t o_gb = off; off += al(sizeof(float) * size_t(h->P_max) * h->gbuf_ld);
-  const size_t o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
-  const size_t o_sy = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
+  const Layout L = make_layout(c, h->n_sm);
+  h->P_max = L.P_max;
+  h->tc = L.tc;
+  h->pf = L.pf;
+  h->gu_stride = L.gu_stride;
+  h->x_ld = L.x_ld;
+  h->h_perm_ld = L.h_perm_ld;
+  h->gbuf_ld = L.gbuf_ld;
+  h->ys_floats = L.ys_floats;
+  h->ws_bytes = L.total;
+  const size_t o_logits = L.o_logits, o_tki = L.o_tki, o_tkw = L.o_tkw, o_off = L.o_off,
+               o_st = L.o_st, o_sw = L.o_sw, o_tp = L.o_tp, o_tk = L.o_tk, o_tc = L.o_tc,
+               o_err = L.o_err, o_gd = L.o_gd, o_sc = L.o_sc, o_sm = L.o_sm, o_gu = L.o_gu,
+               o_xp = L.o_xp, o_hp = L.o_hp, o_ys = L.o_ys, o_sx = L.o_sx, o_sy = L.o_sy;
+  const size_t off = L.total;
   if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
     free_all(h);
     return fail(PW_ERR_OOM, "workspace allocation of %zu bytes failed", off);
@@ -362,10 +445,10 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->x_sorted = reinterpret_cast<uint16_t*>(w + o_xp);
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
   h->ysorted = reinterpret_cast<float*>(w + o_ys);
-  h->gbuf = reinterpret_cast<float*>(w + o_gb);
+  h->gbuf = reinterpret_cast<float*>(w + o_ys);  // shares the partials region
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
   h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
-  if (cudaMemset(w + o_tk, 0, o_sm + al(sizeof(double) * E) - o_tk) != cudaSuccess ||
+  if (cudaMemset(w + o_tk, 0, o_gu - o_tk) != cudaSuccess ||
       cudaMemset(w + o_xp, 0, o_sx - o_xp) != cudaSuccess) {
     free_all(h);
     return fail(PW_ERR_CUDA, "cudaMemset failed");
@@ -516,6 +599,9 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   }
   const int has_shared = c.shared_ffn > 0 ? 1 : 0;
   const bool prefill = h->tc && use_prefill(h, T);
+  // the down partials of split s start at s * split_stride: this forward's
+  // positions times H, so the splits down_splits allows fit the region
+  const long long split_stride = static_cast<long long>(positions(c, T)) * c.hidden;
   // decode: gate/up and down in one launch (PW_FUSED=0 splits them)
   const bool fused = h->tc && !prefill && env_int("PW_FUSED", 1) != 0;
   std::vector<cudaEvent_t> evs;
@@ -592,6 +678,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
       tp.wait_ns = static_cast<unsigned long long>(env_int("PW_TEST_WAIT_US", 0)) * 1000ull;
       tp.test_stall_group = env_int("PW_TEST_STALL_GROUP", -1);
       tp.n_split = down_splits(h, T, 6);
+      if (static_cast<size_t>(tp.n_split) * split_stride > h->ys_floats)
+        return fail(PW_ERR_STATE, "down partials (%d splits) exceed the workspace", tp.n_split);
       // down items wait on other CTAs' gate/up items, so every CTA must be
       // resident: the launch is cooperative (refused rather than stalled when
       // the grid cannot be co-resident); PW_COOP=0 drops the attribute
@@ -599,7 +687,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
       for (int i = 0; i < 4; ++i) tp.h_maps[i] = h->h_maps[i];
       tp.gu_done = h->gu_done;
       tp.ysorted = h->ysorted;
-      tp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
+      tp.split_stride = split_stride;
     }
     if (prefill) {
       // gate -> g (fp32), then up -> h = silu(g) * u
@@ -637,6 +725,8 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     n_split = down_splits(h, T, 6);  // the down items ran in the launch above
   } else if (h->tc) {
     n_split = prefill ? 1 : down_splits(h, T, 4);
+    if (static_cast<size_t>(n_split) * split_stride > h->ys_floats)
+      return fail(PW_ERR_STATE, "down partials (%d splits) exceed the workspace", n_split);
     pw::TcParams tp;
     std::memset(&tp, 0, sizeof(tp));
     tp.test_stall_group = -1;
@@ -657,7 +747,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_perm = h->h_perm;
     tp.h_perm_ld = h->h_perm_ld;
     tp.ysorted = h->ysorted;
-    tp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
+    tp.split_stride = split_stride;
     tp.err = h->err;
     PW_CUDA(pw::launch_tc(tp, h->n_sm, s));
   } else {
@@ -689,7 +779,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   cp.k = c.top_k;
   cp.has_shared = has_shared;
   cp.n_split = n_split;
-  cp.split_stride = static_cast<long long>(h->P_max) * c.hidden;
+  cp.split_stride = split_stride;
   PW_CUDA(pw::launch_combine(cp, s));
   PW_CUDA(mark(4));
   if (h->profiling) h->ev_pending.push_back(evs);

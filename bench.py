@@ -557,10 +557,11 @@ def run_ours(args, rank, world, local_rank):
             del xs2, ys2
         cur[2].close()
         del flush
-        page_move = page_move_stress(dev)
-        prefill = prefill_measure(dev)
-        uniform = uniform_vs_mixed(dev, hbm_peak)
-        paging = paging_measure(dev, hbm_peak)
+        if not args.quick:
+            page_move = page_move_stress(dev)
+            prefill = prefill_measure(dev)
+            uniform = uniform_vs_mixed(dev, hbm_peak)
+            paging = paging_measure(dev, hbm_peak)
     else:
         d.close()
 
@@ -616,6 +617,10 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": int(T * wl.hidden * 2)},
         "clocks": clk.summary(t_begin, t_end),
         "gpu_launches": launches,
+        "workspace_bytes": {"headline_max_tokens_64": int(binding.workspace_bytes(
+                                dict(d.cfg, max_tokens=64))),
+                            "mixtral_max_tokens_4096": int(binding.workspace_bytes(
+                                dict(d.cfg, max_tokens=4096)))},
         "sweep": sweep,
         "page_move": page_move,
         "prefill": prefill,
@@ -724,6 +729,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="headline and decode sweep only (no page-move, prefill, uniform-width "
+                         "and paging measurements)")
     ap.add_argument("--prefill", action="store_true",
                     help="only the prefill-scale measurement (one JSON object; for profiling)")
     args = ap.parse_args()

@@ -138,7 +138,8 @@ typedef struct {
 } pw_block_desc_t;
 
 /* Create a layer over caller-owned pages.  blocks has 3*E (+3 if S > 0)
- * entries in block-id order.  Allocates the workspace on the current device. */
+ * entries in block-id order.  Allocates the workspace on the current device
+ * (pw_workspace_bytes gives its size). */
 pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blocks,
                           int32_t n_blocks, pw_moe_t** out);
 
@@ -171,6 +172,13 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
 pw_status_t pw_moe_forward(pw_moe_t* h, const uint16_t* d_x, int32_t T,
                            const float* d_router_w, const float* d_router_bias,
                            uint16_t* d_y, pw_stream_t stream);
+
+/* Bytes of device workspace pw_moe_create allocates for cfg on the current
+ * device (one allocation: routing lists, gathered activations, the SwiGLU
+ * activations, the down pass's per-split partials -- shared with the
+ * prefill gate outputs, which are dead by the time the down pass writes --
+ * and the host-forward staging rows).  No allocation is made. */
+pw_status_t pw_workspace_bytes(const pw_moe_config_t* cfg, int64_t* bytes);
 
 /* Free the workspace and events after all work of the handle has finished
  * (synchronises on the handle's events).  NULL is accepted. */

@@ -663,3 +663,26 @@ def test_bounded_wait_times_out_and_the_handle_recovers(pw, oracle):
     ref, _, _ = oracle_layer(oracle, layer).forward(x, layer.router_w, threads=8)
     assert_output_close(_to_f32(y), ref)
     dev.close()
+
+
+def test_workspace_is_sized_to_its_use(pw):
+    """The workspace query matches what a handle allocates, and a
+    Mixtral-shaped layer able to run 4096-token prefill needs well under a
+    gigabyte: the down partials are sized for the splits the passes use and
+    share their region with the prefill gate outputs."""
+    wl = synth.WORKLOADS["mixtral_8x7b"]
+    cfg = dict(hidden=wl.hidden, ffn=wl.ffn, n_experts=wl.n_experts, top_k=wl.top_k,
+               shared_ffn=0, n_max=8, renorm_topk=1, max_tokens=4096)
+    big = pw.workspace_bytes(cfg)
+    # gate outputs (fp32) + SwiGLU activations (fp16) + gathered rows (fp16)
+    # + the host-forward staging rows (bf16 in and out)
+    P = 4096 * 2
+    core = P * wl.ffn * 4 + P * wl.ffn * 2 + P * wl.hidden * 2 + 2 * 4096 * wl.hidden * 2
+    assert core <= big <= core + 64 * 2 ** 20, (big, core)
+    small = pw.workspace_bytes(dict(cfg, max_tokens=16))
+    assert small < 64 * 2 ** 20
+    layer = synth.Layer(synth.WORKLOADS["tiny_h256_f512_e8k2"], seed=0)
+    dev = pw.upload_synth_layer(layer, max_tokens=300)
+    tcfg = dict(dev.cfg)
+    assert pw.workspace_bytes(tcfg) > 0
+    dev.close()
