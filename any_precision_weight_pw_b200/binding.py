@@ -24,7 +24,7 @@ EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy"
             "pw_check_device_error", "pw_profile_enable", "pw_profile_read",
             "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
             "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats", "pw_plan_release",
-            "pw_enable_paging", "pw_resident_bytes", "pw_workspace_bytes",
+            "pw_enable_paging", "pw_resident_bytes", "pw_workspace_bytes", "pw_compact_pages",
             "pw_last_error", "pw_abi_version"]
 
 
@@ -74,6 +74,7 @@ def lib():
         L.pw_set_switch_lag.argtypes = [P, i32]
         L.pw_routing_stats.argtypes = [P, P, P, i32, P]
         L.pw_enable_paging.argtypes = [P, P]
+        L.pw_compact_pages.argtypes = [P, P]
         L.pw_workspace_bytes.argtypes = [C.POINTER(Config), C.POINTER(C.c_int64)]
         L.pw_resident_bytes.argtypes = [P, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
         L.pw_plan_release.argtypes = [C.POINTER(PlanBlock), i32, C.c_int64, C.POINTER(i32),
@@ -265,6 +266,10 @@ class MoELayer:
         """Library-owned plane storage holding only each block's resident
         planes (the caller's plane buffers may be freed afterwards)."""
         check(lib().pw_enable_paging(self.h, _stream(stream)))
+
+    def compact_pages(self, stream=None) -> None:
+        """Pack the resident planes into one allocation (on the forward stream)."""
+        check(lib().pw_compact_pages(self.h, _stream(stream)))
 
     def resident_bytes(self, trim: bool = False):
         """(plane bytes resident, pool bytes reserved after a trim or None)."""

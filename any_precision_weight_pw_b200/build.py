@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpw_b200.so")
 SOURCES = ["pw_api.cu", "route.cu", "simple.cu", "tc.cu", "repack.cu", "route_static.cu",
-           "planner.cpp"]
+           "gv.cu", "planner.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -126,6 +126,14 @@ int env_int(const char* name, int dflt) {
 
 }  // namespace
 
+// Paged plane storage: one allocation of the handle's pool, shared by the
+// blocks placed in it (one block after a page move, every block after
+// pw_enable_paging or pw_compact_pages); freed when its last block leaves.
+struct PageAlloc {
+  void* base;
+  int refs;
+};
+
 struct pw_moe {
   pw_moe_config_t cfg{};
   int n_blocks = 0, G = 0, device = 0, n_sm = 0;
@@ -137,14 +145,17 @@ struct pw_moe {
     const uint16_t* h_lut[PW_MAX_BITS + 1];
     int bits, slot;            // active bitwidth and LUT slot
     int stride;                // planes per tile group of d_planes
-    bool owned;                // d_planes is library storage (paging)
+    PageAlloc* alloc;          // paging: the allocation d_planes lies in (null:
+                               // the caller's storage)
     int pend_bits;             // 0 = none
     long long pend_req;        // forwards issued when the change was requested
     uint32_t* pend_planes;     // paging: the storage the pending change fills
+    PageAlloc* pend_alloc;
     cudaEvent_t ready;
   };
   std::vector<Blk> blk;
   bool paging = false;               // plane storage owned by the library
+  bool compacted = false;            // the next forward waits for pw_compact_pages
   cudaMemPool_t pool = nullptr;      // paging: the plane pages' memory pool
   long long n_forwards = 0;
   int max_lag = 8;                   // forwards a page move may stay pending
@@ -171,6 +182,9 @@ struct pw_moe {
   uint16_t* stage_y = nullptr;
   int P_max = 0, gu_stride = 0, last_T = 0;
   size_t ys_floats = 0;   // capacity of the down partials (shared with gbuf)
+  int gv_T = 0, gv_H_pad = 0, gv_F_pad = 0;   // CUDA-core decode passes
+  float* x_gv = nullptr;
+  float* h_gv = nullptr;
   size_t ws_bytes = 0;
   bool tc = false;  // both expert passes on the tensor-core kernel
   void* ws_base = nullptr;
@@ -198,10 +212,15 @@ void free_all(pw_moe* h) {
   for (auto& v : h->ev_pending)
     for (auto e : v) cudaEventDestroy(e);
   for (auto e : h->ev_pool) cudaEventDestroy(e);
+  std::vector<PageAlloc*> allocs;
   for (auto& b : h->blk) {
     if (b.ready) cudaEventDestroy(b.ready);
-    if (b.owned && b.d_planes) cudaFree(b.d_planes);
-    if (b.pend_planes) cudaFree(b.pend_planes);
+    for (PageAlloc* a : {b.alloc, b.pend_alloc})
+      if (a && --a->refs == 0) allocs.push_back(a);
+  }
+  for (PageAlloc* a : allocs) {
+    cudaFree(a->base);
+    delete a;
   }
   if (h->pool) cudaMemPoolDestroy(h->pool);
   if (h->fwd_done) cudaEventDestroy(h->fwd_done);
@@ -226,6 +245,29 @@ int splits_for(const pw_moe_config_t& c, int n_sm, int T, int per_sm) {
   return ns;
 }
 
+// K splits of the CUDA-core down pass (gv.cu): about two rounds of three
+// CTAs per SM over (group, 32-row tile, split) items, at most one split per
+// 256-column tile group of the narrowest down block and kMaxSplit.
+int gv_splits_for(const pw_moe_config_t& c, int n_sm, int T) {
+  int groups = T * c.top_k < c.n_experts ? T * c.top_k : c.n_experts;
+  if (c.shared_ffn > 0) groups += 1;
+  const int row_tiles = (c.hidden + 31) / 32;
+  int ns = (6 * n_sm + groups * row_tiles - 1) / (groups * row_tiles);
+  const int stages = ((c.ffn + 31) / 32 + 7) / 8;
+  if (ns > stages) ns = stages;
+  if (ns > kMaxSplit) ns = kMaxSplit;
+  return ns < 1 ? 1 : ns;
+}
+
+// Largest token count the CUDA-core decode passes take (PW_GV_T, read at
+// create; 0, the default, keeps every decode batch on the tensor cores,
+// which measured faster at every batch of the benchmark workloads).
+int gv_max_tokens(const pw_moe_config_t& c) {
+  const int forced = env_int("PW_GV_T", 0);
+  if (forced <= 0) return 0;
+  return forced < c.max_tokens ? forced : c.max_tokens;
+}
+
 // Sorted positions of a forward of T tokens (routed slots + shared rows).
 size_t positions(const pw_moe_config_t& c, int T) {
   return static_cast<size_t>(T) * c.top_k + (c.shared_ffn > 0 ? T : 0);
@@ -246,9 +288,10 @@ bool prefill_default(const pw_moe_config_t& c, int T) {
 struct Layout {
   bool tc = false, pf = false;
   int P_max = 0, gu_stride = 0, x_ld = 0, h_perm_ld = 0, gbuf_ld = 0;
+  int gv_T = 0, gv_H_pad = 0, gv_F_pad = 0;  // CUDA-core decode passes
   size_t ys_floats = 0;
   size_t o_logits, o_tki, o_tkw, o_off, o_st, o_sw, o_tp, o_tk, o_tc, o_err, o_gd, o_sc, o_sm,
-      o_gu, o_xp, o_hp, o_ys, o_sx, o_sy, total;
+      o_gu, o_xp, o_hp, o_xg, o_hg, o_ys, o_sx, o_sy, total;
 };
 
 Layout make_layout(const pw_moe_config_t& c, int n_sm) {
@@ -265,16 +308,26 @@ Layout make_layout(const pw_moe_config_t& c, int n_sm) {
   L.h_perm_ld = L.tc ? (Fmax + 255) / 256 * 256 : 0;
   L.pf = L.tc && L.P_max >= pw::kTcPfTokens;
   L.gbuf_ld = L.pf ? Fmax : 0;
+  L.gv_T = gv_max_tokens(c);
+  L.gv_H_pad = (c.hidden + 255) / 256 * 256;
+  L.gv_F_pad = (Fmax + 255) / 256 * 256;
   size_t ys = static_cast<size_t>(L.P_max) * c.hidden;
-  if (L.tc)
-    for (int t = 1; t <= T; ++t) {
-      if (L.pf && prefill_default(c, t)) break;
-      int ns = splits_for(c, n_sm, t, 6);
+  for (int t = 1; t <= T; ++t) {
+    if (L.pf && prefill_default(c, t)) break;
+    int ns = 1;
+    if (L.tc) {
+      ns = splits_for(c, n_sm, t, 6);
       const int ns4 = splits_for(c, n_sm, t, 4);
       if (ns4 > ns) ns = ns4;
-      const size_t need = ns * positions(c, t) * c.hidden;
-      if (need > ys) ys = need;
     }
+    if (t <= L.gv_T) {
+      const int ng = gv_splits_for(c, n_sm, t);
+      if (ng > ns) ns = ng;
+    }
+    const size_t need = ns * positions(c, t) * c.hidden;
+    if (need > ys) ys = need;
+  }
+  const size_t P_gv = positions(c, L.gv_T);
   const size_t gb = static_cast<size_t>(L.P_max) * L.gbuf_ld;
   L.ys_floats = ys;
   auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
@@ -295,6 +348,8 @@ Layout make_layout(const pw_moe_config_t& c, int n_sm) {
   L.o_gu = off; off += al(sizeof(float) * size_t(L.P_max) * L.gu_stride);
   L.o_xp = off; off += al(sizeof(uint16_t) * size_t(L.P_max) * L.x_ld);
   L.o_hp = off; off += al(sizeof(uint16_t) * size_t(L.P_max) * L.h_perm_ld);
+  L.o_xg = off; off += al(sizeof(float) * P_gv * L.gv_H_pad);
+  L.o_hg = off; off += al(sizeof(float) * P_gv * L.gv_F_pad);
   L.o_ys = off; off += al(sizeof(float) * (ys > gb ? ys : gb));
   L.o_sx = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
   L.o_sy = off; off += al(sizeof(uint16_t) * size_t(T) * c.hidden);
@@ -303,14 +358,22 @@ Layout make_layout(const pw_moe_config_t& c, int n_sm) {
 }
 
 // Splits of the down pass for a forward of T tokens: the automatic choice
-// (or PW_DOWN_SPLIT), never more than the partials region holds.
+// (or PW_DOWN_SPLIT), never more than the partials region holds.  per_sm 0
+// selects the CUDA-core pass's choice.
 int down_splits(const pw_moe* h, int T, int per_sm) {
   const int forced = env_int("PW_DOWN_SPLIT", 0);
   int ns = forced > 0 ? (forced < kMaxSplit ? forced : kMaxSplit)
-                      : splits_for(h->cfg, h->n_sm, T, per_sm);
+           : per_sm > 0 ? splits_for(h->cfg, h->n_sm, T, per_sm)
+                        : gv_splits_for(h->cfg, h->n_sm, T);
   const size_t per_split = positions(h->cfg, T) * h->cfg.hidden;
   while (ns > 1 && ns * per_split > h->ys_floats) --ns;
   return ns;
+}
+
+// CUDA-core decode passes for T up to the handle's gv_T (PW_GV=0 turns them
+// off).
+bool use_gv(const pw_moe* h, int T) {
+  return h->gv_T > 0 && T <= h->gv_T && env_int("PW_GV", 1) != 0;
 }
 
 // Prefill passes (256-token chunks) when the routed slots average at least
@@ -392,7 +455,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
     d.bits = b.bits;
     d.slot = 0;
     d.stride = c.n_max;
-    d.owned = false;
+    d.alloc = nullptr;
+    d.pend_alloc = nullptr;
     d.pend_bits = 0;
     d.pend_req = 0;
     d.pend_planes = nullptr;
@@ -417,11 +481,15 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->h_perm_ld = L.h_perm_ld;
   h->gbuf_ld = L.gbuf_ld;
   h->ys_floats = L.ys_floats;
+  h->gv_T = L.gv_T;
+  h->gv_H_pad = L.gv_H_pad;
+  h->gv_F_pad = L.gv_F_pad;
   h->ws_bytes = L.total;
   const size_t o_logits = L.o_logits, o_tki = L.o_tki, o_tkw = L.o_tkw, o_off = L.o_off,
                o_st = L.o_st, o_sw = L.o_sw, o_tp = L.o_tp, o_tk = L.o_tk, o_tc = L.o_tc,
                o_err = L.o_err, o_gd = L.o_gd, o_sc = L.o_sc, o_sm = L.o_sm, o_gu = L.o_gu,
-               o_xp = L.o_xp, o_hp = L.o_hp, o_ys = L.o_ys, o_sx = L.o_sx, o_sy = L.o_sy;
+               o_xp = L.o_xp, o_hp = L.o_hp, o_ys = L.o_ys, o_sx = L.o_sx, o_sy = L.o_sy,
+               o_xg = L.o_xg, o_hg = L.o_hg;
   const size_t off = L.total;
   if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
     free_all(h);
@@ -446,6 +514,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
   h->ysorted = reinterpret_cast<float*>(w + o_ys);
   h->gbuf = reinterpret_cast<float*>(w + o_ys);  // shares the partials region
+  h->x_gv = reinterpret_cast<float*>(w + o_xg);
+  h->h_gv = reinterpret_cast<float*>(w + o_hg);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);
   h->stage_y = reinterpret_cast<uint16_t*>(w + o_sy);
   if (cudaMemset(w + o_tk, 0, o_gu - o_tk) != cudaSuccess ||
@@ -498,6 +568,7 @@ pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
                   new_bits);
     }
     uint32_t* dst = static_cast<uint32_t*>(np);
+    b.pend_alloc = new PageAlloc{np, 1};
     const int keep = new_bits < b.bits ? new_bits : b.bits;
     PW_CUDA(cudaMemcpy2DAsync(dst, new_bits * tile, b.d_planes, b.stride * tile, keep * tile, groups,
                               cudaMemcpyDeviceToDevice, s));
@@ -571,15 +642,23 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     if (b.pend_planes) {
       // paging: the forwards issued so far may still read the old storage;
       // this stream-ordered free runs after them and before this forward
-      if (b.owned) PW_CUDA(cudaFreeAsync(b.d_planes, s));
+      if (b.alloc && --b.alloc->refs == 0) {
+        PW_CUDA(cudaFreeAsync(b.alloc->base, s));
+        delete b.alloc;
+      }
       b.d_planes = b.pend_planes;
       b.stride = b.pend_bits;
-      b.owned = true;
+      b.alloc = b.pend_alloc;
       b.pend_planes = nullptr;
+      b.pend_alloc = nullptr;
     }
     b.bits = b.pend_bits;
     b.slot ^= 1;
     b.pend_bits = 0;
+  }
+  if (h->compacted) {
+    PW_CUDA(cudaStreamWaitEvent(s, h->fwd_done, 0));
+    h->compacted = false;
   }
   h->fwd_bits.resize(h->n_blocks);
   for (int i = 0; i < h->n_blocks; ++i) h->fwd_bits[i] = h->blk[i].bits;
@@ -602,8 +681,31 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   // the down partials of split s start at s * split_stride: this forward's
   // positions times H, so the splits down_splits allows fit the region
   const long long split_stride = static_cast<long long>(positions(c, T)) * c.hidden;
-  // decode: gate/up and down in one launch (PW_FUSED=0 splits them)
-  const bool fused = h->tc && !prefill && env_int("PW_FUSED", 1) != 0;
+  // few tokens per expert: the CUDA-core passes (gv.cu)
+  const bool gv = !prefill && use_gv(h, T);
+  // decode on the tensor cores: gate/up and down in one launch (PW_FUSED=0
+  // splits them)
+  const bool fused = h->tc && !prefill && !gv && env_int("PW_FUSED", 1) != 0;
+  pw::GvParams gvp;
+  if (gv) {
+    std::memset(&gvp, 0, sizeof(gvp));
+    gvp.pt = pt;
+    gvp.H = c.hidden;
+    gvp.F = c.ffn;
+    gvp.S = c.shared_ffn;
+    gvp.E = c.n_experts;
+    gvp.n_groups = h->G;
+    gvp.offsets = h->ws.offsets;
+    gvp.slot_token = h->ws.slot_token;
+    gvp.slot_w = h->ws.slot_w;
+    gvp.x = d_x;
+    gvp.x_gv = h->x_gv;
+    gvp.h_gv = h->h_gv;
+    gvp.H_pad = h->gv_H_pad;
+    gvp.F_pad = h->gv_F_pad;
+    gvp.ysorted = h->ysorted;
+    gvp.split_stride = split_stride;
+  }
   std::vector<cudaEvent_t> evs;
   if (h->profiling) {
     for (int i = 0; i < 5; ++i) {
@@ -641,7 +743,10 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   PW_CUDA(mark(1));
 
   // gate/up pass
-  if (h->tc) {
+  if (gv) {
+    PW_CUDA(pw::launch_gv(gvp, 0, static_cast<int>(positions(c, T)), h->n_sm, s));
+    PW_CUDA(pw::launch_gv(gvp, 1, 0, h->n_sm, s));
+  } else if (h->tc) {
     pw::GatherParams gp{};
     gp.x = d_x;
     gp.offsets = h->ws.offsets;
@@ -721,7 +826,13 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
   PW_CUDA(mark(2));
   // down pass
   int n_split = 1;
-  if (fused) {
+  if (gv) {
+    n_split = down_splits(h, T, 0);
+    if (static_cast<size_t>(n_split) * split_stride > h->ys_floats)
+      return fail(PW_ERR_STATE, "down partials (%d splits) exceed the workspace", n_split);
+    gvp.n_split = n_split;
+    PW_CUDA(pw::launch_gv(gvp, 2, 0, h->n_sm, s));
+  } else if (fused) {
     n_split = down_splits(h, T, 6);  // the down items ran in the launch above
   } else if (h->tc) {
     n_split = prefill ? 1 : down_splits(h, T, 4);
@@ -925,36 +1036,78 @@ pw_status_t pw_enable_paging(pw_moe_t* h, pw_stream_t stream) {
   props.location.id = h->device;
   PW_CUDA(cudaMemPoolCreate(&h->pool, &props));
   const size_t tile = pw::pages::kTileBytes;
+  size_t total = 0;
+  for (const auto& b : h->blk)
+    total += static_cast<size_t>(b.bits) * pw::pages::groups_of(b.rows, b.cols) * tile;
+  void* arena = nullptr;
+  if (cudaMallocFromPoolAsync(&arena, total, h->pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    cudaMemPoolDestroy(h->pool);
+    h->pool = nullptr;
+    return fail(PW_ERR_OOM, "plane-page pool allocation of %zu bytes failed", total);
+  }
+  // every block's resident planes, packed one block after another
+  size_t off = 0;
   std::vector<uint32_t*> fresh(h->n_blocks, nullptr);
   for (int i = 0; i < h->n_blocks; ++i) {
     auto& b = h->blk[i];
     const size_t groups = static_cast<size_t>(pw::pages::groups_of(b.rows, b.cols));
-    void* np = nullptr;
-    if (cudaMallocFromPoolAsync(&np, static_cast<size_t>(b.bits) * groups * tile, h->pool, s) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      for (auto q : fresh)
-        if (q) cudaFreeAsync(q, s);
-      cudaStreamSynchronize(s);
-      cudaMemPoolDestroy(h->pool);
-      h->pool = nullptr;
-      return fail(PW_ERR_OOM, "block %d: plane-page pool allocation failed", i);
-    }
-    fresh[i] = static_cast<uint32_t*>(np);
-    PW_CUDA(cudaMemcpy2DAsync(np, b.bits * tile, b.d_planes, b.stride * tile, b.bits * tile, groups,
-                              cudaMemcpyDeviceToDevice, s));
+    fresh[i] = reinterpret_cast<uint32_t*>(static_cast<char*>(arena) + off);
+    PW_CUDA(cudaMemcpy2DAsync(fresh[i], b.bits * tile, b.d_planes, b.stride * tile, b.bits * tile,
+                              groups, cudaMemcpyDeviceToDevice, s));
+    off += static_cast<size_t>(b.bits) * groups * tile;
   }
   // the copies have landed and no forward issued so far still reads the
   // caller's storage
   PW_CUDA(cudaStreamSynchronize(s));
   if (h->any_forward) PW_CUDA(cudaEventSynchronize(h->fwd_done));
+  PageAlloc* a = new PageAlloc{arena, h->n_blocks};
   for (int i = 0; i < h->n_blocks; ++i) {
     auto& b = h->blk[i];
     b.d_planes = fresh[i];
     b.stride = b.bits;
-    b.owned = true;
+    b.alloc = a;
   }
   h->paging = true;
+  return PW_OK;
+}
+
+pw_status_t pw_compact_pages(pw_moe_t* h, pw_stream_t stream) {
+  if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
+  if (!h->paging) return fail(PW_ERR_STATE, "paging is not enabled");
+  for (int i = 0; i < h->n_blocks; ++i)
+    if (h->blk[i].pend_bits)
+      return fail(PW_ERR_STATE, "block %d: a bitwidth change is still pending", i);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tile = pw::pages::kTileBytes;
+  size_t total = 0;
+  for (const auto& b : h->blk)
+    total += static_cast<size_t>(b.stride) * pw::pages::groups_of(b.rows, b.cols) * tile;
+  // after every forward issued so far; the caller's next forwards run on
+  // this stream, behind the copies
+  if (h->any_forward) PW_CUDA(cudaStreamWaitEvent(s, h->fwd_done, 0));
+  void* arena = nullptr;
+  if (cudaMallocFromPoolAsync(&arena, total, h->pool, s) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PW_ERR_OOM, "plane-page pool allocation of %zu bytes failed", total);
+  }
+  size_t off = 0;
+  PageAlloc* a = new PageAlloc{arena, h->n_blocks};
+  for (auto& b : h->blk) {
+    const size_t bytes = static_cast<size_t>(b.stride) * pw::pages::groups_of(b.rows, b.cols) * tile;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<char*>(arena) + off);
+    PW_CUDA(cudaMemcpyAsync(dst, b.d_planes, bytes, cudaMemcpyDeviceToDevice, s));
+    if (b.alloc && --b.alloc->refs == 0) {
+      PW_CUDA(cudaFreeAsync(b.alloc->base, s));
+      delete b.alloc;
+    }
+    b.d_planes = dst;
+    b.alloc = a;
+    off += bytes;
+  }
+  PW_CUDA(cudaEventRecord(h->fwd_done, s));
+  h->any_forward = true;
+  h->compacted = true;  // a forward on another stream waits for the copies
   return PW_OK;
 }
 
@@ -963,7 +1116,7 @@ pw_status_t pw_resident_bytes(pw_moe_t* h, int64_t* plane_bytes, int64_t* pool_r
   int64_t total = 0;
   for (const auto& b : h->blk) {
     const int64_t groups = pw::pages::groups_of(b.rows, b.cols);
-    const int64_t planes = (b.owned || !h->paging) ? b.stride : 0;
+    const int64_t planes = (b.alloc || !h->paging) ? b.stride : 0;
     total += planes * groups * pw::pages::kTileBytes;
     if (b.pend_planes) total += static_cast<int64_t>(b.pend_bits) * groups * pw::pages::kTileBytes;
   }
@@ -1024,8 +1177,9 @@ pw_status_t pw_profile_read(pw_moe_t* h, float* ms, int32_t n, int32_t* n_forwar
 int32_t pw_forward_launches(const pw_moe_t* h, int32_t T) {
   if (!h) return 0;
   if (T <= 0) return 0;
-  if (!h->tc) return 4;
   if (use_prefill(h, T)) return 6;
+  if (use_gv(h, T)) return 5;
+  if (!h->tc) return 4;
   return env_int("PW_FUSED", 1) != 0 ? 4 : 5;
 }
 

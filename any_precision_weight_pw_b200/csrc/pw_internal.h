@@ -129,6 +129,22 @@ struct SimpleParams {
   const uint16_t* lin_lut;
 };
 
+// Decode passes on the CUDA cores for few tokens per expert (gv.cu).
+struct GvParams {
+  PageTable pt;
+  int H, F, S, E, n_groups;
+  const int32_t* offsets;     // [G+1]
+  const int32_t* slot_token;  // [P]
+  const float* slot_w;        // [P]
+  const uint16_t* x;          // bf16 [T][H]
+  float* x_gv;                // [P][H_pad] fp32 activations, dequantiser K order, 0 past H
+  float* h_gv;                // [P][F_pad] fp32 silu(g) * u, same order, 0 past F
+  int H_pad, F_pad;           // multiples of 256
+  float* ysorted;             // [n_split][P][H] routing-weighted partials
+  long long split_stride;     // floats between splits
+  int n_split;                // K splits of the down pass
+};
+
 // Sets the calling thread's pw_last_error() text and returns st (pw_api.cu).
 pw_status_t record_error(pw_status_t st, const char* msg);
 
@@ -139,5 +155,7 @@ cudaError_t launch_repack(const uint32_t* src, uint32_t* dst, int rows, int cols
 cudaError_t launch_gather(const GatherParams& p, int max_rows, int n_sm, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_simple(const SimpleParams& p, int grid_rows, cudaStream_t s);
+// pass 0: gather (max_rows positions at most), 1: gate/up + SwiGLU, 2: down
+cudaError_t launch_gv(const GvParams& p, int pass, int max_rows, int n_sm, cudaStream_t s);
 
 }  // namespace pw

@@ -66,13 +66,13 @@ def whole_job_rate(world, steps, T, ms):
 
 
 # ---------------------------------------------------------------- bytes
-def block_bytes(layer, blk):
+def block_bytes(layer, blk, bits=None):
     rows, cols = layer.shape(blk)
-    b = layer.bits[blk]
+    b = layer.bits[blk] if bits is None else bits[blk]
     return b * rows * ((cols + 31) // 32) * 4 + rows * (1 << b) * 2
 
 
-def algorithmic_bytes(layer, idx):
+def algorithmic_bytes(layer, idx, bits=None):
     """Bytes the method must move for one forward: the active planes and LUTs
     of every expert with at least one routed token (plus the shared expert),
     the router weights, the activations in and the output out."""
@@ -81,8 +81,8 @@ def algorithmic_bytes(layer, idx):
     active = sorted(set(int(e) for e in np.unique(idx)))
     if wl.shared_ffn > 0:
         active.append(wl.n_experts)
-    gu = sum(block_bytes(layer, 3 * e + p) for e in active for p in (0, 1))
-    down = sum(block_bytes(layer, 3 * e + 2) for e in active)
+    gu = sum(block_bytes(layer, 3 * e + p, bits) for e in active for p in (0, 1))
+    down = sum(block_bytes(layer, 3 * e + 2, bits) for e in active)
     router = wl.n_experts * wl.hidden * 4
     act = 2 * T * wl.hidden * 2
     return {"gu": gu + T * wl.hidden * 2, "down": down, "total": gu + down + router + act}
@@ -188,6 +188,11 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
     total = warmup + n_forwards
     sched = synth.switch_schedule(wl, layer.bits, total, every=10)
     pb = [binding.plane_bytes(*layer.shape(blk)) for blk in range(wl.n_blocks)]
+    # routing of each batch (untimed), for the bytes each forward must move
+    routing = []
+    for x, y in zip(xs, ys):
+        d.forward(x, wr, None, y)
+        routing.append(d.routing(T)[0].cpu().numpy())
 
     def run(with_switches, track=False):
         # track: also read back, after every forward, the widths it used, to
@@ -197,6 +202,7 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
         moved = 0
         lags = []        # forwards from a switch's request until all of it applies
         waiting = []     # (forward of the request, widths after it)
+        widths = []      # widths of every forward (tracked pass)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(total)]
         for f in range(total):
@@ -212,26 +218,34 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
             evs[f][0].record(stream)
             d.forward(xs[f % N_BATCHES], wr, None, ys[f % N_BATCHES])
             evs[f][1].record(stream)
-            if waiting:
+            if track:
                 used = d.forward_bits()
+                widths.append(used)
                 while waiting and used == waiting[0][1]:
                     lags.append(f - waiting.pop(0)[0])
         torch.cuda.synchronize()
         d.check_device_error()
         lat = np.array([a.elapsed_time(b) for a, b in evs[warmup:]])
         span = evs[warmup][0].elapsed_time(evs[-1][1])
-        return lat, span, moved, lags
+        return lat, span, moved, lags, widths
 
-    base_lat, base_span, _, _ = run(False)
-    lat, span, moved, _ = run(True)
+    base_lat, base_span, _, _, _ = run(False)
+    lat, span, moved, _, _ = run(True)
     # widths back to the starting table, then the untimed pass that counts lags
     for blk in range(wl.n_blocks):
         d.set_block_bits(blk, layer.bits[blk], side)
     for _ in range(10):
         d.forward(xs[0], wr, None, ys[0])
         torch.cuda.synchronize()
-    _, _, _, lags = run(True, track=True)
+    _, _, _, lags, widths = run(True, track=True)
     n_switch = sum(1 for f in sched if f >= warmup)
+    # achieved GB/s of both runs: the switches change the widths (and so the
+    # bytes) of later forwards; the switch run's widths are those the
+    # tracked pass used, forward by forward
+    base_bytes = sum(algorithmic_bytes(layer, routing[f % N_BATCHES])["total"]
+                     for f in range(warmup, total))
+    sw_bytes = sum(algorithmic_bytes(layer, routing[f % N_BATCHES], widths[f])["total"]
+                   for f in range(warmup, total))
     out = {"workload": "qwen15_moe_a27b decode T=%d, 25%% of blocks switch every 10 forwards" % T,
            "forwards": n_forwards, "tokens_per_s": round(n_forwards * T / (span / 1e3), 1),
            "ms_per_forward_mean": round(float(lat.mean()), 4),
@@ -243,8 +257,12 @@ def page_move_stress(dev, n_forwards=1000, warmup=20):
            "forwards_until_applied": {"mean": round(float(np.mean(lags)), 2) if lags else None,
                                       "max": int(max(lags)) if lags else None,
                                       "max_lag": 8},
+           "gbs": round(sw_bytes / (span / 1e3) / 1e9, 1),
+           "avg_bits": round(float(np.mean([np.mean(w) for w in widths[warmup:]])), 3),
            "no_switch": {"tokens_per_s": round(n_forwards * T / (base_span / 1e3), 1),
-                         "ms_per_forward_p99": round(float(np.percentile(base_lat, 99)), 4)}}
+                         "ms_per_forward_p99": round(float(np.percentile(base_lat, 99)), 4),
+                         "gbs": round(base_bytes / (base_span / 1e3) / 1e9, 1),
+                         "avg_bits": round(float(np.mean(layer.bits)), 3)}}
     d.close()
     return out
 
@@ -313,15 +331,88 @@ def uniform_vs_mixed(dev, hbm_peak):
     return out
 
 
+def small_batch_paths(dev, hbm_peak):
+    """The two decode paths head to head at small batches: the tensor-core
+    passes (the default) and the CUDA-core dequant-GEMV passes (opt-in,
+    PW_GV_T), same layer and token batches, flushed L2, median of 20."""
+    import torch
+    from any_precision_weight_pw_b200 import binding, synth
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = []
+    old = os.environ.get("PW_GV_T")
+    os.environ["PW_GV_T"] = "4"
+    try:
+        for name in ("mixtral_8x7b", "qwen15_moe_a27b"):
+            wl = synth.WORKLOADS[name]
+            layer = synth.Layer(wl, seed=0)
+            d = binding.upload_synth_layer(layer, max_tokens=4)
+            wr = torch.from_numpy(layer.router_w).to(dev)
+            for T in (1, 2, 4):
+                xs = [torch.from_numpy(synth.tokens(wl, T, seed=0, batch=b).view(np.int16)).to(dev)
+                      for b in range(N_BATCHES)]
+                ys = [torch.empty_like(x) for x in xs]
+                mb = []
+                for x, y in zip(xs, ys):
+                    d.forward(x, wr, None, y)
+                    mb.append(algorithmic_bytes(layer, d.routing(T)[0].cpu().numpy())["total"])
+                row = {"workload": "%s decode T=%d" % (name, T)}
+                for tag, gv in (("tensor_core", "0"), ("cuda_core", "1")):
+                    os.environ["PW_GV"] = gv
+                    ms = time_flushed(d, xs, ys, wr, None, flush)
+                    gbs = float(np.mean(mb)) / (ms / 1e3) / 1e9
+                    row[tag] = {"ms": round(ms, 4), "gbs": round(gbs, 1),
+                                "frac_of_measured_hbm": round(gbs / hbm_peak, 4)}
+                os.environ.pop("PW_GV", None)
+                out.append(row)
+            d.close()
+    finally:
+        os.environ.pop("PW_GV", None)
+        if old is None:
+            os.environ.pop("PW_GV_T", None)
+        else:
+            os.environ["PW_GV_T"] = old
+    del flush
+    return out
+
+
+def decode_only(dev, name, T, n=5):
+    """A few forwards of one decode workload (an entry point for ncu
+    captures); returns the mean ms of the last n forwards."""
+    import torch
+    from any_precision_weight_pw_b200 import binding, build, synth
+    build.build()
+    wl = synth.WORKLOADS[name]
+    layer = synth.Layer(wl, seed=0)
+    d = binding.upload_synth_layer(layer, max_tokens=max(T, 1))
+    wr = torch.from_numpy(layer.router_w).to(dev)
+    xs = [torch.from_numpy(synth.tokens(wl, T, seed=0, batch=b).view(np.int16)).to(dev)
+          for b in range(4)]
+    for i in range(3):
+        d.forward(xs[i % 4], wr)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        d.forward(xs[i % 4], wr)
+    e1.record()
+    torch.cuda.synchronize()
+    d.check_device_error()
+    out = {"workload": "%s decode T=%d" % (name, T), "ms_per_forward": e0.elapsed_time(e1) / n,
+           "launches_per_forward": d.launches(T)}
+    d.close()
+    return out
+
+
 def paging_measure(dev, hbm_peak, T=16, n_fwd=200):
     """Residency paging on the Mixtral-shaped layer (decode batch 16): the
     layer switched to library-owned plane storage (only each block's
     resident planes on the device), then the planner frees 25% and then 50%
     of the resident plane bytes (damage = synthetic offline sensitivity x
     the routing mass the library counted over the warm-up forwards), the
-    plan is applied as page moves, and each table is reported as resident
-    plane bytes, pool bytes after a trim, device free memory, and forward
-    tokens/s (back to back, inputs larger than L2)."""
+    plan is applied as page moves and the resident planes are packed, and
+    each table is reported as resident plane bytes, pool bytes after a
+    trim, device free memory, and forward tokens/s (back to back, inputs
+    larger than L2)."""
     import torch
     from any_precision_weight_pw_b200 import binding, synth
     wl = synth.WORKLOADS["mixtral_8x7b"]
@@ -373,6 +464,8 @@ def paging_measure(dev, hbm_peak, T=16, n_fwd=200):
                 d.set_block_bits(blk, b, side)
             bits = plan["bits"]
             d.forward(xs[0], wr, None, ys[0])
+            # pack the resident planes so the pool can hand the freed bytes back
+            d.compact_pages()
             torch.cuda.synchronize()
             ms = timed()
         resident, reserved = d.resident_bytes(trim=True)
@@ -538,6 +631,7 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     uniform = None
     paging = None
+    small = None
     if rank == 0 and not args.no_sweep:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         cur = (name, layer, d, wr, bias)
@@ -562,6 +656,7 @@ def run_ours(args, rank, world, local_rank):
             prefill = prefill_measure(dev)
             uniform = uniform_vs_mixed(dev, hbm_peak)
             paging = paging_measure(dev, hbm_peak)
+            small = small_batch_paths(dev, hbm_peak)
     else:
         d.close()
 
@@ -626,6 +721,7 @@ def run_ours(args, rank, world, local_rank):
         "prefill": prefill,
         "uniform_vs_mixed": uniform,
         "paging": paging,
+        "small_batch_paths": small,
     }
     return out
 
@@ -729,6 +825,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--decode", nargs=2, metavar=("WORKLOAD", "T"),
+                    help="only a few forwards of one decode workload (an entry point for ncu "
+                         "captures; one JSON object)")
     ap.add_argument("--quick", action="store_true",
                     help="headline and decode sweep only (no page-move, prefill, uniform-width "
                          "and paging measurements)")
@@ -738,6 +837,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.decode:
+        import torch
+        print(json.dumps(decode_only(torch.device("cuda", local_rank), args.decode[0],
+                                     int(args.decode[1]))), flush=True)
+        return
     if args.prefill:
         import torch
         print(json.dumps(prefill_measure(torch.device("cuda", local_rank), steps=max(args.steps, 1),

@@ -269,6 +269,16 @@ pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_
  * is pending.  Idempotent. */
 pw_status_t pw_enable_paging(pw_moe_t* h, pw_stream_t stream);
 
+/* Pack every block's resident planes into one new allocation of the pool
+ * and free the old storage, so the memory that page moves left scattered
+ * across the pool's mappings can go back to the device (pw_resident_bytes
+ * with pool_reserved trims the pool).  Enqueued on stream after the last
+ * issued forward; pass the stream the forwards run on (their next forward
+ * then reads the packed copy).  PW_ERR_STATE without paging or while a
+ * bitwidth change is pending; PW_ERR_OOM (nothing changed) if the pool
+ * cannot hold a second copy of the resident planes. */
+pw_status_t pw_compact_pages(pw_moe_t* h, pw_stream_t stream);
+
 /* Device bytes of plane pages the handle keeps resident (a block's
  * resident planes x its plane page size, plus the storage of pending
  * changes; without paging, n_max planes per block).  If pool_reserved is

@@ -686,3 +686,96 @@ def test_workspace_is_sized_to_its_use(pw):
     tcfg = dict(dev.cfg)
     assert pw.workspace_bytes(tcfg) > 0
     dev.close()
+
+
+@pytest.mark.parametrize("name,T,bias_expert", [("tiny_h256_f512_e8k2", 1, None),
+                                                ("tiny_h256_f512_e8k2", 3, None),
+                                                ("tiny_h256_f512_e8k2", 4, 2),
+                                                ("qwen15_moe_a27b", 2, None),
+                                                ("mixtral_8x7b", 2, None)])
+def test_cuda_core_decode_passes(pw, oracle, name, T, bias_expert):
+    """The CUDA-core decode passes (few tokens per expert: gather, gate/up
+    with SwiGLU, split-K down) against the oracle, and against the
+    tensor-core passes on the same inputs (PW_GV=0) within the same bound;
+    with a router bias all tokens share one expert (one token chunk)."""
+    layer = synth.Layer(synth.WORKLOADS[name], seed=9)
+    if bias_expert is not None:
+        layer.router_bias = np.zeros(layer.wl.n_experts, np.float32)
+        layer.router_bias[bias_expert] = 50.0
+    y, idx, w, x = _run_layer_env(pw, layer, T, {"PW_GV_T": str(T)}, batch=T)
+    ref, ridx, rw = _oracle_forward(oracle, layer, x, threads=32)
+    np.testing.assert_array_equal(idx, ridx)
+    assert_output_close(y, ref)
+    y2, idx2, _, _ = _run_layer_env(pw, layer, T, {"PW_GV": "0"}, batch=T)
+    np.testing.assert_array_equal(idx2, ridx)
+    assert_output_close(y2, ref)
+
+
+def test_cuda_core_decode_token_chunks_and_paging(pw, oracle):
+    """Groups with more tokens than one item carries (12 tokens on one
+    expert: three chunks of four), on paged storage after page moves."""
+    wl = synth.WORKLOADS["tiny_h256_f512_e8k2"]
+    layer = synth.Layer(wl, seed=10)
+    layer.router_bias = np.zeros(8, np.float32)
+    layer.router_bias[5] = 50.0
+    old = os.environ.get("PW_GV_T")
+    os.environ["PW_GV_T"] = "12"
+    try:
+        dev = pw.upload_synth_layer(layer, max_tokens=12, host_copies=True)
+    finally:
+        if old is None:
+            os.environ.pop("PW_GV_T", None)
+        else:
+            os.environ["PW_GV_T"] = old
+    dev.enable_paging()
+    dev.set_switch_lag(0)
+    side = torch.cuda.Stream()
+    for blk, b in {15: 2, 16: 6, 17: 8, 3: 5}.items():
+        dev.set_block_bits(blk, b, side)
+    wr = torch.from_numpy(layer.router_w).cuda()
+    bias = torch.from_numpy(layer.router_bias).cuda()
+    x = synth.tokens(wl, 12, seed=10)
+    y = dev.forward(_dev_bf16(x), wr, bias)
+    used = dev.forward_bits()
+    assert dev.launches(12) == 5          # route, gather, gate/up, down, combine
+    torch.cuda.synchronize()
+    dev.check_device_error()
+    ref, ridx, _ = oracle_layer(oracle, layer, used).forward(x, layer.router_w, layer.router_bias,
+                                                            threads=8)
+    assert np.all(ridx[:, 0] == 5)
+    assert_output_close(_to_f32(y), ref)
+    dev.close()
+
+
+def test_paging_compaction_returns_memory(pw, oracle):
+    """Lower most blocks' widths on paged storage, then pack the resident
+    planes into one allocation: after a trim the pool reserves little more
+    than the resident bytes, and the forwards before and after match the
+    oracle."""
+    wl = synth.WORKLOADS["qwen15_moe_a27b"]
+    layer = synth.Layer(wl, seed=13)
+    T = 8
+    dev = pw.upload_synth_layer(layer, max_tokens=T, host_copies=True)
+    dev.enable_paging()
+    wr = torch.from_numpy(layer.router_w).cuda()
+    side = torch.cuda.Stream()
+    dev.set_switch_lag(0)
+    bits = [max(2, b - 2) for b in layer.bits]
+    for blk, b in enumerate(bits):
+        dev.set_block_bits(blk, b, side)
+    x = synth.tokens(wl, T, seed=13)
+    y1 = dev.forward(_dev_bf16(x), wr)
+    assert dev.forward_bits() == bits
+    torch.cuda.synchronize()
+    resident, reserved_before = dev.resident_bytes(trim=True)
+    dev.compact_pages()
+    y2 = dev.forward(_dev_bf16(x), wr)
+    torch.cuda.synchronize()
+    resident2, reserved_after = dev.resident_bytes(trim=True)
+    assert resident2 == resident == _plane_total(pw, layer, bits)
+    assert reserved_after <= resident + 4 * 2 ** 20, (reserved_after, resident, reserved_before)
+    assert torch.equal(y1, y2)
+    ref, _, _ = oracle_layer(oracle, layer, bits).forward(x, layer.router_w, threads=32)
+    assert_output_close(_to_f32(y2), ref)
+    dev.check_device_error()
+    dev.close()
