@@ -699,11 +699,17 @@ def run_ours(args, rank, world, local_rank):
                    "batches": N_BATCHES, "parallelism": "replicas" if world > 1 else "1 GPU"},
         "hbm_gbs": round(fwd_gbs, 1),
         "hbm_frac": round(fwd_gbs / hbm_peak, 4),
+        # the same against the nominal ~8 TB/s of B200 HBM3e
+        "hbm_frac_of_8tbs": round(fwd_gbs / 8000.0, 4),
         "hbm_peak": {"gbs": hbm_peak, "kind": peak_kind},
         "roofline": {"bound": "hbm", "kernel": "tc_kernel (gate/up and down items; one fused launch at decode)",
                      "achieved": round(tc_gbs, 1) if tc_gbs else None, "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(tc_gbs / hbm_peak, 4) if tc_gbs else None,
                      "traffic": traffic,
+                     "traffic_source": ("recorded: dram__bytes_read.sum + dram__bytes_write.sum "
+                                        "of an ncu capture of this kernel source "
+                                        "(profiles/traffic_per_forward.json)")
+                                       if traffic else None,
                      "launch_ms_per_forward": [round(m / max(n_fwd, 1), 5) for m in per_launch]},
         "cpu_baseline": cpu,
         "accuracy": accuracy,

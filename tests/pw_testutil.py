@@ -12,6 +12,8 @@ outputs near zero.  output_errors also reports that arithmetic part on its
 own (arith_excess) and how often the output differs from the correctly
 rounded oracle value (rne_mismatch).
 """
+import os
+
 import numpy as np
 
 REL_TOL = 2e-3
@@ -54,8 +56,15 @@ def output_errors(y_gpu, y_ref):
     }
 
 
+# (test id, errors) of every comparison made in this session, for the
+# summary the test session prints at the end (tests/conftest.py)
+RECORDED = []
+
+
 def assert_output_close(y_gpu, y_ref):
     e = output_errors(y_gpu, y_ref)
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    RECORDED.append((test, e))
     assert e["excess"] <= 0.0, e
     return e
 

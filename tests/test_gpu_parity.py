@@ -748,10 +748,10 @@ def test_cuda_core_decode_token_chunks_and_paging(pw, oracle):
 
 
 def test_paging_compaction_returns_memory(pw, oracle):
-    """Lower most blocks' widths on paged storage, then pack the resident
-    planes into one allocation: after a trim the pool reserves little more
-    than the resident bytes, and the forwards before and after match the
-    oracle."""
+    """Lower every block's width on paged storage, then pack the resident
+    planes into one allocation: after a trim the pool reserves less than
+    before and at most one mapping chunk more than the resident bytes, and
+    the forwards before and after match the oracle."""
     wl = synth.WORKLOADS["qwen15_moe_a27b"]
     layer = synth.Layer(wl, seed=13)
     T = 8
@@ -773,7 +773,10 @@ def test_paging_compaction_returns_memory(pw, oracle):
     torch.cuda.synchronize()
     resident2, reserved_after = dev.resident_bytes(trim=True)
     assert resident2 == resident == _plane_total(pw, layer, bits)
-    assert reserved_after <= resident + 4 * 2 ** 20, (reserved_after, resident, reserved_before)
+    # the pool maps memory in chunks (32 MiB on the B200s measured): after
+    # the trim it holds the packed copy rounded up to its mapping granularity
+    assert reserved_after < reserved_before, (reserved_after, reserved_before)
+    assert reserved_after <= resident + 32 * 2 ** 20, (reserved_after, resident, reserved_before)
     assert torch.equal(y1, y2)
     ref, _, _ = oracle_layer(oracle, layer, bits).forward(x, layer.router_w, threads=32)
     assert_output_close(_to_f32(y2), ref)
