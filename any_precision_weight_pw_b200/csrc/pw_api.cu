@@ -170,7 +170,7 @@ struct pw_moe {
   int x_ld = 0, h_perm_ld = 0;
   CUtensorMap x_maps[4], h_maps[4];  // token-tile maps over x_sorted and h_perm
   CUtensorMap x_pf_map, h_pf_map;    // 256-row chunk maps (prefill passes)
-  float* gbuf = nullptr;             // prefill: gate outputs [P_max][Fmax] fp32
+  uint16_t* gbuf = nullptr;          // prefill: gate outputs [P_max][Fmax] fp16
   int* gu_done = nullptr;            // fused decode launch: per-group gate/up counts
   int gbuf_ld = 0;
   bool pf = false;                   // the prefill passes are available
@@ -290,7 +290,7 @@ struct Layout {
   int P_max = 0, gu_stride = 0, x_ld = 0, h_perm_ld = 0, gbuf_ld = 0;
   int gv_T = 0, gv_H_pad = 0, gv_F_pad = 0;  // CUDA-core decode passes
   size_t ys_floats = 0;
-  size_t o_logits, o_tki, o_tkw, o_off, o_st, o_sw, o_tp, o_tk, o_tc, o_err, o_gd, o_sc, o_sm,
+  size_t o_tki, o_tkw, o_off, o_st, o_sw, o_tp, o_tk, o_err, o_gd, o_sc, o_sm,
       o_gu, o_xp, o_hp, o_xg, o_hg, o_ys, o_sx, o_sy, total;
 };
 
@@ -328,11 +328,10 @@ Layout make_layout(const pw_moe_config_t& c, int n_sm) {
     if (need > ys) ys = need;
   }
   const size_t P_gv = positions(c, L.gv_T);
-  const size_t gb = static_cast<size_t>(L.P_max) * L.gbuf_ld;
+  const size_t gb = (static_cast<size_t>(L.P_max) * L.gbuf_ld + 1) / 2;  // fp16, in floats
   L.ys_floats = ys;
   auto al = [](size_t n) { return (n + 255) & ~size_t(255); };
   size_t off = 0;
-  L.o_logits = off; off += al(sizeof(float) * T * E);
   L.o_tki = off; off += al(sizeof(int32_t) * T * k);
   L.o_tkw = off; off += al(sizeof(float) * T * k);
   L.o_off = off; off += al(sizeof(int32_t) * (G + 1));
@@ -340,7 +339,6 @@ Layout make_layout(const pw_moe_config_t& c, int n_sm) {
   L.o_sw = off; off += al(sizeof(float) * L.P_max);
   L.o_tp = off; off += al(sizeof(int32_t) * (T * k + T));
   L.o_tk = off; off += al(sizeof(uint32_t) * 4);
-  L.o_tc = off; off += al(sizeof(uint32_t) * T);
   L.o_err = off; off += al(sizeof(int) * 4);
   L.o_gd = off; off += al(sizeof(int) * (G + 1));
   L.o_sc = off; off += al(sizeof(unsigned long long) * E);
@@ -485,8 +483,8 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->gv_H_pad = L.gv_H_pad;
   h->gv_F_pad = L.gv_F_pad;
   h->ws_bytes = L.total;
-  const size_t o_logits = L.o_logits, o_tki = L.o_tki, o_tkw = L.o_tkw, o_off = L.o_off,
-               o_st = L.o_st, o_sw = L.o_sw, o_tp = L.o_tp, o_tk = L.o_tk, o_tc = L.o_tc,
+  const size_t o_tki = L.o_tki, o_tkw = L.o_tkw, o_off = L.o_off,
+               o_st = L.o_st, o_sw = L.o_sw, o_tp = L.o_tp, o_tk = L.o_tk,
                o_err = L.o_err, o_gd = L.o_gd, o_sc = L.o_sc, o_sm = L.o_sm, o_gu = L.o_gu,
                o_xp = L.o_xp, o_hp = L.o_hp, o_ys = L.o_ys, o_sx = L.o_sx, o_sy = L.o_sy,
                o_xg = L.o_xg, o_hg = L.o_hg;
@@ -496,7 +494,6 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
     return fail(PW_ERR_OOM, "workspace allocation of %zu bytes failed", off);
   }
   char* w = static_cast<char*>(h->ws_base);
-  h->ws.logits = reinterpret_cast<float*>(w + o_logits);
   h->ws.topk_idx = reinterpret_cast<int32_t*>(w + o_tki);
   h->ws.topk_w = reinterpret_cast<float*>(w + o_tkw);
   h->ws.offsets = reinterpret_cast<int32_t*>(w + o_off);
@@ -504,7 +501,6 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->ws.slot_w = reinterpret_cast<float*>(w + o_sw);
   h->ws.token_pos = reinterpret_cast<int32_t*>(w + o_tp);
   h->ws.ticket = reinterpret_cast<uint32_t*>(w + o_tk);
-  h->ws.tok_ctr = reinterpret_cast<uint32_t*>(w + o_tc);
   h->err = reinterpret_cast<int*>(w + o_err);
   h->gu_done = reinterpret_cast<int*>(w + o_gd);
   h->stat_count = reinterpret_cast<unsigned long long*>(w + o_sc);
@@ -513,7 +509,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
   h->x_sorted = reinterpret_cast<uint16_t*>(w + o_xp);
   h->h_perm = reinterpret_cast<uint16_t*>(w + o_hp);
   h->ysorted = reinterpret_cast<float*>(w + o_ys);
-  h->gbuf = reinterpret_cast<float*>(w + o_ys);  // shares the partials region
+  h->gbuf = reinterpret_cast<uint16_t*>(w + o_ys);  // shares the partials region
   h->x_gv = reinterpret_cast<float*>(w + o_xg);
   h->h_gv = reinterpret_cast<float*>(w + o_hg);
   h->stage_x = reinterpret_cast<uint16_t*>(w + o_sx);

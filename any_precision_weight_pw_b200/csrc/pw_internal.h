@@ -69,15 +69,13 @@ struct PageTable {
 // Sorted positions: group g owns positions [offsets[g], offsets[g+1]); the
 // routed lists are ordered by token, the shared list is tokens 0..T-1.
 struct RouteWorkspace {
-  float* logits;        // [T][E]
   int32_t* topk_idx;    // [T][k]
   float* topk_w;        // [T][k]
   int32_t* offsets;     // [G+1]
   int32_t* slot_token;  // [P] token of each sorted position
   float* slot_w;        // [P] routing weight of each sorted position
   int32_t* token_pos;   // [T][k] (+ [T] shared) sorted position of (t, j)
-  uint32_t* ticket;     // last-block-done counter (self-resetting)
-  uint32_t* tok_ctr;    // [T] logits written per token (self-resetting)
+  uint32_t* ticket;     // last-cluster-done counter (self-resetting)
 };
 
 struct RouteParams {
@@ -90,7 +88,24 @@ struct RouteParams {
   int n_zero;              // (may be null / 0)
   unsigned long long* stat_count;  // [E] routing statistics, accumulated over
   double* stat_mass;               // forwards (both null: none kept)
+  // launch geometry (launch_route fills these from route_geometry)
+  int cb, ce;         // blocks per cluster = token groups x ce expert groups
+  int tb, tbb, eb;    // tokens per cluster, tokens per block, experts per block
+  int kc;             // columns per staged chunk (a multiple of 32)
+  int n_clusters;
+  int logits_off;     // shared-memory offset of the cluster's logits [tb][E]
+  int sel_staged;     // every selection fits in shared memory for the bucketing
+  int vec;            // 16-byte asynchronous copies of x and wr are legal
 };
+
+// Router launch geometry for T tokens, E experts, hidden H and top-k (host).
+struct RouteGeometry {
+  int cb, ce, tb, tbb, eb, kc, n_clusters;
+  int tt, te;         // register tile of a warp: tokens x experts (tt = 0: none fits)
+  bool sel_staged;
+  size_t logits_off, smem;
+};
+RouteGeometry route_geometry(int T, int E, int H, int k);
 
 struct GatherParams {
   const uint16_t* x;         // bf16 [T][H]

@@ -9,6 +9,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "dequant.cuh"
 #include "pw_internal.h"
 
@@ -17,29 +19,109 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kRouteThreads = 256;
-constexpr int kStageSel = 16384;    // selections kept in shared memory (one byte each)
-constexpr int kStageW = 2048;       // routing weights kept in shared memory (8 KB)
+constexpr int kRouteWarps = kRouteThreads / 32;
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
-// Top-k and softmax of token t by one warp, once all E logits of t are in
-// global memory: lane i holds experts i + 32 q (q < 4); each of the k rounds
-// is an argmax over the warp under the ranking order (logit descending,
-// index ascending); the softmax denominator is a lane-wise sum met in a xor
-// butterfly.  Lane 0 writes the selections and their weights.
-__device__ void topk_token(const RouteParams& p, int t, int lane) {
+// ---- cluster and asynchronous-copy primitives ------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// store v to the shared-memory word at local address a in cluster block 0
+__device__ __forceinline__ void st_leader(uint32_t a, float v) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(a));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(r), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---- the lane butterfly, for N accumulators at once ------------------------
+// Every lane holds N partial sums (N a power of two <= 32).  The logit order
+// adds, at levels m = 16, 8, 4, 2, 1, each lane's value to that of lane ^ m.
+// Here each level also halves the live values: the lane with bit m set keeps
+// the upper half, receives its partner's copy of that half and adds it to its
+// own, the other lane keeps the lower half.  Every sum is the one the plain
+// butterfly forms (own value + partner's, the same operands), so the result
+// is bit-identical.  Afterwards lane l holds accumulator l >> (5 - log2 N);
+// the levels past log2 N are plain butterfly levels.
+template <int N>
+__device__ __forceinline__ float tree_sum(float (&a)[N], int lane) {
+#pragma unroll
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    const int m = 16 >> lvl;
+    constexpr int kN = N;
+    const int n = kN >> lvl;  // live values before this level
+    if (n > 1) {
+      const bool hi = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < n / 2; ++i) {
+        const float send = hi ? a[i] : a[i + n / 2];
+        const float keep = hi ? a[i + n / 2] : a[i];
+        a[i] = keep + __shfl_xor_sync(kFull, send, m);
+      }
+    } else {
+      a[0] = a[0] + __shfl_xor_sync(kFull, a[0], m);
+    }
+  }
+  return a[0];
+}
+template <int N>
+struct Log2 {
+  static constexpr int value = N <= 1 ? 0 : 1 + Log2<(N > 1 ? N / 2 : 1)>::value;
+};
+template <>
+struct Log2<1> {
+  static constexpr int value = 0;
+};
+
+// Top-k and softmax of one token by a group of L lanes (L a power of two,
+// 4 L >= E) from its E logits in shared memory: lane i of the group holds
+// experts i + L q (q < 4); each of the k rounds is an argmax over the group
+// under the ranking order (logit descending, index ascending), met in xor
+// shuffles within the group, so every lane of the group ends with the same
+// selection; the softmax denominator is a group-wise xor sum.  Every lane of
+// the warp calls this (the shuffles take the whole warp); `active` is false
+// for groups without a token.  Lane 0 of a group writes the selections and
+// their weights to global memory and, when sel is non-null, to the shared-
+// memory staging arrays.
+__device__ __forceinline__ void topk_group(const RouteParams& p, const float* l, int t,
+                                           bool active, int gl, int L, uint8_t* sel,
+                                           float* selw) {
   const int E = p.E, k = p.k;
-  const float* l = p.ws.logits + static_cast<size_t>(t) * E;
   float v[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int e = lane + 32 * q;
-    v[q] = e < E ? __ldcg(l + e) : 0.0f;
+    const int e = gl + L * q;
+    v[q] = (active && e < E) ? l[e] : 0.0f;
   }
-  uint32_t taken = 0u;  // bit q: expert lane + 32 q already selected
-  int sel[PW_MAX_TOPK];
+  uint32_t taken = 0u;  // bit q: expert gl + L q already selected
+  int sidx[PW_MAX_TOPK];
   float lsel[PW_MAX_TOPK];
 #pragma unroll
   for (int j = 0; j < PW_MAX_TOPK; ++j) {
@@ -48,14 +130,13 @@ __device__ void topk_token(const RouteParams& p, int t, int lane) {
     int bi = -1;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int e = lane + 32 * q;
-      if (e < E && !((taken >> q) & 1u) && (bi < 0 || v[q] > bv)) {
+      const int e = gl + L * q;
+      if (active && e < E && !((taken >> q) & 1u) && (bi < 0 || v[q] > bv)) {
         bv = v[q];
         bi = e;
       }
     }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
+    for (int m = L >> 1; m >= 1; m >>= 1) {
       const float ov = __shfl_xor_sync(kFull, bv, m);
       const int oi = __shfl_xor_sync(kFull, bi, m);
       if (oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oi < bi))) {
@@ -63,18 +144,17 @@ __device__ void topk_token(const RouteParams& p, int t, int lane) {
         bi = oi;
       }
     }
-    if (bi >= 0 && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-    sel[j] = bi;
+    if (bi >= 0 && (bi & (L - 1)) == gl) taken |= 1u << (bi / L);
+    sidx[j] = bi;
     lsel[j] = bv;
   }
   const float mx = lsel[0];
   float z = 0.0f;
 #pragma unroll
   for (int q = 0; q < 4; ++q)
-    if (lane + 32 * q < E) z += expf(v[q] - mx);
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) z += __shfl_xor_sync(kFull, z, m);
-  if (lane == 0) {
+    if (active && gl + L * q < E) z += expf(v[q] - mx);
+  for (int m = L >> 1; m >= 1; m >>= 1) z += __shfl_xor_sync(kFull, z, m);
+  if (active && gl == 0) {
     float psel[PW_MAX_TOPK];
     float ssum = 0.0f;
 #pragma unroll
@@ -86,131 +166,229 @@ __device__ void topk_token(const RouteParams& p, int t, int lane) {
 #pragma unroll
     for (int j = 0; j < PW_MAX_TOPK; ++j) {
       if (j >= k) break;
-      p.ws.topk_idx[t * k + j] = sel[j];
-      p.ws.topk_w[t * k + j] = p.renorm ? psel[j] / ssum : psel[j];
+      const float w = p.renorm ? psel[j] / ssum : psel[j];
+      p.ws.topk_idx[t * k + j] = sidx[j];
+      p.ws.topk_w[t * k + j] = w;
+      if (sel) {
+        sel[t * k + j] = static_cast<uint8_t>(sidx[j]);
+        selw[t * k + j] = w;
+      }
     }
   }
 }
 
-// One launch.  Phase 1: every warp computes router logits for (token,
-// expert) pairs; lane j owns columns j, j+32, ... and fuses them in
-// ascending order, then the 32 partial sums meet in a xor butterfly
-// (16, 8, 4, 2, 1), so every lane ends with the same value.  A per-token
-// counter finds the warp that writes a token's last logit; that warp takes
-// the token's top-k and softmax at once (topk_token), so the selections of
-// all tokens are made in parallel.  Phase 2 runs in the block that finishes
-// last (a ticket counter, no waiting): per-expert counts from warp ballots
-// over the staged selections, one warp-wide scan over the experts, and
-// per-expert token lists ordered by token; it also puts the counters back
-// to zero for the next launch.
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams p) {
+// One launch, in clusters of p.cb = (token groups) x p.ce (expert groups)
+// blocks.  Cluster c owns tokens [c tb, c tb + tb); its block r owns the
+// p.tbb tokens of token group r / ce and the p.eb experts of expert group
+// r % ce.
+//
+// Phase 1 (every block): the block's token rows and router rows are copied
+// into shared memory in column chunks (16-byte asynchronous copies, two
+// buffers), and each warp computes the logits of a TT x TE tile of (token,
+// expert) pairs: lane j owns columns j, j + 32, ... and fuses them in
+// ascending order into TT x TE accumulators, which meet in the lane butterfly
+// (tree_sum).  The logits go to the shared memory of the cluster's block 0
+// (distributed shared memory), and a cluster barrier hands them over.
+//
+// Phase 2 (block 0 of each cluster): a group of lanes per token takes its
+// top-k and softmax from the logits in shared memory.
+//
+// Phase 3 (bucketing, one block): with one cluster, its block 0 carries on
+// from the selections it holds in shared memory; with several, the block 0
+// that finishes last (a ticket counter, no waiting) stages every selection
+// with coalesced loads.  Per-expert counts come from warp ballots over
+// 32-token blocks, offsets from one warp-wide scan, and per-expert token
+// lists ordered by token; the ticket goes back to zero for the next launch.
+template <int TT, int TE>
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const RouteParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int warps_per_block = kRouteThreads / 32;
   const int E = p.E, H = p.H, T = p.T, k = p.k;
   const RouteWorkspace& ws = p.ws;
+  const int rank = static_cast<int>(cluster_rank());
+  const int tc0 = static_cast<int>(blockIdx.x) / p.cb * p.tb;  // the cluster's first token
+  const int tl0 = (rank / p.ce) * p.tbb;                         // the block's, within the cluster
+  const int t0 = tc0 + tl0;
+  const int e0 = (rank - (rank / p.ce) * p.ce) * p.eb;
+  const int nt = min(min(p.tbb, p.tb - tl0), T - t0);  // may be <= 0
+  const int ne = min(p.eb, E - e0);                    // may be <= 0 (trailing block)
+  cluster_arrive_relaxed();  // block 0's shared memory is live once all have arrived
   // the previous kernel on the stream may produce x and still read the
   // workspace; the gather kernel may be scheduled from here on
   pdl_wait();
   pdl_trigger();
 
-  const int total_pairs = T * E;
-  for (int pair = blockIdx.x * warps_per_block + warp; pair < total_pairs;
-       pair += gridDim.x * warps_per_block) {
-    const int t = pair / E;
-    const int e = pair - t * E;
-    const uint16_t* xr = p.x + static_cast<size_t>(t) * H;
-    const float* wr = p.wr + static_cast<size_t>(e) * H;
-    // loads in batches of 32 per lane (independent of the sum, so their
-    // latencies overlap), the next batch issued before the current one is
-    // summed; the fused multiply-adds stay in ascending i
-    float s = 0.0f;
-    int i0 = lane;
-    float xv[32], wv[32];
-    bool have = i0 + 32 * 31 < H;
-    if (have) {
+  // ---- phase 1: logits ----------------------------------------------------
+  const int kc_max = p.kc;
+  const size_t xbytes = (static_cast<size_t>(p.tbb) * kc_max * 2 + 15) & ~static_cast<size_t>(15);
+  const size_t sbytes = xbytes + static_cast<size_t>(p.eb) * kc_max * 4;
+  const int n_chunks = (H + kc_max - 1) / kc_max;
+  auto issue = [&](int ci) {
+    const int k0 = ci * kc_max;
+    const int kc = min(kc_max, H - k0);
+    unsigned char* dx = smem + (ci & 1) * sbytes;
+    float* dw = reinterpret_cast<float*>(dx + xbytes);
+    uint16_t* dxh = reinterpret_cast<uint16_t*>(dx);
+    if (p.vec) {
+      const int xp = kc >> 3;  // 16-byte pieces of a token row chunk
+      for (int r = 0; r < nt; ++r) {
+        const uint16_t* src = p.x + static_cast<size_t>(t0 + r) * H + k0;
+        for (int q = threadIdx.x; q < xp; q += kRouteThreads)
+          cp_async16(dxh + r * kc_max + 8 * q, src + 8 * q);
+      }
+      const int wp = kc >> 2;
+      for (int r = 0; r < ne; ++r) {
+        const float* src = p.wr + static_cast<size_t>(e0 + r) * H + k0;
+        for (int q = threadIdx.x; q < wp; q += kRouteThreads)
+          cp_async16(dw + r * kc_max + 4 * q, src + 4 * q);
+      }
+    } else {
+      for (int r = 0; r < nt; ++r)
+        for (int q = threadIdx.x; q < kc; q += kRouteThreads)
+          dxh[r * kc_max + q] = p.x[static_cast<size_t>(t0 + r) * H + k0 + q];
+      for (int r = 0; r < ne; ++r)
+        for (int q = threadIdx.x; q < kc; q += kRouteThreads)
+          dw[r * kc_max + q] = p.wr[static_cast<size_t>(e0 + r) * H + k0 + q];
+    }
+    cp_async_commit();
+  };
+
+  constexpr int kN = TT * TE;
+  const int tasks_e = (p.eb + TE - 1) / TE;
+  const int n_tasks = ((p.tbb + TT - 1) / TT) * tasks_e;  // <= kRouteWarps (host)
+  const bool busy = warp < n_tasks;
+  const int tt0 = (warp / tasks_e) * TT;
+  const int te0 = (warp - (warp / tasks_e) * tasks_e) * TE;
+  float acc[kN];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        xv[u] = bf16_bits_to_f32(xr[i0 + 32 * u]);
-        wv[u] = wr[i0 + 32 * u];
+  for (int i = 0; i < kN; ++i) acc[i] = 0.0f;
+
+  issue(0);
+  if (n_chunks > 1) issue(1);
+  for (int ci = 0; ci < n_chunks; ++ci) {
+    if (ci + 1 < n_chunks)
+      cp_async_wait<1>();
+    else
+      cp_async_wait<0>();
+    __syncthreads();
+    if (busy) {
+      const int kc = min(kc_max, H - ci * kc_max);
+      const unsigned char* base = smem + (ci & 1) * sbytes;
+      // a tile's rows past the buffer's tbb token rows or eb router rows
+      // read the last row instead; rows past the block's tokens or experts
+      // hold stale data; the sums of both are never written
+      const uint16_t* xr[TT];
+      const float* wrs[TE];
+#pragma unroll
+      for (int a = 0; a < TT; ++a)
+        xr[a] = reinterpret_cast<const uint16_t*>(base) + min(tt0 + a, p.tbb - 1) * kc_max;
+#pragma unroll
+      for (int b = 0; b < TE; ++b)
+        wrs[b] = reinterpret_cast<const float*>(base + xbytes) + min(te0 + b, p.eb - 1) * kc_max;
+#pragma unroll 4
+      for (int c = lane; c < kc; c += 32) {
+        float xv[TT], wv[TE];
+#pragma unroll
+        for (int a = 0; a < TT; ++a) xv[a] = bf16_bits_to_f32(xr[a][c]);
+#pragma unroll
+        for (int b = 0; b < TE; ++b) wv[b] = wrs[b][c];
+#pragma unroll
+        for (int a = 0; a < TT; ++a)
+#pragma unroll
+          for (int b = 0; b < TE; ++b) acc[a * TE + b] = __fmaf_rn(xv[a], wv[b], acc[a * TE + b]);
       }
     }
-    while (have) {
-      const int i1 = i0 + 32 * 32;
-      const bool more = i1 + 32 * 31 < H;
-      float xn[32], wn[32];
-      if (more) {
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          xn[u] = bf16_bits_to_f32(xr[i1 + 32 * u]);
-          wn[u] = wr[i1 + 32 * u];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 32; ++u) s = __fmaf_rn(xv[u], wv[u], s);
-      i0 = i1;
-      have = more;
-      if (more) {
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          xv[u] = xn[u];
-          wv[u] = wn[u];
-        }
-      }
+    __syncthreads();  // this buffer is free again
+    if (ci + 2 < n_chunks) issue(ci + 2);
+  }
+
+  float* s_logits = reinterpret_cast<float*>(smem + p.logits_off);  // [tb][E], block 0
+  cluster_wait();  // pairs with the arrive at the start
+  if (busy) {
+    const float v = tree_sum<kN>(acc, lane);
+    constexpr int kShift = 5 - Log2<kN>::value;
+    const int a = lane >> kShift;
+    const int tl = tt0 + a / TE, el = te0 + a % TE;
+    if ((lane & ((1 << kShift) - 1)) == 0 && tl < nt && el < ne) {
+      const int e = e0 + el;
+      st_leader(smem_u32(s_logits + (tl0 + tl) * E + e), p.bias ? v + p.bias[e] : v);
     }
-    for (int i = i0; i < H; i += 32) s = __fmaf_rn(bf16_bits_to_f32(xr[i]), wr[i], s);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) s = s + __shfl_xor_sync(kFull, s, m);
-    int last = 0;
-    if (lane == 0) {
-      ws.logits[pair] = p.bias ? s + p.bias[e] : s;
-      __threadfence();
-      last = atomicAdd(ws.tok_ctr + t, 1u) == static_cast<unsigned>(E - 1);
-    }
-    if (__shfl_sync(kFull, last, 0)) {
-      __threadfence();
-      topk_token(p, t, lane);
+  }
+  cluster_arrive_release();
+  cluster_wait();
+  if (rank != 0) return;
+
+  // ---- phase 2: top-k per token (block 0 of the cluster) -------------------
+  // With one cluster the selections also go to shared memory for phase 3;
+  // they reuse the staging buffers, which no warp reads any more.
+  const bool one = p.n_clusters == 1;
+  const bool staged = p.sel_staged != 0;
+  uint8_t* s_idx = smem;
+  float* s_w = reinterpret_cast<float*>(smem + ((static_cast<size_t>(T) * k + 15) & ~static_cast<size_t>(15)));
+  {
+    int L = 1;
+    while (4 * L < E) L <<= 1;
+    const int per_warp = 32 / L;
+    const int ntc = min(p.tb, T - tc0);
+    const int gl = lane & (L - 1);
+    for (int base = warp * per_warp; base < ntc; base += kRouteWarps * per_warp) {
+      const int tl = base + lane / L;
+      const bool act = tl < ntc;
+      topk_group(p, s_logits + (act ? tl : 0) * E, tc0 + tl, act, gl, L,
+                 (one && staged) ? s_idx : nullptr, s_w);
     }
   }
 
   __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(ws.ticket, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // ---- phase 2 (one block): bucketing ------------------------------------
-  // Every token's selections are in global memory; they are staged in shared
-  // memory (one byte each) with coalesced loads, with the weights when they
-  // fit, and the token counters go back to zero for the next launch.
-  __shared__ uint8_t s_idx[kStageSel];
-  __shared__ float s_w[kStageW];
-  const bool sel_staged = T * k <= kStageSel;
-  const bool w_staged = T * k <= kStageW;
-  for (int j = threadIdx.x; j < T * k; j += kRouteThreads) {
-    if (sel_staged) s_idx[j] = static_cast<uint8_t>(__ldcg(ws.topk_idx + j));
-    if (w_staged) s_w[j] = __ldcg(ws.topk_w + j);
+  if (!one) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(ws.ticket, 1u) == static_cast<unsigned>(p.n_clusters - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (staged) {
+      // every selection, eight independent loads per thread in flight
+      const int n = T * k;
+      for (int j0 = threadIdx.x; j0 < n; j0 += 8 * kRouteThreads) {
+        int iv[8];
+        float wv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u * kRouteThreads;
+          iv[u] = j < n ? __ldcg(ws.topk_idx + j) : 0;
+          wv[u] = j < n ? __ldcg(ws.topk_w + j) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int j = j0 + u * kRouteThreads;
+          if (j < n) {
+            s_idx[j] = static_cast<uint8_t>(iv[u]);
+            s_w[j] = wv[u];
+          }
+        }
+      }
+    }
   }
-  for (int t = threadIdx.x; t < T; t += kRouteThreads) ws.tok_ctr[t] = 0u;
   __syncthreads();
-  auto sel_of = [&](int t, int j) -> int {
-    return sel_staged ? static_cast<int>(s_idx[t * k + j]) : __ldcg(ws.topk_idx + t * k + j);
+  // the slot of token t that selected expert e, or -1
+  auto slot_of = [&](int t, int e) -> int {
+    int slot = -1;
+    if (t < T)
+      for (int j = 0; j < k; ++j)
+        if ((staged ? static_cast<int>(s_idx[t * k + j]) : __ldcg(ws.topk_idx + t * k + j)) == e)
+          slot = j;
+    return slot;
   };
 
-  // ---- bucketing: counts per expert with warp ballots ---------------------
+  // ---- phase 3: counts per expert with warp ballots -----------------------
   __shared__ int s_cnt[kMaxGroups + 1];
   __shared__ int s_off[kMaxGroups + 2];
-  for (int e = warp; e < E; e += warps_per_block) {
+  for (int e = warp; e < E; e += kRouteWarps) {
     int cnt = 0;
-    for (int base = 0; base < T; base += 32) {
-      const int t = base + lane;
-      bool hit = false;
-      if (t < T)
-        for (int j = 0; j < k; ++j) hit |= (sel_of(t, j) == e);
-      cnt += __popc(__ballot_sync(kFull, hit));
-    }
+    for (int base = 0; base < T; base += 32)
+      cnt += __popc(__ballot_sync(kFull, slot_of(base + lane, e) >= 0));
     if (lane == 0) s_cnt[e] = cnt;
   }
   __syncthreads();
@@ -244,50 +422,45 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
         s_cnt[E] = T;
         s_off[E + 1] = routed + T;
       }
-      *ws.ticket = 0u;  // ready for the next forward (kernels on a stream do not overlap)
+      if (!one) *ws.ticket = 0u;  // ready for the next forward (kernels on a stream do not overlap)
     }
   }
   __syncthreads();
   for (int g = threadIdx.x; g <= G; g += kRouteThreads) ws.offsets[g] = s_off[g];
   for (int j = threadIdx.x; j < p.n_zero; j += kRouteThreads) p.zero_words[j] = 0;
 
-  // ---- bucketing: lists ordered by token ----------------------------------
+  // ---- phase 3: lists ordered by token ------------------------------------
   // With routing statistics on, the warp of expert e also sums the weights of
-  // e's slots (in double: per 32-token block a xor butterfly, blocks in token
-  // order) and adds its count and weight sum to the handle's counters; one
-  // warp owns each expert, so the counters need no atomics.
+  // e's slots (in double: each lane over its tokens in order, then a xor
+  // butterfly) and adds its count and weight sum to the handle's counters
+  // (reductions whose results are not waited for); one warp owns each
+  // expert, so every counter gets one addition per forward.
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int e = warp; e < E; e += warps_per_block) {
+  for (int e = warp; e < E; e += kRouteWarps) {
+    if (s_off[e + 1] == s_off[e]) continue;  // no token chose e: nothing to list or count
     int run = s_off[e];
     double mass = 0.0;
     for (int base = 0; base < T; base += 32) {
       const int t = base + lane;
-      int slot = -1;
-      if (t < T)
-        for (int j = 0; j < k; ++j)
-          if (sel_of(t, j) == e) slot = j;
+      const int slot = slot_of(t, e);
       const unsigned m = __ballot_sync(kFull, slot >= 0);
-      double wm = 0.0;
       if (slot >= 0) {
         const int pos = run + __popc(m & lt_mask);
+        const float w = staged ? s_w[t * k + slot] : __ldcg(ws.topk_w + t * k + slot);
         ws.slot_token[pos] = t;
         ws.token_pos[t * k + slot] = pos;
-        const float w = w_staged       ? s_w[t * k + slot]
-                        : p.stat_count ? __ldcg(ws.topk_w + t * k + slot)
-                                       : 0.0f;
-        if (w_staged) ws.slot_w[pos] = w;
-        wm = static_cast<double>(w);
-      }
-      if (p.stat_count) {
-#pragma unroll
-        for (int sh = 16; sh >= 1; sh >>= 1) wm += __shfl_xor_sync(kFull, wm, sh);
-        mass += wm;
+        ws.slot_w[pos] = w;
+        mass += static_cast<double>(w);
       }
       run += __popc(m);
     }
-    if (p.stat_count && lane == 0) {
-      p.stat_count[e] += static_cast<unsigned long long>(s_off[e + 1] - s_off[e]);
-      p.stat_mass[e] += mass;
+    if (p.stat_count) {
+#pragma unroll
+      for (int sh = 16; sh >= 1; sh >>= 1) mass += __shfl_xor_sync(kFull, mass, sh);
+      if (lane == 0) {
+        atomicAdd(p.stat_count + e, static_cast<unsigned long long>(s_off[e + 1] - s_off[e]));
+        atomicAdd(p.stat_mass + e, mass);
+      }
     }
   }
   if (p.has_shared) {
@@ -297,12 +470,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteParams 
       ws.slot_w[pos] = 1.0f;
       ws.token_pos[T * k + t] = pos;
     }
-  }
-  if (!w_staged) {
-    // routing weight of every routed position (independent loads, all threads)
-    __syncthreads();
-    for (int j = threadIdx.x; j < T * k; j += kRouteThreads)
-      ws.slot_w[__ldcg(ws.token_pos + j)] = __ldcg(ws.topk_w + j);
   }
 }
 
@@ -350,23 +517,47 @@ __global__ void gather_kernel(const GatherParams p) {
 
 // out[t] = sum_j ysorted[pos(t, j)] (+ shared) in slot order, summing the
 // split-K partials of each position in split order; fp32, rounded to bf16.
+// The positions are read first and the partials of up to eight (slot, split)
+// terms are loaded before any is added, so their latencies overlap; the sums
+// keep the slot-then-split order.
 __global__ void combine_kernel(const CombineParams p) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.y;
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (c >= p.H) return;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   const int nslots = p.k + (p.has_shared ? 1 : 0);
-  for (int j = 0; j < nslots; ++j) {
-    const int pos = (j < p.k) ? p.token_pos[t * p.k + j] : p.token_pos[p.T * p.k + t];
-    for (int s = 0; s < p.n_split; ++s) {
-      const float4 v = *reinterpret_cast<const float4*>(
-          p.ysorted + s * p.split_stride + static_cast<size_t>(pos) * p.H + c);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+  int pos[PW_MAX_TOPK + 1];
+#pragma unroll
+  for (int j = 0; j < PW_MAX_TOPK + 1; ++j)
+    pos[j] = j < p.k ? p.token_pos[t * p.k + j] : (j == p.k && p.has_shared ? p.token_pos[p.T * p.k + t] : 0);
+  const int terms = nslots * p.n_split;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q0 = 0; q0 < terms; q0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = q0 + i;
+      if (q < terms) {
+        const int j = q / p.n_split, s = q - j * p.n_split;
+        int pj = pos[0];
+#pragma unroll
+        for (int jj = 1; jj < PW_MAX_TOPK + 1; ++jj)
+          if (jj == j) pj = pos[jj];
+        v[i] = *reinterpret_cast<const float4*>(p.ysorted + s * p.split_stride +
+                                                static_cast<size_t>(pj) * p.H + c);
+      } else {
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (q0 + i < terms) {
+        acc.x += v[i].x;
+        acc.y += v[i].y;
+        acc.z += v[i].z;
+        acc.w += v[i].w;
+      }
     }
   }
   __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
@@ -377,15 +568,144 @@ __global__ void combine_kernel(const CombineParams p) {
   *reinterpret_cast<uint2*>(p.y + static_cast<size_t>(t) * p.H + c) = out;
 }
 
+// Launch of one router shape: the per-device shared-memory attribute is set
+// once (under a lock), then the grid goes out in clusters of p.cb blocks with
+// programmatic dependent launch.
+constexpr size_t kStageBudget = 96 * 1024;  // bytes of one staging buffer, at most
+constexpr size_t kRouteSmemMax = 2 * kStageBudget + 16 * 1024 + 32 * PW_MAX_EXPERTS * 4;
+
+template <int TT, int TE>
+cudaError_t launch_route_shape(const RouteParams& p, size_t smem, cudaStream_t s) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(route_kernel<TT, TE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kRouteSmemMax));
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_clusters * p.cb);
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.cb;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, route_kernel<TT, TE>, p);
+}
+
 }  // namespace
 
-cudaError_t launch_route(const RouteParams& p, int n_sm, cudaStream_t s) {
-  const int pairs = p.T * p.E;
-  const int warps = kRouteThreads / 32;
-  int grid = (pairs + warps - 1) / warps;
-  if (grid > 4 * n_sm) grid = 4 * n_sm;
-  if (grid < 1) grid = 1;
-  return launch_pdl(route_kernel, dim3(grid), dim3(kRouteThreads), 0, s, p);
+RouteGeometry route_geometry(int T, int E, int H, int k) {
+  RouteGeometry g{};
+  const bool big = T >= 256;
+  if (big) {
+    // many clusters: each block covers up to 8 experts of 16-32 tokens
+    const int cb0 = (E + 7) / 8 < 8 ? (E + 7) / 8 : 8;
+    g.eb = (E + cb0 - 1) / cb0;
+    g.ce = (E + g.eb - 1) / g.eb;
+    g.cb = g.ce;
+    g.tb = g.eb <= 8 ? 32 : 16;
+    g.tbb = g.tb;
+  } else {
+    // one cluster of up to 8 blocks per 16 tokens, split between token and
+    // expert groups so each block stages the fewest bytes
+    int tb = 1;
+    while (tb < T && tb < 16) tb *= 2;
+    g.tb = tb;
+    const int cb = E * tb < 8 ? E * tb : 8;
+    size_t best = ~static_cast<size_t>(0);
+    for (int ca = 1; ca <= cb; ca *= 2) {
+      if (cb % ca || ca > tb) continue;
+      const int ce = cb / ca;
+      if (ce > E) continue;
+      const int tbb = (tb + ca - 1) / ca, eb = (E + ce - 1) / ce;
+      const size_t bytes = static_cast<size_t>(tbb) * H * 2 + static_cast<size_t>(eb) * H * 4;
+      if (bytes < best) {
+        best = bytes;
+        g.ce = (E + eb - 1) / eb;  // expert groups that hold an expert
+        g.cb = ca * g.ce;
+        g.tbb = tbb;
+        g.eb = eb;
+      }
+    }
+  }
+  // the smallest register tile that needs at most one task per warp
+  static const int kTiles[][2] = {{1, 1}, {2, 1}, {1, 4}, {4, 1}, {2, 4},
+                                  {8, 1}, {1, 8}, {4, 4}, {2, 8}, {4, 8}};
+  g.tt = 0;
+  for (const auto& tl : kTiles) {
+    const int tasks = ((g.tbb + tl[0] - 1) / tl[0]) * ((g.eb + tl[1] - 1) / tl[1]);
+    if (tasks <= kRouteWarps) {
+      g.tt = tl[0];
+      g.te = tl[1];
+      break;
+    }
+  }
+  const int per_col = 2 * g.tbb + 4 * g.eb;
+  int kc = static_cast<int>(kStageBudget / per_col) & ~31;
+  if (kc < 32) kc = 32;
+  const int h32 = (H + 31) & ~31;
+  if (kc > h32) kc = h32;
+  g.kc = kc;
+  const int n_chunks = (H + kc - 1) / kc;
+  const size_t xbytes = (static_cast<size_t>(g.tbb) * kc * 2 + 15) & ~static_cast<size_t>(15);
+  const size_t stage = (n_chunks > 1 ? 2 : 1) * (xbytes + static_cast<size_t>(g.eb) * kc * 4);
+  const size_t tk = static_cast<size_t>(T) * k;
+  const size_t sel = ((tk + 15) & ~static_cast<size_t>(15)) + 4 * tk;
+  g.sel_staged = sel <= 2 * kStageBudget;
+  size_t region = stage;
+  if (g.sel_staged && sel > region) region = sel;
+  g.logits_off = (region + 15) & ~static_cast<size_t>(15);
+  g.smem = g.logits_off + static_cast<size_t>(g.tb) * E * 4;
+  g.n_clusters = T > 0 ? (T + g.tb - 1) / g.tb : 1;
+  return g;
+}
+
+cudaError_t launch_route(const RouteParams& p_in, int n_sm, cudaStream_t s) {
+  (void)n_sm;
+  RouteParams p = p_in;
+  const RouteGeometry g = route_geometry(p.T, p.E, p.H, p.k);
+  if (g.tt == 0 || g.smem > kRouteSmemMax) return cudaErrorInvalidConfiguration;
+  p.cb = g.cb;
+  p.ce = g.ce;
+  p.tb = g.tb;
+  p.tbb = g.tbb;
+  p.eb = g.eb;
+  p.kc = g.kc;
+  p.n_clusters = g.n_clusters;
+  p.logits_off = static_cast<int>(g.logits_off);
+  p.sel_staged = g.sel_staged ? 1 : 0;
+  p.vec = (p.H % 8 == 0) && (reinterpret_cast<uintptr_t>(p.x) % 16 == 0) &&
+          (reinterpret_cast<uintptr_t>(p.wr) % 16 == 0);
+  switch (g.tt * 16 + g.te) {
+    case 0x11: return launch_route_shape<1, 1>(p, g.smem, s);
+    case 0x21: return launch_route_shape<2, 1>(p, g.smem, s);
+    case 0x14: return launch_route_shape<1, 4>(p, g.smem, s);
+    case 0x41: return launch_route_shape<4, 1>(p, g.smem, s);
+    case 0x24: return launch_route_shape<2, 4>(p, g.smem, s);
+    case 0x81: return launch_route_shape<8, 1>(p, g.smem, s);
+    case 0x18: return launch_route_shape<1, 8>(p, g.smem, s);
+    case 0x44: return launch_route_shape<4, 4>(p, g.smem, s);
+    case 0x28: return launch_route_shape<2, 8>(p, g.smem, s);
+    case 0x48: return launch_route_shape<4, 8>(p, g.smem, s);
+    default: return cudaErrorInvalidConfiguration;
+  }
 }
 
 cudaError_t launch_gather(const GatherParams& p, int max_rows, int n_sm, cudaStream_t s) {

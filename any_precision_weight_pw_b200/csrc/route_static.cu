@@ -27,22 +27,18 @@ namespace {
 // Carve of the scratch (every piece 256-byte aligned).
 constexpr size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 constexpr int kMaxT = PW_ROUTE_STATIC_MAX_TOKENS;
-constexpr size_t kLogitsOff = 0;
-constexpr size_t kLogitsBytes = align256(sizeof(float) * kMaxT * PW_MAX_EXPERTS);
-constexpr size_t kOffsetsOff = kLogitsOff + kLogitsBytes;
+constexpr size_t kOffsetsOff = 0;
 constexpr size_t kOffsetsBytes = align256(sizeof(int32_t) * (PW_MAX_EXPERTS + 2));
 constexpr size_t kSlotTokOff = kOffsetsOff + kOffsetsBytes;
 constexpr size_t kSlotBytes = align256(sizeof(int32_t) * kMaxT * PW_MAX_TOPK);
 constexpr size_t kSlotWOff = kSlotTokOff + kSlotBytes;
 constexpr size_t kTokPosOff = kSlotWOff + kSlotBytes;
-constexpr size_t kTokCtrOff = kTokPosOff + kSlotBytes;
-constexpr size_t kTokCtrBytes = align256(sizeof(uint32_t) * kMaxT);
-constexpr size_t kTicketOff = kTokCtrOff + kTokCtrBytes;
+constexpr size_t kTicketOff = kTokPosOff + kSlotBytes;
 constexpr size_t kScratchBytes = kTicketOff + 256;
 static_assert(kScratchBytes == PW_ROUTE_STATIC_SCRATCH_BYTES, "pw.h states the scratch size");
 
-// Zero at module load; the route kernel puts its ticket and token counters
-// back to zero at the end of every launch, so the next call finds them ready.
+// Zero at module load; the route kernel puts its ticket back to zero at the
+// end of every launch that uses it, so the next call finds it ready.
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -106,7 +102,6 @@ extern "C" pw_status_t pw_route_static(const uint16_t* d_x, const float* d_route
   rp.k = top_k;
   rp.renorm = renorm_topk;
   rp.has_shared = 0;
-  rp.ws.logits = reinterpret_cast<float*>(base + kLogitsOff);
   rp.ws.topk_idx = d_idx;
   rp.ws.topk_w = d_w;
   rp.ws.offsets = reinterpret_cast<int32_t*>(base + kOffsetsOff);
@@ -114,7 +109,6 @@ extern "C" pw_status_t pw_route_static(const uint16_t* d_x, const float* d_route
   rp.ws.slot_w = reinterpret_cast<float*>(base + kSlotWOff);
   rp.ws.token_pos = reinterpret_cast<int32_t*>(base + kTokPosOff);
   rp.ws.ticket = reinterpret_cast<uint32_t*>(base + kTicketOff);
-  rp.ws.tok_ctr = reinterpret_cast<uint32_t*>(base + kTokCtrOff);
   e = pw::launch_route(rp, n_sm, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return pw::record_error(PW_ERR_CUDA, cudaGetErrorString(e));
   return PW_OK;

@@ -44,11 +44,15 @@
 //               two buffers, alternating items, gate and up side by side).
 //   warps 11-14 epilogue: tcgen05.ld the accumulators; write h = silu(g)*u
 //               as fp16 in the down pass's K order (gate/up), the routing-
-//               weighted fp32 partials (down), g (prefill gate) or the fp32
-//               result (linear).
+//               weighted fp32 partials (down), g as fp16 (prefill gate) or
+//               the fp32 result (linear).
 // The forward's kernels are launched with programmatic dependent launch;
-// this kernel waits for its predecessor before it reads anything and does
-// not release its successor early.
+// this kernel waits for its predecessor before it reads anything and
+// releases its successor at once: the successor's blocks can only take an
+// SM that one of this grid's CTAs has left (all of them are resident by
+// then, one per SM, and no other block fits beside one), where they wait
+// for this grid to finish, so the successor's launch latency hides behind
+// this kernel's tail.
 // Every wait is an mbarrier try_wait (with a suspend hint, so waiting warps
 // do not spin) bounded by a global-timer deadline; a timeout raises the CTA's
 // abort flag and the device error word, and every role drains what it has in
@@ -212,6 +216,22 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           dst),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+// The same with an L2 policy (the decode configuration streams each plane
+// page once per forward: evict-first keeps the L2 for the data and code the
+// other kernels of the forward reuse).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes,
+                                               uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
@@ -713,9 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   const int lane = threadIdx.x & 31;
   const int G = (p.mode == kTcLinear) ? 1 : p.n_groups;
   // everything below reads what earlier kernels of the forward wrote (or
-  // writes what they read); the successor is not released early, so it
-  // cannot take SM resources while the grid's CTAs wait on one another
+  // writes what they read); the successor may launch once every CTA of this
+  // grid has released it here, i.e. once all of them are resident
   pdl_wait();
+  pdl_trigger();
   // group offsets into shared memory with one parallel load (the item
   // counts below and every item decode read them)
   if (p.mode != kTcLinear)
@@ -839,6 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       uint32_t t = 0, ring_end = 0;
       int gh[2] = {0, 0};
       bool ok = true;
+      const uint64_t stream_pol = l2_evict_first_policy();
       for (int i = blockIdx.x; i < total && ok; i += gridDim.x) {
         Item it;
         decode_item<C>(p, s_prefix, s_prefix2, G, i, it, gh);
@@ -874,8 +896,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             const int64_t grp_idx = static_cast<int64_t>(rt) * n_kt + s;
             const uint32_t bytes = static_cast<uint32_t>(ps.bits) * kSlotBytes;
             mbar_arrive_tx(&sf[e], bytes);
-            bulk_load(smem_addr(smem + C::kOffSlots + start * kSlotBytes),
-                      ps.planes + grp_idx * ps.stride * (kSlotBytes / 4), bytes, &sf[e]);
+            if constexpr (C::kPrefill)  // row tiles are shared by several CTAs' token chunks
+              bulk_load(smem_addr(smem + C::kOffSlots + start * kSlotBytes),
+                        ps.planes + grp_idx * ps.stride * (kSlotBytes / 4), bytes, &sf[e]);
+            else
+              bulk_load_hint(smem_addr(smem + C::kOffSlots + start * kSlotBytes),
+                             ps.planes + grp_idx * ps.stride * (kSlotBytes / 4), bytes, &sf[e],
+                             stream_pol);
           }
         }
       }
@@ -1068,15 +1095,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
         const bool up = p.mode == kTcPfUp;
         // gate values of the next 16-token chunk are loaded one chunk ahead
         // (the first chunk's before the accumulator is ready), so their
-        // latency hides behind the MMAs and the previous chunk's work
+        // latency hides behind the MMAs and the previous chunk's work; they
+        // stay raw fp16 bits until used, so no instruction waits on a load
+        // before the chunk that needs it
         constexpr int kCh = 16;
-        float gn[kCh];
+        uint16_t gn[kCh];
         auto load_g = [&](int c) {
           const int nv = min(kCh, it.ntok - kCh * c);
           const int pos = it.pos0 + kCh * c;
 #pragma unroll
           for (int n = 0; n < kCh; ++n)
-            gn[n] = (live && n < nv) ? p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] : 0.0f;
+            gn[n] = (live && n < nv) ? p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o]
+                                     : static_cast<uint16_t>(0);
         };
         if (up) load_g(0);
         const uint32_t jd = d_ctr % kNDBuf;
@@ -1089,7 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
           if (kCh * c >= it.ntok) break;
           uint32_t v[kCh];
           tmem_ld16(tmem_lane + jd * C::kDColsPerBuf + kCh * c, v);
-          float g[kCh];
+          uint16_t g[kCh];
           if (up) {
 #pragma unroll
             for (int n = 0; n < kCh; ++n) g[n] = gn[n];
@@ -1103,7 +1133,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
 #pragma unroll
             for (int n = 0; n < kCh; ++n) {
               if (n >= nv) break;
-              p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] = __uint_as_float(v[n]);
+              p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o] =
+                  __half_as_ushort(__float2half_rn(__uint_as_float(v[n])));
             }
           } else if (up) {
 #pragma unroll
@@ -1111,7 +1142,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
               if (n >= nv) break;
               // the accumulator waits for this epilogue (one buffer), so the
               // activation uses the fast exponential and division
-              const float h = __fdividef(g[n], 1.0f + __expf(-g[n])) * __uint_as_float(v[n]);
+              const float gf = __half2float(__ushort_as_half(g[n]));
+              const float h = __fdividef(gf, 1.0f + __expf(-gf)) * __uint_as_float(v[n]);
               hp[static_cast<size_t>(pos + n) * 64] = __half_as_ushort(__float2half_rn(h));
             }
           } else {

@@ -14,7 +14,7 @@ constexpr int kTcGateUp = 0;    // gate and up blocks of every group -> h = silu
 constexpr int kTcDown = 1;      // down blocks, B = h -> routing-weighted partials
 constexpr int kTcLinear = 2;    // one standalone block -> y
 // prefill modes (256-token chunks; gate and up in separate launches)
-constexpr int kTcPfGate = 3;    // gate blocks -> g (fp32, gbuf)
+constexpr int kTcPfGate = 3;    // gate blocks -> g (fp16, gbuf)
 constexpr int kTcPfUp = 4;      // up blocks -> h = silu(g) * u (h_perm)
 constexpr int kTcPfDown = 5;    // down blocks -> routing-weighted outputs (ysorted)
 // decode, both passes in one launch: gate/up items, then down items; a down
@@ -47,7 +47,7 @@ struct TcParams {
   const uint32_t* lin_planes;    // plane pages of the standalone block (mode 2)
   int* gu_done;                   // fused mode: per group, 4 x gate/up items written
                                  // (zero at launch)
-  float* gbuf;                   // prefill: gate outputs [rows][gbuf_ld] fp32
+  uint16_t* gbuf;                // prefill: gate outputs [rows][gbuf_ld] fp16
   int gbuf_ld;
   int* err;                      // device error word (may be null)
   int cooperative;               // fused mode: launch with the cooperative attribute

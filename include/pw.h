@@ -366,7 +366,7 @@ int32_t pw_forward_launches(const pw_moe_t* h, int32_t T);
  * the caller serialises calls per device, e.g. by issuing them all on one
  * stream. */
 #define PW_ROUTE_STATIC_MAX_TOKENS 256
-#define PW_ROUTE_STATIC_SCRATCH_BYTES 157696 /* logits 128 KB + lists and counters */
+#define PW_ROUTE_STATIC_SCRATCH_BYTES 25600 /* offsets, per-expert lists and a ticket */
 pw_status_t pw_route_static(const uint16_t* d_x, const float* d_router_w,
                             const float* d_router_bias, int32_t T, int32_t hidden,
                             int32_t n_experts, int32_t top_k, int32_t renorm_topk,

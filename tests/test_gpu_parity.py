@@ -674,10 +674,10 @@ def test_workspace_is_sized_to_its_use(pw):
     cfg = dict(hidden=wl.hidden, ffn=wl.ffn, n_experts=wl.n_experts, top_k=wl.top_k,
                shared_ffn=0, n_max=8, renorm_topk=1, max_tokens=4096)
     big = pw.workspace_bytes(cfg)
-    # gate outputs (fp32) + SwiGLU activations (fp16) + gathered rows (fp16)
+    # gate outputs (fp16) + SwiGLU activations (fp16) + gathered rows (fp16)
     # + the host-forward staging rows (bf16 in and out)
     P = 4096 * 2
-    core = P * wl.ffn * 4 + P * wl.ffn * 2 + P * wl.hidden * 2 + 2 * 4096 * wl.hidden * 2
+    core = P * wl.ffn * 2 + P * wl.ffn * 2 + P * wl.hidden * 2 + 2 * 4096 * wl.hidden * 2
     assert core <= big <= core + 64 * 2 ** 20, (big, core)
     small = pw.workspace_bytes(dict(cfg, max_tokens=16))
     assert small < 64 * 2 ** 20

@@ -89,3 +89,32 @@ def test_rejects_more_tokens_than_the_scratch_holds(pw):
     x = torch.zeros((257, wl.hidden), dtype=torch.int16, device="cuda")
     with pytest.raises(pw.PwError):
         pw.route_static(x, wr, wl.top_k, wl.renorm_topk)
+
+
+@pytest.mark.parametrize("T,E,H,k,bias", [
+    (1, 9, 100, 2, False),      # hidden not a multiple of 8: plain staging loads
+    (5, 7, 7, 3, True),         # hidden below one 32-column step
+    (17, 1, 64, 1, False),      # one expert
+    (33, 100, 264, 4, True),    # 13 experts per block, several clusters
+    (200, 3, 40, 2, False),     # three single-expert blocks, 13 clusters
+    (256, 60, 2048, 4, False),  # prefill geometry: 32-token clusters, 4 x 8 tiles
+    (256, 128, 520, 8, True),   # 128 experts, 16 per block, several column chunks
+])
+def test_route_geometries_match_oracle(pw, oracle, T, E, H, k, bias):
+    """Every launch geometry of the router (cluster size, tokens per cluster,
+    register tile, column chunks, plain or 16-byte staging) gives the oracle's
+    selections exactly; rows of zeros make every logit tie (lower index wins)."""
+    rng = np.random.default_rng(T * 1000 + E)
+    xf = rng.standard_normal((T, H)).astype(np.float32)
+    xf[::4] = 0.0
+    x_h = (xf.view(np.uint32) >> 16).astype(np.uint16)   # bf16 by truncation
+    wr_h = (rng.standard_normal((E, H)) / np.sqrt(H)).astype(np.float32)
+    b_h = (0.5 * rng.standard_normal(E)).astype(np.float32) if bias else None
+    x = torch.from_numpy(x_h.view(np.int16)).cuda()
+    wr = torch.from_numpy(wr_h).cuda()
+    b = None if b_h is None else torch.from_numpy(b_h).cuda()
+    i, w = pw.route_static(x, wr, k, 1, router_bias=b)
+    torch.cuda.synchronize()
+    oi, ow = oracle.topk_softmax(oracle.router_logits(x_h, wr_h, b_h), k, True)
+    np.testing.assert_array_equal(i.cpu().numpy(), oi)
+    np.testing.assert_allclose(w.cpu().numpy(), ow, rtol=1e-5, atol=1e-7)
