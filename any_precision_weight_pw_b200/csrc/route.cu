@@ -517,47 +517,23 @@ __global__ void gather_kernel(const GatherParams p) {
 
 // out[t] = sum_j ysorted[pos(t, j)] (+ shared) in slot order, summing the
 // split-K partials of each position in split order; fp32, rounded to bf16.
-// The positions are read first and the partials of up to eight (slot, split)
-// terms are loaded before any is added, so their latencies overlap; the sums
-// keep the slot-then-split order.
 __global__ void combine_kernel(const CombineParams p) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.y;
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (c >= p.H) return;
-  const int nslots = p.k + (p.has_shared ? 1 : 0);
-  int pos[PW_MAX_TOPK + 1];
-#pragma unroll
-  for (int j = 0; j < PW_MAX_TOPK + 1; ++j)
-    pos[j] = j < p.k ? p.token_pos[t * p.k + j] : (j == p.k && p.has_shared ? p.token_pos[p.T * p.k + t] : 0);
-  const int terms = nslots * p.n_split;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int q0 = 0; q0 < terms; q0 += 8) {
-    float4 v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int q = q0 + i;
-      if (q < terms) {
-        const int j = q / p.n_split, s = q - j * p.n_split;
-        int pj = pos[0];
-#pragma unroll
-        for (int jj = 1; jj < PW_MAX_TOPK + 1; ++jj)
-          if (jj == j) pj = pos[jj];
-        v[i] = *reinterpret_cast<const float4*>(p.ysorted + s * p.split_stride +
-                                                static_cast<size_t>(pj) * p.H + c);
-      } else {
-        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (q0 + i < terms) {
-        acc.x += v[i].x;
-        acc.y += v[i].y;
-        acc.z += v[i].z;
-        acc.w += v[i].w;
-      }
+  const int nslots = p.k + (p.has_shared ? 1 : 0);
+  for (int j = 0; j < nslots; ++j) {
+    const int pos = (j < p.k) ? p.token_pos[t * p.k + j] : p.token_pos[p.T * p.k + t];
+    for (int s = 0; s < p.n_split; ++s) {
+      const float4 v = *reinterpret_cast<const float4*>(
+          p.ysorted + s * p.split_stride + static_cast<size_t>(pos) * p.H + c);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
   }
   __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
@@ -567,6 +543,7 @@ __global__ void combine_kernel(const CombineParams p) {
   out.y = *reinterpret_cast<uint32_t*>(&hi);
   *reinterpret_cast<uint2*>(p.y + static_cast<size_t>(t) * p.H + c) = out;
 }
+
 
 // Launch of one router shape: the per-device shared-memory attribute is set
 // once (under a lock), then the grid goes out in clusters of p.cb blocks with
