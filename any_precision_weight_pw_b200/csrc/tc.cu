@@ -237,6 +237,11 @@ __device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void* src, ui
       "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint64_t* bar) {
   asm volatile(
@@ -1144,9 +1149,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             for (int n = 0; n < kCh; ++n) {
               if (n >= nv) break;
               // the accumulator waits for this epilogue (one buffer), so the
-              // activation uses the fast exponential and division
+              // activation takes one special-function instruction:
+              // silu(g) = g sigmoid(g) = g (1 + tanh(g / 2)) / 2, with the
+              // hardware tanh approximation (h is rounded to fp16 anyway)
               const float gf = __half2float(__ushort_as_half(g[n]));
-              const float h = __fdividef(gf, 1.0f + __expf(-gf)) * __uint_as_float(v[n]);
+              const float hg = 0.5f * gf;
+              const float h = fmaf(hg, tanh_approx(hg), hg) * __uint_as_float(v[n]);
               hp[static_cast<size_t>(pos + n) * 64] = __half_as_ushort(__float2half_rn(h));
             }
           } else {
