@@ -1116,7 +1116,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             gn[n] = (live && n < nv) ? p.gbuf[static_cast<size_t>(pos + n) * p.gbuf_ld + o]
                                      : static_cast<uint16_t>(0);
         };
+        // down: the routing weights of the next chunk's tokens, one chunk
+        // ahead likewise (loaded when used, each chunk waited on L2)
+        const bool down = p.mode == kTcPfDown;
+        float wn[kCh];
+        auto load_w = [&](int c) {
+          const int nv = min(kCh, it.ntok - kCh * c);
+          const int pos = it.pos0 + kCh * c;
+#pragma unroll
+          for (int n = 0; n < kCh; ++n) wn[n] = n < nv ? p.slot_w[pos + n] : 0.0f;
+        };
         if (up) load_g(0);
+        if (down) load_w(0);
         const uint32_t jd = d_ctr % kNDBuf;
         if (!mbar_wait_warp(&df[jd], (d_ctr / kNDBuf) & 1u, ctl)) break;
         tc_fence_after();
@@ -1128,10 +1139,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
           uint32_t v[kCh];
           tmem_ld16(tmem_lane + jd * C::kDColsPerBuf + kCh * c, v);
           uint16_t g[kCh];
+          float w[kCh];
           if (up) {
 #pragma unroll
             for (int n = 0; n < kCh; ++n) g[n] = gn[n];
             if (kCh * (c + 1) < it.ntok) load_g(c + 1);
+          }
+          if (down) {
+#pragma unroll
+            for (int n = 0; n < kCh; ++n) w[n] = wn[n];
+            if (kCh * (c + 1) < it.ntok) load_w(c + 1);
           }
           tmem_wait_ld();
           if (!live) continue;
@@ -1161,8 +1178,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
 #pragma unroll
             for (int n = 0; n < kCh; ++n) {
               if (n >= nv) break;
-              p.ysorted[static_cast<size_t>(pos + n) * p.H + o] =
-                  p.slot_w[pos + n] * __uint_as_float(v[n]);
+              p.ysorted[static_cast<size_t>(pos + n) * p.H + o] = w[n] * __uint_as_float(v[n]);
             }
           }
         }
