@@ -773,6 +773,9 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_rows = h->P_max;
     tp.err = h->err;
     tp.test_stall_group = -1;
+    // a group's token tile holds at most T rows: small batches get a deeper
+    // token-tile ring in the same shared memory
+    tp.b_slots = T <= 8 ? 16 : (T <= 16 ? 8 : 4);
     if (fused) {
       // test switches: a shorter wait limit, and one group's down items
       // waiting for a count that never arrives (failure-detection tests)
@@ -791,7 +794,7 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
       tp.split_stride = split_stride;
     }
     if (prefill) {
-      // gate -> g (fp32), then up -> h = silu(g) * u
+      // gate -> g (fp16), then up -> h = silu(g) * u
       tp.pf_map = h->x_pf_map;
       tp.gbuf = h->gbuf;
       tp.gbuf_ld = h->gbuf_ld;

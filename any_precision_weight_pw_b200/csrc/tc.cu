@@ -108,7 +108,9 @@ struct Cfg {
   static constexpr int kBStageK = PF ? 64 : 128;
   static constexpr int kBStageBytes = kNT * kBStageK * 2;
   static constexpr int kBPerStage = 256 / kBStageK;
-  static constexpr int kNB = PF ? 3 : 4;        // token-tile ring depth
+  static constexpr int kNB = PF ? 3 : 4;        // token-tile ring depth (slots of kBStageBytes)
+  static constexpr int kNBB = PF ? kNB : 16;    // token-tile barrier pairs (decode: up to 16
+                                                // slots when the launch's tiles are small)
   static constexpr int kNA = PF ? 4 : 6;        // TMEM A ring slots (128 K each)
   static constexpr int kNDBuf = PF ? 1 : 2;     // accumulator buffers
   static constexpr int kDColsPerBuf = PF ? 256 : 64;
@@ -116,7 +118,7 @@ struct Cfg {
   static constexpr uint32_t kOffSlots = kOffLut + kLutBytes;
   static constexpr uint32_t kOffB = kOffSlots + kNSlot * kSlotBytes;
   static constexpr uint32_t kOffBars = kOffB + kNB * kBStageBytes;
-  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNB + 2 * kNA + 2 * kNDBuf + 1 + 4;
+  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNBB + 2 * kNA + 2 * kNDBuf + 1 + 4;
   static constexpr uint32_t kOffMisc = kOffBars + kNumBars * 8;
   // misc: tmem holder, abort flag, then s_prefix, s_prefix2 and the group
   // offsets (kMaxGroups + 2 ints each)
@@ -723,8 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   uint64_t* sf = bars;      // plane stage full (bulk copy landed)
   uint64_t* se = sf + kNS;  // plane stage empty (all dequantisers read it)
   uint64_t* bfull = se + kNS;
-  uint64_t* bempty = bfull + kNB;
-  uint64_t* af = bempty + kNB;
+  uint64_t* bempty = bfull + C::kNBB;
+  uint64_t* af = bempty + C::kNBB;
   uint64_t* ae = af + kNA;
   uint64_t* df = ae + kNA;
   uint64_t* de = df + kNDBuf;
@@ -740,6 +742,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = (p.mode == kTcLinear) ? 1 : p.n_groups;
+  // token-tile ring: the prefill configuration has kNB slots; at decode the
+  // ring's kNB * kBStageBytes hold 4, 8 or 16 slots by the launch's tile rows
+  const uint32_t nb_lg = C::kPrefill ? 0u : (p.b_slots == 16 ? 4u : (p.b_slots == 8 ? 3u : 2u));
+  const uint32_t nb = C::kPrefill ? static_cast<uint32_t>(kNB) : (1u << nb_lg);
+  const uint32_t b_bytes = C::kPrefill ? static_cast<uint32_t>(C::kBStageBytes)
+                                       : static_cast<uint32_t>(kNB * C::kBStageBytes) >> nb_lg;
+  auto b_slot = [&](uint32_t c) -> uint32_t { return C::kPrefill ? c % kNB : (c & (nb - 1u)); };
+  auto b_par = [&](uint32_t c) -> uint32_t { return C::kPrefill ? (c / kNB) & 1u : (c >> nb_lg) & 1u; };
   // everything below reads what earlier kernels of the forward wrote (or
   // writes what they read); the successor may launch once every CTA of this
   // grid has released it here, i.e. once all of them are resident
@@ -756,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       mbar_init(&sf[i], 1);
       mbar_init(&se[i], kDqThreads / 32);
     }
-    for (int i = 0; i < kNB; ++i) {
+    for (int i = 0; i < C::kNBB; ++i) {
       mbar_init(&bfull[i], p.mode == kTcLinear ? 32 : 1);
       mbar_init(&bempty[i], 1);
     }
@@ -937,12 +947,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
       for (int q = 0; q < it.npass && ok; ++q) {
         for (int s = it.s_begin; s < it.s_end && ok; ++s) {
           for (int j = 0; j < C::kBPerStage; ++j) {
-            const uint32_t jb = b_ctr % kNB;
-            if (!mbar_wait_warp(&bempty[jb], ((b_ctr / kNB) & 1u) ^ 1u, ctl)) {
+            const uint32_t jb = b_slot(b_ctr);
+            if (!mbar_wait_warp(&bempty[jb], b_par(b_ctr) ^ 1u, ctl)) {
               ok = false;
               break;
             }
-            const uint32_t buf = smem_addr(smem + C::kOffB + jb * C::kBStageBytes);
+            const uint32_t buf = smem_addr(smem + C::kOffB + jb * b_bytes);
             if constexpr (C::kPrefill) {
               if (lane == 0) {
                 // {64 columns, 256 rows, 1 atom}: atom 4 s + j of the chunk's rows
@@ -965,8 +975,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
     }
     if (!ok && lane == 0 && p.mode != kTcLinear) {
       // let issued copies land before the CTA's shared memory goes away
-      const uint32_t lo = b_ctr > kNB ? b_ctr - kNB : 0u;
-      for (uint32_t c = lo; c < b_ctr; ++c) mbar_drain(&bfull[c % kNB], (c / kNB) & 1u);
+      const uint32_t lo = b_ctr > nb ? b_ctr - nb : 0u;
+      for (uint32_t c = lo; c < b_ctr; ++c) mbar_drain(&bfull[b_slot(c)], b_par(c));
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------ MMA issuer
@@ -997,14 +1007,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
             const uint32_t at = tmem_base + C::kAColBase + qa * kAColsPerSlot;
             // two 64-column B stages per 128-column A slot
             for (int j = 0; j < 2; ++j) {
-              const uint32_t jb = b_ctr % kNB;
-              if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+              const uint32_t jb = b_slot(b_ctr);
+              if (!mbar_wait_warp(&bfull[jb], b_par(b_ctr), ctl)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              const uint64_t bdesc =
-                  smem_desc_sw128(smem_addr(smem + C::kOffB + jb * C::kBStageBytes));
+              const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + C::kOffB + jb * b_bytes));
               if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
@@ -1044,8 +1053,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
           for (int s = it.s_begin; s < it.s_end && ok; ++s) {
             // each 128-column half of the stage: one B stage, one A slot
             for (int sub = 0; sub < 2; ++sub) {
-              const uint32_t jb = b_ctr % kNB;
-              if (!mbar_wait_warp(&bfull[jb], (b_ctr / kNB) & 1u, ctl)) {
+              const uint32_t jb = b_slot(b_ctr);
+              if (!mbar_wait_warp(&bfull[jb], b_par(b_ctr), ctl)) {
                 ok = false;
                 break;
               }
@@ -1055,8 +1064,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
                 break;
               }
               tc_fence_after();
-              const uint64_t bdesc =
-                  smem_desc_sw128(smem_addr(smem + C::kOffB + jb * C::kBStageBytes));
+              const uint64_t bdesc = smem_desc_sw128(smem_addr(smem + C::kOffB + jb * b_bytes));
               const uint32_t at = tmem_base + C::kAColBase + qa * kAColsPerSlot;
               if (leader) {
                 // K step kk: atom kk / 4 of the B stage, 32 bytes per 16
