@@ -773,9 +773,6 @@ static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
     tp.h_rows = h->P_max;
     tp.err = h->err;
     tp.test_stall_group = -1;
-    // a group's token tile holds at most T rows: small batches get a deeper
-    // token-tile ring in the same shared memory
-    tp.b_slots = T <= 8 ? 16 : (T <= 16 ? 8 : 4);
     if (fused) {
       // test switches: a shorter wait limit, and one group's down items
       // waiting for a count that never arrives (failure-detection tests)

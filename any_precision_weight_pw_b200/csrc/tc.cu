@@ -742,14 +742,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = (p.mode == kTcLinear) ? 1 : p.n_groups;
-  // token-tile ring: the prefill configuration has kNB slots; at decode the
-  // ring's kNB * kBStageBytes hold 4, 8 or 16 slots by the launch's tile rows
-  const uint32_t nb_lg = C::kPrefill ? 0u : (p.b_slots == 16 ? 4u : (p.b_slots == 8 ? 3u : 2u));
-  const uint32_t nb = C::kPrefill ? static_cast<uint32_t>(kNB) : (1u << nb_lg);
-  const uint32_t b_bytes = C::kPrefill ? static_cast<uint32_t>(C::kBStageBytes)
-                                       : static_cast<uint32_t>(kNB * C::kBStageBytes) >> nb_lg;
-  auto b_slot = [&](uint32_t c) -> uint32_t { return C::kPrefill ? c % kNB : (c & (nb - 1u)); };
-  auto b_par = [&](uint32_t c) -> uint32_t { return C::kPrefill ? (c / kNB) & 1u : (c >> nb_lg) & 1u; };
   // everything below reads what earlier kernels of the forward wrote (or
   // writes what they read); the successor may launch once every CTA of this
   // grid has released it here, i.e. once all of them are resident
@@ -760,6 +752,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_kernel(const __grid_constant__
   if (p.mode != kTcLinear)
     for (int g = threadIdx.x; g <= G; g += blockDim.x) s_offs[g] = p.offsets[g];
   __syncthreads();
+  // token-tile ring: the prefill configuration has kNB slots; at decode the
+  // ring's kNB * kBStageBytes hold 4, 8 or 16 slots by the largest token
+  // tile of this launch (every CTA derives the same count from the offsets)
+  uint32_t nb_lg = 2u;
+  if (!C::kPrefill && p.mode != kTcLinear) {
+    int maxn = 0;
+    for (int g = 0; g < G; ++g) maxn = max(maxn, s_offs[g + 1] - s_offs[g]);
+    nb_lg = maxn <= 8 ? 4u : (maxn <= 16 ? 3u : 2u);
+  }
+  const uint32_t nb = C::kPrefill ? static_cast<uint32_t>(kNB) : (1u << nb_lg);
+  const uint32_t b_bytes = C::kPrefill ? static_cast<uint32_t>(C::kBStageBytes)
+                                       : static_cast<uint32_t>(kNB * C::kBStageBytes) >> nb_lg;
+  auto b_slot = [&](uint32_t c) -> uint32_t { return C::kPrefill ? c % kNB : (c & (nb - 1u)); };
+  auto b_par = [&](uint32_t c) -> uint32_t { return C::kPrefill ? (c / kNB) & 1u : (c >> nb_lg) & 1u; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNS; ++i) {

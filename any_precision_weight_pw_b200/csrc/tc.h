@@ -51,9 +51,6 @@ struct TcParams {
   int gbuf_ld;
   int* err;                      // device error word (may be null)
   int cooperative;               // fused mode: launch with the cooperative attribute
-  int b_slots;                   // decode: token-tile ring slots, 4, 8 or 16 (0 = 4); with
-                                 // 8 (16) every token tile of the launch has at most 16 (8)
-                                 // rows and the ring's 32 KB hold twice (four times) as many
   unsigned long long wait_ns;    // limit of one device-side wait (0: 2 s)
   int test_stall_group;          // test switch: this group's down items wait for
                                  // a count that never arrives (-1: off)
