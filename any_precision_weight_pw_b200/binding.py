@@ -25,7 +25,7 @@ EXPORTED = ["pw_moe_create", "pw_set_block_bits", "pw_moe_forward", "pw_destroy"
             "pw_forward_launches", "pw_plane_bytes", "pw_repack_planes", "pw_route_static",
             "pw_get_forward_bits", "pw_set_switch_lag", "pw_routing_stats", "pw_plan_release",
             "pw_enable_paging", "pw_resident_bytes", "pw_workspace_bytes", "pw_compact_pages",
-            "pw_last_error", "pw_abi_version"]
+            "pw_last_error", "pw_abi_version", "pw_route_geometry"]
 
 
 class PwError(RuntimeError):
@@ -90,6 +90,7 @@ def lib():
         L.pw_plane_bytes.restype = C.c_int64
         L.pw_repack_planes.argtypes = [P, P, i32, i32, i32, P]
         L.pw_route_static.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P]
+        L.pw_route_geometry.argtypes = [i32, i32, i32, i32, C.POINTER(C.c_int64)]
         L.pw_last_error.restype = C.c_char_p
         L.pw_abi_version.restype = i32
         for name in EXPORTED:
@@ -161,6 +162,15 @@ def route_static(x, router_w, top_k: int, renorm_topk: int, router_bias=None, id
     check(lib().pw_route_static(_ptr(x), _ptr(router_w), _ptr(router_bias), T, H, E, top_k,
                                 renorm_topk, _ptr(idx), _ptr(w), _stream(stream)))
     return idx, w
+
+
+def route_geometry(T: int, E: int, H: int, top_k: int) -> dict:
+    """The route kernel's launch geometry for a shape (host arithmetic)."""
+    out = (C.c_int64 * 12)()
+    check(lib().pw_route_geometry(T, E, H, top_k, out))
+    keys = ("cb", "ce", "tb", "tbb", "eb", "kc", "n_clusters", "tt", "te", "sel_staged",
+            "logits_off", "smem")
+    return dict(zip(keys, list(out)))
 
 
 def workspace_bytes(cfg: dict) -> int:

@@ -113,3 +113,17 @@ extern "C" pw_status_t pw_route_static(const uint16_t* d_x, const float* d_route
   if (e != cudaSuccess) return pw::record_error(PW_ERR_CUDA, cudaGetErrorString(e));
   return PW_OK;
 }
+
+extern "C" pw_status_t pw_route_geometry(int32_t T, int32_t E, int32_t H, int32_t top_k,
+                                         int64_t* out) {
+  if (!out) return pw::record_error(PW_ERR_INVALID_ARG, "pw_route_geometry: null output");
+  if (T < 0 || E < 1 || E > PW_MAX_EXPERTS || H < 1 || top_k < 1 || top_k > E ||
+      top_k > PW_MAX_TOPK)
+    return pw::record_error(PW_ERR_INVALID_ARG, "pw_route_geometry: shape out of range");
+  const pw::RouteGeometry g = pw::route_geometry(T, E, H, top_k);
+  const int64_t v[12] = {g.cb, g.ce, g.tb, g.tbb, g.eb, g.kc, g.n_clusters, g.tt, g.te,
+                         g.sel_staged ? 1 : 0, static_cast<int64_t>(g.logits_off),
+                         static_cast<int64_t>(g.smem)};
+  for (int i = 0; i < 12; ++i) out[i] = v[i];
+  return PW_OK;
+}

@@ -365,6 +365,17 @@ int32_t pw_forward_launches(const pw_moe_t* h, int32_t T);
  * them, or several host threads) corrupt each other's scratch and results;
  * the caller serialises calls per device, e.g. by issuing them all on one
  * stream. */
+/* Launch geometry of the route kernel for T tokens, E experts, hidden H and
+ * top_k: pure host arithmetic (no device call, so it also runs without a
+ * GPU).  out[0..11] = blocks per cluster, expert groups per cluster, tokens
+ * per cluster, tokens per block, experts per block, columns per staged
+ * chunk, clusters, register-tile tokens, register-tile experts, selections
+ * staged in shared memory for the bucketing (0/1), shared-memory offset of
+ * the cluster's logits, dynamic shared memory bytes per block.
+ * PW_ERR_INVALID_ARG unless 0 <= T, 1 <= E <= 128, H >= 1 and
+ * 1 <= top_k <= min(E, 8). */
+pw_status_t pw_route_geometry(int32_t T, int32_t E, int32_t H, int32_t top_k, int64_t* out);
+
 #define PW_ROUTE_STATIC_MAX_TOKENS 256
 #define PW_ROUTE_STATIC_SCRATCH_BYTES 25600 /* offsets, per-expert lists and a ticket */
 pw_status_t pw_route_static(const uint16_t* d_x, const float* d_router_w,
