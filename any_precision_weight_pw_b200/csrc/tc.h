@@ -24,7 +24,7 @@ constexpr int kTcFused = 6;
 struct TcParams {
   CUtensorMap b_maps[4];         // token-tile source (modes 0, 1): x_sorted or h_perm
                                  // as {64 columns, rows, atoms}; box i holds 8(i+1)
-                                 // rows x 4 atoms, 128-byte swizzle
+                                 // rows x 2 atoms, 128-byte swizzle
   CUtensorMap pf_map;            // prefill modes: the same source, box 256 rows x 1 atom
   CUtensorMap h_maps[4];         // fused mode: the down items' source (h_perm)
   PageTable pt;                  // planes, bits, active LUT slot per block (modes 0, 1)

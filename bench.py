@@ -482,7 +482,7 @@ def paging_measure(dev, hbm_peak, T=16, n_fwd=200):
             "steps": rows_out}
 
 
-def prefill_measure(dev, steps=5, warmup=2):
+def prefill_measure(dev, steps=20, warmup=3):
     """The Mixtral-shaped layer at prefill scale (4096 tokens, Zipf-skewed
     routing): forward time with CUDA events, tokens/s and achieved TFLOP/s of
     the expert contractions (2 x 3 x H x F per routed slot) against the
@@ -749,9 +749,14 @@ def cpu_baseline(layer, x_np, T, budget_s=12.0):
         outs.append(o[0])
         done += 1
     dt = time.perf_counter() - t0
+    # the same oracle on one thread, one token (the per-core figure)
+    t1 = time.perf_counter()
+    L.forward(x_np[0:1], layer.router_w, layer.router_bias, threads=1)
+    one = 1.0 / (time.perf_counter() - t1)
     return ({"value": round(done / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
              "sample": "%d of the %d tokens of one batch, one token per oracle call, %.1f s"
-                       % (done, T, dt)}, outs)
+                       % (done, T, dt),
+             "one_thread_tokens_per_s": round(one, 4)}, outs)
 
 
 def run_reference(args):
