@@ -20,11 +20,33 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "pages.h"
 #include "pw_internal.h"
 #include "tc.h"
 
 namespace {
+
+// Host-side NVTX ranges around the calls a profiler should see (a forward, a
+// page move, paging and compaction); free when no tool is attached, and off
+// with PW_NVTX=0.
+struct NvtxRange {
+  bool on;
+  explicit NvtxRange(const char* name) : on(nvtx_on()) {
+    if (on) nvtxRangePushA(name);
+  }
+  ~NvtxRange() {
+    if (on) nvtxRangePop();
+  }
+  static bool nvtx_on() {
+    static const bool v = [] {
+      const char* e = std::getenv("PW_NVTX");
+      return !(e && e[0] == '0');
+    }();
+    return v;
+  }
+};
 
 thread_local std::string g_err;
 
@@ -536,6 +558,7 @@ pw_status_t pw_moe_create(const pw_moe_config_t* cfg, const pw_block_desc_t* blo
 
 pw_status_t pw_set_block_bits(pw_moe_t* h, int32_t block_id, int32_t new_bits,
                               pw_stream_t side_stream) {
+  const NvtxRange nvtx("pw_set_block_bits (page move)");
   if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
   if (block_id < 0 || block_id >= h->n_blocks)
     return fail(PW_ERR_INVALID_ARG, "block id %d out of range", block_id);
@@ -623,6 +646,7 @@ pw_status_t pw_set_switch_lag(pw_moe_t* h, int32_t max_lag) {
 static pw_status_t forward_impl(pw_moe_t* h, const uint16_t* d_x, int32_t T,
                                 const float* d_wr, const float* d_bias, uint16_t* d_y,
                                 cudaStream_t s) {
+  const NvtxRange nvtx("pw_moe_forward");
   const pw_moe_config_t& c = h->cfg;
   // pending page moves: one whose copy has already completed takes effect
   // now, without any wait; one that has stayed pending for max_lag forwards
@@ -1017,6 +1041,7 @@ pw_status_t pw_routing_stats(pw_moe_t* h, uint64_t* counts, double* mass, int32_
 }
 
 pw_status_t pw_enable_paging(pw_moe_t* h, pw_stream_t stream) {
+  const NvtxRange nvtx("pw_enable_paging");
   if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
   if (h->paging) return PW_OK;
   for (int i = 0; i < h->n_blocks; ++i) {
@@ -1069,6 +1094,7 @@ pw_status_t pw_enable_paging(pw_moe_t* h, pw_stream_t stream) {
 }
 
 pw_status_t pw_compact_pages(pw_moe_t* h, pw_stream_t stream) {
+  const NvtxRange nvtx("pw_compact_pages");
   if (!h) return fail(PW_ERR_INVALID_ARG, "null handle");
   if (!h->paging) return fail(PW_ERR_STATE, "paging is not enabled");
   for (int i = 0; i < h->n_blocks; ++i)
